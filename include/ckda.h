@@ -1,0 +1,139 @@
+/*
+ * ckda.h -- C ABI of the B200 (sm_100a) gated delta-rule library.
+ *
+ * The recurrence, per sequence and head, token t:
+ *
+ *   S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *   o_t = S_t^T q_t
+ *
+ * transition from "Complex KDA: Understanding and Enhancing the Expressivity of
+ * Kimi Delta Attention" (paper review page), section "Diagonal-plus-rank-one
+ * (DPR1) transition"; the write term is the gated delta rule (CyFA blog,
+ * section 2.2, with gate and strength); state S in R^{dk x dv}, row = key
+ * channel, read S^T q ("Dual DeltaNet" abstract).  There is no 1/sqrt(dk)
+ * scale: callers pre-scale q.
+ *
+ * Gate forms (signed_gate):
+ *   0  KDA   alpha = sigma(a) in (0,1)^dk,    beta = sigma(b) in (0,1)
+ *   1  CKDA  alpha = 2 sigma(a) - 1 in [-1,1], beta = 2 sigma(b) in [0,2]
+ *            (CKDA review, "Method steps", step 1: both ranges widen together)
+ *   2  raw   a holds alpha and b holds beta directly (tests and special cases)
+ * Logits of +-inf are legal and exact: alpha = 0, +-1 and beta = 0, 1, 2.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers, dense and row-major.  Alignment
+ *     (CKDA_ERR_ALIGN otherwise): states (S0, S_T, S) 16 bytes; b and
+ *     cu_seqlens 4 bytes; ckda_chunk_fwd's q, k, v, a, o 16 bytes;
+ *     ckda_decode_step's q, k, v, a, o their element size.  The caller allocates and
+ *     owns every buffer, workspace included; the library never allocates,
+ *     never frees and never synchronises.  Work is enqueued on `stream`
+ *     (a cudaStream_t; NULL = legacy default stream) and runs asynchronously:
+ *     a return of CKDA_OK means "validated and enqueued".
+ *   - io_dtype (q, k, v, a) and o_dtype (o) are CKDA_F32 or CKDA_BF16.
+ *     b is always float32; states are always float32.
+ *   - dk, dv in {16, 32, 64, 128}.
+ *   - Errors: a negative CKDA_ERR_* code, nothing enqueued, no output written.
+ *     No entry point aborts, throws or traps; device-side checks (offsets in
+ *     cu_seqlens, bounded waits) set a status word in the workspace that
+ *     ckda_workspace_status() reads back.
+ *   - NaN or Inf in q, k, v give undefined values but no fault.
+ */
+#ifndef CKDA_H
+#define CKDA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define CKDA_OK 0
+#define CKDA_ERR_NULL (-1)      /* a required pointer is NULL                      */
+#define CKDA_ERR_DIM (-2)       /* dk/dv not in {16,32,64,128}, or bad B/T/H/n_seqs */
+#define CKDA_ERR_CHUNK (-3)     /* chunk not in {16,32,64}                          */
+#define CKDA_ERR_DTYPE (-4)     /* io_dtype / o_dtype / signed_gate out of range    */
+#define CKDA_ERR_ALIGN (-5)     /* a pointer misaligned for its argument            */
+#define CKDA_ERR_SEQLENS (-6)   /* cu_seqlens offsets invalid (device-detected)     */
+#define CKDA_ERR_WORKSPACE (-7) /* workspace NULL or smaller than required          */
+#define CKDA_ERR_TIMEOUT (-8)   /* a bounded device wait gave up                    */
+#define CKDA_ERR_CUDA (-9)      /* a CUDA runtime call or kernel launch failed      */
+#define CKDA_ERR_DEVICE (-10)   /* current device is not sm_100 (B200 class)        */
+
+#define CKDA_F32 0
+#define CKDA_BF16 1
+
+/*
+ * Chunkwise (WY / UT-transform) parallel forward, "prefill".
+ *
+ * The CKDA review states that the DPR1 transition keeps WY chunk-wise
+ * parallel training (section "Diagonal-plus-rank-one (DPR1) transition");
+ * tokens are processed `chunk` at a time, the state is carried between
+ * chunks, and the result equals the token-by-token recurrence.
+ *
+ *   q, k, a : [B, T, H, dk]  io_dtype       v : [B, T, H, dv]  io_dtype
+ *   b       : [B, T, H]      float32        o : [B, T, H, dv]  o_dtype (NULL: not written)
+ *   S0      : [N, H, dk, dv] float32, NULL = zero initial state
+ *   S_T     : [N, H, dk, dv] float32, NULL = not written; may alias S0
+ *   cu_seqlens : NULL, or int32 [n_seqs + 1] device offsets into the T axis
+ *            (packed variable-length batch): B must be 1, N = n_seqs,
+ *            offsets must start at 0, be non-decreasing and end at T.
+ *            Without it N = B and every batch row is one sequence of T tokens.
+ *            Offsets are checked on the device: a bad sequence is skipped
+ *            and CKDA_ERR_SEQLENS is recorded in the workspace status word.
+ *   chunk   : 16, 32 or 64 tokens per chunk (a ragged last chunk is fine;
+ *            chunks never span two sequences).
+ *   workspace : device scratch of at least ckda_chunk_fwd_workspace_size()
+ *            bytes, 256-byte aligned; owned by the caller, reused freely
+ *            between calls on the same stream, never shared by two calls in
+ *            flight at once.
+ *   stream  : cudaStream_t.
+ * Returns CKDA_OK or a negative CKDA_ERR_* code.
+ */
+int ckda_chunk_fwd(const void *q, const void *k, const void *v, const void *a, const float *b,
+                   const float *S0, const int32_t *cu_seqlens, int n_seqs, int B, int T, int H,
+                   int dk, int dv, int chunk, int signed_gate, int io_dtype, int o_dtype,
+                   void *o, float *S_T, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Bytes of workspace ckda_chunk_fwd needs for these sizes (same meaning as
+ * there; n_seqs is ignored when the batch is not packed).  Pure host
+ * arithmetic, no CUDA call.
+ */
+size_t ckda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int chunk,
+                                     int n_seqs);
+
+/*
+ * One recurrent decode step for B x H heads: the recurrence above for a
+ * single token, applied to the state in place.  The CKDA review notes the
+ * extended ranges add no per-token inference cost (section "Research
+ * motivation"); the step reads and writes each head's fp32 state once.
+ *
+ *   q, k, a : [B, H, dk] io_dtype     v : [B, H, dv] io_dtype     b : [B, H] float32
+ *   S       : [B, H, dk, dv] float32, updated in place (S_{t-1} -> S_t)
+ *   o       : [B, H, dv] o_dtype, o = S_t^T q (NULL: not written)
+ * Returns CKDA_OK or a negative CKDA_ERR_* code.
+ */
+int ckda_decode_step(const void *q, const void *k, const void *v, const void *a, const float *b,
+                     float *S, int B, int H, int dk, int dv, int signed_gate, int io_dtype,
+                     int o_dtype, void *o, void *stream);
+
+/*
+ * Reads the device status word that ckda_chunk_fwd records in `workspace`
+ * (CKDA_OK, CKDA_ERR_SEQLENS or CKDA_ERR_TIMEOUT) into *status.  This call
+ * SYNCHRONISES `stream` (it copies 4 bytes to the host).  Returns CKDA_OK or
+ * CKDA_ERR_NULL / CKDA_ERR_CUDA.
+ */
+int ckda_workspace_status(const void *workspace, int *status, void *stream);
+
+/* Static, human-readable text for a status code (never NULL). */
+const char *ckda_status_string(int status);
+
+/* Library ABI version: major * 10000 + minor * 100 + patch. */
+int ckda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CKDA_H */

@@ -1,0 +1,134 @@
+// ckda_abi.cu -- host side of the C ABI declared in include/ckda.h:
+// argument validation, device check, workspace layout and kernel dispatch.
+// Nothing here allocates device memory or synchronises (except the explicit
+// status read-back, which says so).
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/ckda.h"
+#include "internal.h"
+
+namespace {
+
+bool valid_dim(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+bool aligned(const void *p, uintptr_t n) {
+  return p == nullptr || (reinterpret_cast<uintptr_t>(p) & (n - 1)) == 0;
+}
+bool aligned16(const void *p) { return aligned(p, 16); }
+
+// sm_100 check for the current device, cached per device.
+int check_device() {
+  static int cached[64];  // 0 unknown, 1 ok, -1 not sm_100
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return CKDA_ERR_CUDA;
+  if (dev >= 0 && dev < 64 && cached[dev] != 0) return cached[dev] > 0 ? CKDA_OK : CKDA_ERR_DEVICE;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return CKDA_ERR_CUDA;
+  const bool ok = (major == 10 && minor == 0);
+  if (dev >= 0 && dev < 64) cached[dev] = ok ? 1 : -1;
+  return ok ? CKDA_OK : CKDA_ERR_DEVICE;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *ckda_status_string(int status) {
+  switch (status) {
+    case CKDA_OK: return "ok";
+    case CKDA_ERR_NULL: return "a required pointer is NULL";
+    case CKDA_ERR_DIM: return "unsupported dimension (dk, dv must be 16, 32, 64 or 128; B, T, H, n_seqs valid)";
+    case CKDA_ERR_CHUNK: return "unsupported chunk size (16, 32 or 64)";
+    case CKDA_ERR_DTYPE: return "unsupported dtype code or signed_gate value";
+    case CKDA_ERR_ALIGN: return "a pointer is not aligned as its argument requires";
+    case CKDA_ERR_SEQLENS: return "invalid cu_seqlens offsets";
+    case CKDA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case CKDA_ERR_TIMEOUT: return "a bounded device wait timed out";
+    case CKDA_ERR_CUDA: return "CUDA runtime error";
+    case CKDA_ERR_DEVICE: return "current device is not an sm_100 (B200-class) GPU";
+  }
+  return "unknown status";
+}
+
+int ckda_version(void) { return 100; }
+
+size_t ckda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int chunk, int n_seqs) {
+  (void)B; (void)T; (void)H; (void)dk; (void)dv; (void)chunk; (void)n_seqs;
+  return ckda::kWorkspaceHeader;
+}
+
+int ckda_chunk_fwd(const void *q, const void *k, const void *v, const void *a, const float *b,
+                   const float *S0, const int32_t *cu_seqlens, int n_seqs, int B, int T, int H,
+                   int dk, int dv, int chunk, int signed_gate, int io_dtype, int o_dtype,
+                   void *o, float *S_T, void *workspace, size_t workspace_bytes, void *stream) {
+  if (!q || !k || !v || !a || !b) return CKDA_ERR_NULL;
+  if (!valid_dim(dk) || !valid_dim(dv) || B < 0 || T < 0 || H <= 0) return CKDA_ERR_DIM;
+  if (chunk != 16 && chunk != 32 && chunk != 64) return CKDA_ERR_CHUNK;
+  if (signed_gate < 0 || signed_gate > 2 || (io_dtype != CKDA_F32 && io_dtype != CKDA_BF16) ||
+      (o_dtype != CKDA_F32 && o_dtype != CKDA_BF16))
+    return CKDA_ERR_DTYPE;
+  int N = B;
+  if (cu_seqlens) {
+    if (B != 1 || n_seqs < 0) return CKDA_ERR_DIM;
+    N = n_seqs;
+  }
+  if ((long long)B * T * H > (1LL << 40)) return CKDA_ERR_DIM;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(a) || !aligned(b, 4) ||
+      !aligned16(S0) || !aligned16(o) || !aligned16(S_T) || !aligned(cu_seqlens, 4))
+    return CKDA_ERR_ALIGN;
+  const size_t need = ckda_chunk_fwd_workspace_size(B, T, H, dk, dv, chunk, n_seqs);
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return CKDA_ERR_WORKSPACE;
+  const int dev_rc = check_device();
+  if (dev_rc != CKDA_OK) return dev_rc;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(workspace, 0, ckda::kWorkspaceHeader, s) != cudaSuccess) return CKDA_ERR_CUDA;
+  ckda::ChunkArgs g;
+  g.q = q; g.k = k; g.v = v; g.a = a; g.b = b; g.S0 = S0; g.cu_seqlens = cu_seqlens;
+  g.o = o; g.S_T = S_T; g.n_seqs = N; g.B = B; g.T = T; g.H = H; g.dk = dk; g.dv = dv;
+  g.chunk = chunk; g.signed_gate = signed_gate; g.io_dtype = io_dtype; g.o_dtype = o_dtype;
+  g.status = static_cast<int *>(workspace);
+  g.workspace = workspace;
+  g.workspace_bytes = workspace_bytes;
+  return ckda::launch_chunk_simt(g, s);
+}
+
+int ckda_decode_step(const void *q, const void *k, const void *v, const void *a, const float *b,
+                     float *S, int B, int H, int dk, int dv, int signed_gate, int io_dtype,
+                     int o_dtype, void *o, void *stream) {
+  if (!q || !k || !v || !a || !b || !S) return CKDA_ERR_NULL;
+  if (!valid_dim(dk) || !valid_dim(dv) || B < 0 || H <= 0) return CKDA_ERR_DIM;
+  if ((long long)B * H > (1LL << 31) - 1) return CKDA_ERR_DIM;
+  if (signed_gate < 0 || signed_gate > 2 || (io_dtype != CKDA_F32 && io_dtype != CKDA_BF16) ||
+      (o_dtype != CKDA_F32 && o_dtype != CKDA_BF16))
+    return CKDA_ERR_DTYPE;
+  const uintptr_t in_sz = io_dtype == CKDA_BF16 ? 2 : 4, out_sz = o_dtype == CKDA_BF16 ? 2 : 4;
+  if (!aligned(q, in_sz) || !aligned(k, in_sz) || !aligned(v, in_sz) || !aligned(a, in_sz) ||
+      !aligned(b, 4) || !aligned16(S) || !aligned(o, out_sz))
+    return CKDA_ERR_ALIGN;
+  const int dev_rc = check_device();
+  if (dev_rc != CKDA_OK) return dev_rc;
+  ckda::DecodeArgs g;
+  g.q = q; g.k = k; g.v = v; g.a = a; g.b = b; g.S = S; g.o = o;
+  g.B = B; g.H = H; g.dk = dk; g.dv = dv; g.signed_gate = signed_gate;
+  g.io_dtype = io_dtype; g.o_dtype = o_dtype;
+  return ckda::launch_decode(g, static_cast<cudaStream_t>(stream));
+}
+
+int ckda_workspace_status(const void *workspace, int *status, void *stream) {
+  if (!workspace || !status) return CKDA_ERR_NULL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int host = 0;
+  if (cudaMemcpyAsync(&host, workspace, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return CKDA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return CKDA_ERR_CUDA;
+  *status = host;
+  return CKDA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,77 @@
+// common.cuh -- device helpers shared by the sm_100a kernels of this library.
+//
+// Gate activation (CKDA review, "Method steps", step 1):
+//   KDA   alpha = sigma(a),        beta = sigma(b)
+//   CKDA  alpha = 2 sigma(a) - 1,  beta = 2 sigma(b)
+//   raw   alpha = a,               beta = b
+// Accurate libdevice functions (expf, expm1f, log1pf, logf, tanhf) are used:
+// this file is compiled without fast-math.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/ckda.h"
+
+namespace ckda {
+
+constexpr float kLn2 = 0.693147180559945309f;
+constexpr float kInvLn2 = 1.442695040888963407f;
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T>
+__device__ __forceinline__ T from_f32(float x);
+template <>
+__device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// Linear gate value alpha (decode path).  Exact at +-inf: KDA 1/0, CKDA +-1.
+__device__ __forceinline__ float gate_alpha(float a, int signed_gate) {
+  if (signed_gate == 0) return 1.0f / (1.0f + expf(-a));
+  if (signed_gate == 1) return tanhf(0.5f * a);  // 2 sigma(a) - 1 == tanh(a/2)
+  return a;
+}
+
+// Strength beta.  Exact at +-inf: KDA 1/0, CKDA 2/0.
+__device__ __forceinline__ float gate_beta(float b, int signed_gate) {
+  if (signed_gate == 0) return 1.0f / (1.0f + expf(-b));
+  if (signed_gate == 1) return 2.0f / (1.0f + expf(-b));
+  return b;
+}
+
+// Log-space gate: log2|alpha| (finite unless is_zero), sign bit, exact-zero flag.
+//   KDA : log sigma(a) = -softplus(-a);       zero iff a == -inf
+//   CKDA: log |tanh(a/2)| = log(-expm1(-|a|)) - log1p(exp(-|a|));  zero iff a == 0
+//   raw : log |a|;                            zero iff a == 0
+__device__ __forceinline__ void gate_log2(float a, int signed_gate, float &log2abs, bool &is_zero,
+                                          bool &is_neg) {
+  if (signed_gate == 0) {
+    is_neg = false;
+    is_zero = (a == -INFINITY);
+    const float x = -a;  // softplus(x) = max(x, 0) + log1p(exp(-|x|))
+    const float sp = fmaxf(x, 0.0f) + log1pf(expf(-fabsf(x)));
+    log2abs = is_zero ? 0.0f : -sp * kInvLn2;
+  } else if (signed_gate == 1) {
+    is_neg = (a < 0.0f);
+    is_zero = (a == 0.0f);
+    const float x = fabsf(a);
+    log2abs = is_zero ? 0.0f : (logf(-expm1f(-x)) - log1pf(expf(-x))) * kInvLn2;
+  } else {
+    is_neg = (a < 0.0f);
+    is_zero = (a == 0.0f);
+    log2abs = is_zero ? 0.0f : log2f(fabsf(a));
+  }
+}
+
+// Records the first device-detected error in the workspace status word.
+__device__ __forceinline__ void set_status(int *status, int code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+}  // namespace ckda

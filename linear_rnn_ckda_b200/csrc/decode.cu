@@ -1,0 +1,158 @@
+// decode.cu -- one recurrent decode step on sm_100a (HBM-bound).
+//
+// Per head:  S' = Diag(alpha) S;  p = S'^T k;  S = S' + beta k (v - p)^T;  o = S^T q
+// which is S_t = (I - beta k k^T) Diag(alpha) S_{t-1} + beta k v^T, o_t = S_t^T q_t
+// (CKDA review, section "Diagonal-plus-rank-one (DPR1) transition"; the
+// review notes the extended ranges add no per-token inference cost).
+//
+// Each head's fp32 state [dk][dv] is read once and written once, in 16-byte
+// vectors.  A warp owns 16 state columns: lane l holds columns
+// 16*w + 4*(l%4) .. +3 for rows l/4 + 8*m (m = 0 .. dk/8-1), so one warp load
+// instruction covers 8 rows x 64 contiguous bytes, and the reductions over the
+// key channel (k . S' and q . S) are in-thread sums followed by three xor
+// shuffles across the 8 lanes that share a column group.  No shared-memory
+// reduction and no block barrier touch the state.
+#include "common.cuh"
+#include "internal.h"
+
+namespace ckda {
+namespace {
+
+constexpr int kDecodeThreads = 256;
+
+template <int DK, int DV, typename TIn, typename TOut>
+__global__ void __launch_bounds__(kDecodeThreads)
+    decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
+                  const TIn *__restrict__ a, const float *__restrict__ b, float *__restrict__ S,
+                  TOut *__restrict__ o, int n_heads, int signed_gate) {
+  constexpr int kWarpsPerHead = DV / 16;
+  constexpr int kHeadsPerBlock = (kDecodeThreads / 32) / kWarpsPerHead;
+  constexpr int kRows = DK / 8;  // state rows per thread
+  __shared__ float s_q[kHeadsPerBlock][DK];
+  __shared__ float s_k[kHeadsPerBlock][DK];
+  __shared__ float s_al[kHeadsPerBlock][DK];
+  __shared__ float s_beta[kHeadsPerBlock];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int hl = warp / kWarpsPerHead;
+  const int head = blockIdx.x * kHeadsPerBlock + hl;
+  const int gtid = threadIdx.x - hl * kWarpsPerHead * 32;  // thread index within the head group
+
+  // Stage q, k and the activated gate for this head group.
+  if (head < n_heads) {
+    for (int i = gtid; i < DK; i += kWarpsPerHead * 32) {
+      const size_t e = (size_t)head * DK + i;
+      s_q[hl][i] = to_f32(q[e]);
+      s_k[hl][i] = to_f32(k[e]);
+      s_al[hl][i] = gate_alpha(to_f32(a[e]), signed_gate);
+    }
+    if (gtid == 0) s_beta[hl] = gate_beta(b[head], signed_gate);
+  }
+  __syncthreads();
+  if (head >= n_heads) return;
+
+  const int cq = lane & 3, r0 = lane >> 2;
+  const int col = (warp % kWarpsPerHead) * 16 + cq * 4;
+  float *Sh = S + (size_t)head * DK * DV;
+
+  float4 st[kRows];
+#pragma unroll
+  for (int m = 0; m < kRows; ++m)
+    st[m] = *reinterpret_cast<const float4 *>(Sh + (size_t)(r0 + 8 * m) * DV + col);
+
+  // S' = Diag(alpha) S and p = S'^T k (partial over this thread's rows)
+  float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+#pragma unroll
+  for (int m = 0; m < kRows; ++m) {
+    const int i = r0 + 8 * m;
+    const float al = s_al[hl][i], ki = s_k[hl][i];
+    st[m].x *= al; st[m].y *= al; st[m].z *= al; st[m].w *= al;
+    p0 = fmaf(ki, st[m].x, p0); p1 = fmaf(ki, st[m].y, p1);
+    p2 = fmaf(ki, st[m].z, p2); p3 = fmaf(ki, st[m].w, p3);
+  }
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    p0 += __shfl_xor_sync(0xffffffffu, p0, off);
+    p1 += __shfl_xor_sync(0xffffffffu, p1, off);
+    p2 += __shfl_xor_sync(0xffffffffu, p2, off);
+    p3 += __shfl_xor_sync(0xffffffffu, p3, off);
+  }
+
+  // u = beta (v - p)
+  const float beta = s_beta[hl];
+  const TIn *vh = v + (size_t)head * DV + col;
+  const float u0 = beta * (to_f32(vh[0]) - p0), u1 = beta * (to_f32(vh[1]) - p1);
+  const float u2 = beta * (to_f32(vh[2]) - p2), u3 = beta * (to_f32(vh[3]) - p3);
+
+  // S = S' + k u^T, written back; o = S^T q
+  float r0s = 0.f, r1s = 0.f, r2s = 0.f, r3s = 0.f;
+#pragma unroll
+  for (int m = 0; m < kRows; ++m) {
+    const int i = r0 + 8 * m;
+    const float ki = s_k[hl][i], qi = s_q[hl][i];
+    st[m].x = fmaf(ki, u0, st[m].x); st[m].y = fmaf(ki, u1, st[m].y);
+    st[m].z = fmaf(ki, u2, st[m].z); st[m].w = fmaf(ki, u3, st[m].w);
+    *reinterpret_cast<float4 *>(Sh + (size_t)i * DV + col) = st[m];
+    r0s = fmaf(qi, st[m].x, r0s); r1s = fmaf(qi, st[m].y, r1s);
+    r2s = fmaf(qi, st[m].z, r2s); r3s = fmaf(qi, st[m].w, r3s);
+  }
+  if (o == nullptr) return;
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    r0s += __shfl_xor_sync(0xffffffffu, r0s, off);
+    r1s += __shfl_xor_sync(0xffffffffu, r1s, off);
+    r2s += __shfl_xor_sync(0xffffffffu, r2s, off);
+    r3s += __shfl_xor_sync(0xffffffffu, r3s, off);
+  }
+  if (r0 == 0) {
+    TOut *oh = o + (size_t)head * DV + col;
+    oh[0] = from_f32<TOut>(r0s); oh[1] = from_f32<TOut>(r1s);
+    oh[2] = from_f32<TOut>(r2s); oh[3] = from_f32<TOut>(r3s);
+  }
+}
+
+template <int DK, int DV, typename TIn, typename TOut>
+int launch_typed(const DecodeArgs &g, cudaStream_t stream) {
+  const int n_heads = g.B * g.H;
+  constexpr int kHeadsPerBlock = (kDecodeThreads / 32) / (DV / 16);
+  const int blocks = (n_heads + kHeadsPerBlock - 1) / kHeadsPerBlock;
+  decode_kernel<DK, DV, TIn, TOut><<<blocks, kDecodeThreads, 0, stream>>>(
+      static_cast<const TIn *>(g.q), static_cast<const TIn *>(g.k), static_cast<const TIn *>(g.v),
+      static_cast<const TIn *>(g.a), g.b, g.S, static_cast<TOut *>(g.o), n_heads, g.signed_gate);
+  return cudaGetLastError() == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
+}
+
+template <int DK, int DV>
+int launch_dims(const DecodeArgs &g, cudaStream_t s) {
+  const bool in_bf = g.io_dtype == CKDA_BF16, out_bf = g.o_dtype == CKDA_BF16;
+  if (in_bf && out_bf) return launch_typed<DK, DV, __nv_bfloat16, __nv_bfloat16>(g, s);
+  if (in_bf) return launch_typed<DK, DV, __nv_bfloat16, float>(g, s);
+  if (out_bf) return launch_typed<DK, DV, float, __nv_bfloat16>(g, s);
+  return launch_typed<DK, DV, float, float>(g, s);
+}
+
+template <int DK>
+int launch_dv(const DecodeArgs &g, cudaStream_t s) {
+  switch (g.dv) {
+    case 16: return launch_dims<DK, 16>(g, s);
+    case 32: return launch_dims<DK, 32>(g, s);
+    case 64: return launch_dims<DK, 64>(g, s);
+    case 128: return launch_dims<DK, 128>(g, s);
+  }
+  return CKDA_ERR_DIM;
+}
+
+}  // namespace
+
+int launch_decode(const DecodeArgs &g, cudaStream_t s) {
+  if (g.B * g.H == 0) return CKDA_OK;
+  switch (g.dk) {
+    case 16: return launch_dv<16>(g, s);
+    case 32: return launch_dv<32>(g, s);
+    case 64: return launch_dv<64>(g, s);
+    case 128: return launch_dv<128>(g, s);
+  }
+  return CKDA_ERR_DIM;
+}
+
+}  // namespace ckda

@@ -1,0 +1,41 @@
+// internal.h -- launch interface between the C ABI (ckda_abi.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace ckda {
+
+struct ChunkArgs {
+  const void *q, *k, *v, *a;
+  const float *b;
+  const float *S0;
+  const int32_t *cu_seqlens;  // device, or NULL
+  void *o;                    // may be NULL
+  float *S_T;                 // may be NULL
+  int n_seqs;                 // N (sequences)
+  int B, T, H, dk, dv, chunk, signed_gate, io_dtype, o_dtype;
+  int *status;                // device status word (workspace)
+  void *workspace;            // whole workspace (status word first)
+  size_t workspace_bytes;
+};
+
+struct DecodeArgs {
+  const void *q, *k, *v, *a;
+  const float *b;
+  float *S;
+  void *o;
+  int B, H, dk, dv, signed_gate, io_dtype, o_dtype;
+};
+
+// Exact fp32 SIMT chunkwise forward (any dk, dv, chunk).  Returns a CKDA_* code.
+int launch_chunk_simt(const ChunkArgs &args, cudaStream_t stream);
+
+// One decode step.  Returns a CKDA_* code.
+int launch_decode(const DecodeArgs &args, cudaStream_t stream);
+
+// Bytes of the workspace header (status word and counters).
+constexpr size_t kWorkspaceHeader = 256;
+
+}  // namespace ckda

@@ -1,0 +1,149 @@
+"""Python binding of ``libckda.so`` (the C ABI in ``include/ckda.h``).
+
+Argument marshalling only: torch tensors supply device memory and the current
+CUDA stream; every step of the recurrence runs in the library's kernels.
+There is no CPU fallback: if the library is missing or the tensors are not on
+a CUDA device, these functions raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libckda.so")
+_lock = threading.Lock()
+_lib = None
+
+CKDA_F32 = 0
+CKDA_BF16 = 1
+_DT = {torch.float32: CKDA_F32, torch.bfloat16: CKDA_BF16}
+_TORCH_DT = {CKDA_F32: torch.float32, CKDA_BF16: torch.bfloat16}
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+
+# name -> (restype, argtypes), mirroring include/ckda.h
+SIGNATURES = {
+    "ckda_chunk_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i,
+                            _i, _i, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
+    "ckda_chunk_fwd_workspace_size": (ctypes.c_size_t, [_i, _i, _i, _i, _i, _i, _i]),
+    "ckda_decode_step": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp]),
+    "ckda_workspace_status": (_i, [_vp, ctypes.POINTER(_i), _vp]),
+    "ckda_status_string": (ctypes.c_char_p, [_i]),
+    "ckda_version": (_i, []),
+}
+
+
+class CkdaError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} failed: {status_string(code)} (code {code})")
+        self.code = code
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load():
+    """Loads ``libckda.so`` (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(_LIB_PATH):
+                raise RuntimeError(
+                    f"{_LIB_PATH} is missing: build it with `python -m linear_rnn_ckda_b200.build` "
+                    "(there is no CPU fallback)")
+            lib = ctypes.CDLL(_LIB_PATH)
+            for name, (res, args) in SIGNATURES.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = lib
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return load().ckda_status_string(int(code)).decode()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def workspace_size(B, T, H, dk, dv, chunk, n_seqs=0) -> int:
+    return int(load().ckda_chunk_fwd_workspace_size(B, T, H, dk, dv, chunk, n_seqs))
+
+
+def new_workspace(B, T, H, dk, dv, chunk, n_seqs=0, device=None) -> torch.Tensor:
+    n = workspace_size(B, T, H, dk, dv, chunk, n_seqs)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def chunk_fwd(q, k, v, a, b, S0=None, cu_seqlens=None, chunk: int = 64, signed_gate: int = 1,
+              o_dtype=None, o=None, S_T=None, workspace=None, want_o: bool = True,
+              want_state: bool = True):
+    """Chunkwise forward.  Returns (o, S_T) (either may be None when not wanted).
+
+    q, k, a: [B,T,H,dk]; v: [B,T,H,dv] (fp32 or bf16, same dtype); b: [B,T,H] fp32;
+    S0: [N,H,dk,dv] fp32 or None; cu_seqlens: int32 CUDA tensor [N+1] or None.
+    """
+    lib = load()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    io = _DT[q.dtype]
+    od = io if o_dtype is None else _DT[o_dtype]
+    N = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    dev = q.device
+    if want_o and o is None:
+        o = torch.empty((B, T, H, dv), dtype=_TORCH_DT[od], device=dev)
+    if want_state and S_T is None:
+        S_T = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = new_workspace(B, T, H, dk, dv, chunk, N, dev)
+    rc = lib.ckda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(S0),
+                            _ptr(cu_seqlens), N if cu_seqlens is not None else 0, B, T, H, dk, dv,
+                            chunk, signed_gate, io, od, _ptr(o if want_o else None),
+                            _ptr(S_T if want_state else None), _ptr(workspace),
+                            workspace.numel(), _stream(dev))
+    if rc != 0:
+        raise CkdaError("ckda_chunk_fwd", rc)
+    return (o if want_o else None), (S_T if want_state else None)
+
+
+def decode_step(q, k, v, a, b, S, signed_gate: int = 1, o_dtype=None, o=None, want_o=True):
+    """One decode step; S [B,H,dk,dv] fp32 is updated in place.  Returns o [B,H,dv]."""
+    lib = load()
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    io = _DT[q.dtype]
+    od = io if o_dtype is None else _DT[o_dtype]
+    if want_o and o is None:
+        o = torch.empty((B, H, dv), dtype=_TORCH_DT[od], device=q.device)
+    rc = lib.ckda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(S), B, H, dk, dv,
+                              signed_gate, io, od, _ptr(o if want_o else None), _stream(q.device))
+    if rc != 0:
+        raise CkdaError("ckda_decode_step", rc)
+    return o if want_o else None
+
+
+def workspace_status(workspace: torch.Tensor) -> int:
+    """Device status word of the last chunk_fwd that used ``workspace`` (synchronises)."""
+    st = ctypes.c_int(0)
+    rc = load().ckda_workspace_status(_ptr(workspace), ctypes.byref(st), _stream(workspace.device))
+    if rc != 0:
+        raise CkdaError("ckda_workspace_status", rc)
+    return st.value

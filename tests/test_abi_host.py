@@ -1,0 +1,123 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every function ``include/ckda.h`` declares, and rejects bad arguments with the
+documented codes before touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ckda.h")
+
+from linear_rnn_ckda_b200 import build as lib_build  # noqa: E402
+from linear_rnn_ckda_b200 import ops  # noqa: E402
+
+
+@pytest.fixture(scope="module")
+def lib():
+    lib_build.build_library()
+    return ops.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ckda_\w+)\s*\(", text)))
+
+
+def declared_codes():
+    text = open(HEADER).read()
+    return {m[0]: int(m[1]) for m in re.findall(r"#define (CKDA_\w+) \(?(-?\d+)\)?", text)}
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    for n in ("ckda_chunk_fwd", "ckda_chunk_fwd_workspace_size", "ckda_decode_step",
+              "ckda_status_string", "ckda_workspace_status", "ckda_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in ckda.h but not exported"
+        assert name in ops.SIGNATURES, f"{name} has no binding signature"
+
+
+def test_binding_codes_match_header():
+    codes = declared_codes()
+    assert codes["CKDA_F32"] == ops.CKDA_F32 and codes["CKDA_BF16"] == ops.CKDA_BF16
+
+
+def test_status_strings(lib):
+    codes = declared_codes()
+    for name, code in codes.items():
+        if name.startswith("CKDA_ERR") or name == "CKDA_OK":
+            s = lib.ckda_status_string(code).decode()
+            assert s and s != "unknown status", name
+    assert lib.ckda_status_string(12345).decode() == "unknown status"
+    assert lib.ckda_version() >= 100
+
+
+def test_workspace_size(lib):
+    assert lib.ckda_chunk_fwd_workspace_size(4, 4096, 16, 128, 128, 64, 0) >= 256
+    assert lib.ckda_chunk_fwd_workspace_size(1, 0, 1, 16, 16, 16, 0) >= 256
+
+
+# Fake, aligned, never-dereferenced host addresses: every call below has exactly
+# one invalid argument, so validation rejects it before any CUDA call.
+P = ctypes.c_void_p(1 << 20)
+MIS = ctypes.c_void_p((1 << 20) + 4)     # 4-byte aligned, not 16
+ODD = ctypes.c_void_p((1 << 20) + 2)     # 2-byte aligned only
+
+
+def _fwd(lib, **kw):
+    args = dict(q=P, k=P, v=P, a=P, b=P, S0=None, cu=None, n_seqs=0, B=1, T=8, H=1, dk=16, dv=16,
+                chunk=16, sg=1, io=0, od=0, o=P, S_T=P, ws=P, wsb=256, stream=None)
+    args.update(kw)
+    return lib.ckda_chunk_fwd(*args.values())
+
+
+def _dec(lib, **kw):
+    args = dict(q=P, k=P, v=P, a=P, b=P, S=P, B=1, H=1, dk=16, dv=16, sg=1, io=0, od=0, o=P,
+                stream=None)
+    args.update(kw)
+    return lib.ckda_decode_step(*args.values())
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), -1), (dict(b=None), -1),
+    (dict(dk=24), -2), (dict(dv=256), -2), (dict(H=0), -2), (dict(T=-1), -2), (dict(B=-1), -2),
+    (dict(cu=P, B=2, n_seqs=1), -2),
+    (dict(chunk=128), -3), (dict(chunk=8), -3),
+    (dict(sg=3), -4), (dict(io=2), -4), (dict(od=-1), -4),
+    (dict(k=MIS), -5), (dict(o=MIS), -5), (dict(S0=MIS), -5), (dict(S_T=MIS), -5),
+    (dict(b=ODD), -5), (dict(cu=ODD), -5),
+    (dict(ws=None), -7), (dict(wsb=16), -7), (dict(ws=ctypes.c_void_p((1 << 20) + 16)), -7),
+])
+def test_chunk_fwd_rejects(lib, kw, code):
+    assert _fwd(lib, **kw) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(S=None), -1), (dict(q=None), -1), (dict(dk=48), -2), (dict(H=0), -2),
+    (dict(sg=-1), -4), (dict(io=5), -4), (dict(v=ODD), -5), (dict(q=ODD), -5), (dict(S=MIS), -5),
+    (dict(b=ODD), -5), (dict(io=1, od=0, o=ODD), -5),
+])
+def test_decode_rejects(lib, kw, code):
+    assert _dec(lib, **kw) == code
+
+
+def test_workspace_status_rejects_null(lib):
+    st = ctypes.c_int(0)
+    assert lib.ckda_workspace_status(None, ctypes.byref(st), None) == -1
+
+
+def test_binding_has_no_cpu_fallback(lib):
+    x = torch.zeros(1, 8, 1, 16)
+    with pytest.raises(ValueError):
+        ops.chunk_fwd(x, x, x, x, torch.zeros(1, 8, 1), chunk=16)
+    with pytest.raises(ValueError):
+        ops.decode_step(x[:, 0], x[:, 0], x[:, 0], x[:, 0], torch.zeros(1, 1),
+                        torch.zeros(1, 1, 16, 16))

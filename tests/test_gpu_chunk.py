@@ -1,0 +1,225 @@
+"""Parity of the chunkwise forward (``ckda_chunk_fwd`` through the C ABI)
+against the fp64 oracle on the same seeded inputs."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from helpers import (TOL_BF16, TOL_FP32, bf16_round, f64, oracle_prefill, oracle_units, rel,
+                     to_device, unit_rows)
+from linear_rnn_ckda_b200 import synth
+
+pytestmark = pytest.mark.gpu
+INF = float("inf")
+
+
+def run_gpu(ops, inp, w, chunk=None, o_dtype=None, S0_alias=False):
+    d = to_device(inp)
+    S_T = None
+    if S0_alias and d["S0"] is not None:
+        S_T = d["S0"]
+    o, S = ops.chunk_fwd(d["q"], d["k"], d["v"], d["a"], d["b"], d["S0"], d["cu_seqlens"],
+                         chunk=chunk or w.chunk, signed_gate=w.signed_gate,
+                         o_dtype=o_dtype, S_T=S_T)
+    torch.cuda.synchronize()
+    return o, S
+
+
+def check(ops, w, seed=0, tol=None, chunk=None, o_dtype=None):
+    inp = synth.make_prefill(w, seed)
+    o, S = run_gpu(ops, inp, w, chunk, o_dtype)
+    ro, rS = oracle_prefill(inp, w.signed_gate)
+    if o.dtype == torch.bfloat16:
+        ro = bf16_round(ro)
+    tol = tol or (TOL_FP32 if w.io_dtype == "f32" and o.dtype == torch.float32 else TOL_BF16)
+    eo, es = rel(f64(o), ro), rel(f64(S), rS)
+    assert eo <= tol and es <= tol, (w.name, eo, es, tol)
+    return eo, es
+
+
+def test_tiny_ckda_fp32(cuda_lib):
+    """The tiny CKDA workload: B=1, H=1, T=64, d=16, fp32, chunk 16, seed 0."""
+    check(cuda_lib, synth.TINY_CKDA_FP32)
+
+
+@pytest.mark.parametrize("dk,dv", [(16, 16), (16, 64), (32, 32), (64, 16), (64, 128), (128, 32),
+                                   (128, 128)])
+@pytest.mark.parametrize("chunk", [16, 32, 64])
+def test_dims_and_chunks_fp32(cuda_lib, dk, dv, chunk):
+    w = synth.TINY_CKDA_FP32.with_(name="dims", B=2, T=77, H=3, dk=dk, dv=dv, chunk=chunk, s0=True,
+                                   gate="spread", strength="spread")
+    check(cuda_lib, w, seed=1)
+
+
+@pytest.mark.parametrize("base", [synth.KDA_STD, synth.CKDA_SPREAD], ids=["kda_std", "ckda_spread"])
+@pytest.mark.parametrize("o_dtype", [torch.float32, torch.bfloat16], ids=["o_f32", "o_bf16"])
+def test_bf16_small(cuda_lib, base, o_dtype):
+    """Same distributions as the full workloads on a smaller grid (several chunks, ragged tail)."""
+    w = base.with_(B=2, T=300, H=3)
+    check(cuda_lib, w, seed=2, o_dtype=o_dtype)
+
+
+def test_fp32_io_d128(cuda_lib):
+    w = synth.CKDA_SPREAD.with_(B=1, T=200, H=2, io_dtype="f32", o_dtype="f32")
+    check(cuda_lib, w, seed=3, tol=TOL_FP32)
+
+
+def test_varlen_edge_lengths(cuda_lib):
+    """Packed batch with empty, length-1, ragged and chunk-multiple sequences."""
+    lens = (0, 1, 63, 64, 65, 200, 0, 129)
+    w = synth.CKDA_SPREAD.with_(B=1, H=2, seq_lens=lens, T=sum(lens), io_dtype="f32",
+                                o_dtype="f32")
+    inp = synth.make_prefill(w, seed=4)
+    o, S = run_gpu(cuda_lib, inp, w)
+    ro, rS = oracle_prefill(inp, w.signed_gate)
+    assert rel(f64(o), ro) <= TOL_FP32
+    assert rel(f64(S), rS) <= TOL_FP32
+    S0 = f64(inp["S0"])
+    assert np.array_equal(f64(S)[0], S0[0]) and np.array_equal(f64(S)[6], S0[6])
+
+
+def _raw_case(T, dk, dv, alpha, beta, seed=0, H=1):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((1, T, H, dk))
+    k = rng.standard_normal((1, T, H, dk))
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((1, T, H, dv))
+    S0 = rng.standard_normal((1, H, dk, dv)) * 0.1
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x)).float()
+    return {"q": t(q), "k": t(k), "v": t(v), "a": t(alpha), "b": t(beta), "S0": t(S0),
+            "cu_seqlens": None}
+
+
+@pytest.mark.parametrize("chunk", [16, 64])
+def test_degenerate_gates(cuda_lib, chunk):
+    """Exact zeros, +-1, strong decay and beta at 0 and 2 (raw gates), and the
+    same through +-inf logits in both gate forms."""
+    rng = np.random.default_rng(5)
+    T, dk, dv = 150, 32, 32
+    alpha = rng.uniform(-1, 1, (1, T, 1, dk))
+    alpha[0, 10, 0, :] = 0.0            # a full state wipe
+    alpha[0, 20:30, 0, 3] = 0.0         # one channel held at zero
+    alpha[0, 40:60, 0, 5] = -1.0
+    alpha[0, 70:90, 0, :8] = 1e-4       # strong decay (products underflow fp32)
+    alpha[0, 100:, 0, 9] = 1.0
+    beta = rng.uniform(0, 2, (1, T, 1))
+    beta[0, 5] = 0.0
+    beta[0, 6:9] = 2.0
+    inp = _raw_case(T, dk, dv, alpha, beta)
+    w = synth.TINY_CKDA_FP32.with_(B=1, T=T, H=1, dk=dk, dv=dv, chunk=chunk, signed_gate=2)
+    o, S = run_gpu(cuda_lib, inp, w)
+    ro, rS = oracle_prefill(inp, 2)
+    assert rel(f64(o), ro) <= TOL_FP32 and rel(f64(S), rS) <= TOL_FP32
+    # logits at +-inf and 0 in the CKDA and KDA forms
+    for sg in (0, 1):
+        a = rng.standard_normal((1, T, 1, dk)) * 3
+        a[0, 3, 0, :4] = INF
+        a[0, 4, 0, :4] = -INF
+        a[0, 7, 0, 4:8] = 0.0
+        b = rng.standard_normal((1, T, 1))
+        b[0, 11], b[0, 12] = INF, -INF
+        inp = _raw_case(T, dk, dv, a, b, seed=6)
+        o, S = run_gpu(cuda_lib, inp, w.with_(signed_gate=sg))
+        ro, rS = oracle_prefill(inp, sg)
+        assert rel(f64(o), ro) <= TOL_FP32 and rel(f64(S), rS) <= TOL_FP32
+
+
+def test_exact_rotation_on_gpu(cuda_lib):
+    """alpha = (-1, 1), beta = 2 (logits -inf/+inf/+inf), k = (cos t, sin t) in a 16-dim
+    head (other channels alpha = 1, k = 0): the top-left 2x2 block of the state
+    is rotated by 2 * sum(t) and the rest is unchanged."""
+    T, dk, dv, m = 48, 16, 16, 5
+    rng = np.random.default_rng(7)
+    x = rng.integers(0, m, size=T)
+    th = np.pi * x / m
+    k = np.zeros((1, T, 1, dk))
+    k[0, :, 0, 0], k[0, :, 0, 1] = np.cos(th), np.sin(th)
+    a = np.full((1, T, 1, dk), INF)
+    a[0, :, 0, 0] = -INF
+    inp = {"q": torch.zeros(1, T, 1, dk), "k": torch.from_numpy(k).float(),
+           "v": torch.zeros(1, T, 1, dv), "a": torch.from_numpy(a).float(),
+           "b": torch.full((1, T, 1), INF), "S0": torch.eye(dk).reshape(1, 1, dk, dv).contiguous(),
+           "cu_seqlens": None}
+    w = synth.TINY_CKDA_FP32.with_(B=1, T=T, H=1, dk=dk, dv=dv, chunk=16, signed_gate=1)
+    _, S = run_gpu(cuda_lib, inp, w)
+    S = f64(S)[0, 0]
+    ang = 2 * np.pi * (x.sum() % m) / m
+    R = np.array([[math.cos(ang), -math.sin(ang)], [math.sin(ang), math.cos(ang)]])
+    assert np.allclose(S[:2, :2], R, atol=1e-5)
+    assert np.allclose(S[2:, 2:], np.eye(dk - 2), atol=1e-6)
+
+
+def test_state_alias_and_resume(cuda_lib):
+    """S_T may alias S0; run(T1) then run(T2) from its state equals run(T1 + T2)."""
+    w = synth.CKDA_SPREAD.with_(B=2, T=190, H=2, io_dtype="f32", o_dtype="f32")
+    inp = synth.make_prefill(w, seed=8)
+    o_full, S_full = run_gpu(cuda_lib, inp, w)
+    T1 = 77
+    first = {k: (v[:, :T1].contiguous() if k in "qkvab" else v) for k, v in inp.items()}
+    second = {k: (v[:, T1:].contiguous() if k in "qkvab" else v) for k, v in inp.items()}
+    d1 = to_device(first)
+    o1, S1 = cuda_lib.chunk_fwd(d1["q"], d1["k"], d1["v"], d1["a"], d1["b"], d1["S0"], chunk=64,
+                                signed_gate=1)
+    d2 = to_device(second)
+    o2, S2 = cuda_lib.chunk_fwd(d2["q"], d2["k"], d2["v"], d2["a"], d2["b"], S1, chunk=64,
+                                signed_gate=1, S_T=S1)           # in place
+    torch.cuda.synchronize()
+    assert S2.data_ptr() == S1.data_ptr()
+    assert rel(f64(torch.cat([o1, o2], 1)), f64(o_full)) < 1e-5
+    assert rel(f64(S2), f64(S_full)) < 1e-5
+
+
+def test_chunk_size_invariance(cuda_lib):
+    w = synth.CKDA_SPREAD.with_(B=1, T=257, H=2, io_dtype="f32", o_dtype="f32")
+    inp = synth.make_prefill(w, seed=9)
+    outs = [run_gpu(cuda_lib, inp, w, chunk=c) for c in (16, 32, 64)]
+    for o, S in outs[1:]:
+        assert rel(f64(o), f64(outs[0][0])) < 1e-5 and rel(f64(S), f64(outs[0][1])) < 1e-5
+
+
+def test_bad_seqlens_sets_status(cuda_lib):
+    """Decreasing offsets: the kernel skips the bad sequences and records the error."""
+    w = synth.CKDA_SPREAD.with_(B=1, H=1, seq_lens=(10, 10), T=20, io_dtype="f32", o_dtype="f32")
+    inp = to_device(synth.make_prefill(w, seed=10))
+    cu = torch.tensor([0, 15, 12], dtype=torch.int32, device="cuda")  # ends below start
+    ws = cuda_lib.new_workspace(1, 20, 1, 128, 128, 64, 2)
+    cuda_lib.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["a"], inp["b"], inp["S0"], cu,
+                       signed_gate=1, workspace=ws)
+    assert cuda_lib.workspace_status(ws) == -6
+    cuda_lib.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["a"], inp["b"], inp["S0"],
+                       inp["cu_seqlens"], signed_gate=1, workspace=ws)
+    assert cuda_lib.workspace_status(ws) == 0
+
+
+# ---------------------------------------------------------------- full-size workloads
+# Sampled (sequence, head) units of the full workloads, in the launch
+# configuration the benchmark times (bf16 io, bf16 o, chunk 64).
+
+
+def _sampled(ops, w, units, seed=0):
+    inp = synth.make_prefill(w, seed)
+    o, S = run_gpu(ops, inp, w)
+    ref = oracle_units(inp, w.signed_gate, units)
+    o, S = f64(o), f64(S)
+    worst = 0.0
+    for (n, h), (ro, rS) in ref.items():
+        go = unit_rows(o, inp, n, h)
+        eo = rel(go, bf16_round(ro) if w.o_dtype == "bf16" else ro)
+        es = rel(S[n, h], rS)
+        assert eo <= TOL_BF16 and es <= TOL_BF16, (w.name, n, h, eo, es)
+        worst = max(worst, eo, es)
+    return worst
+
+
+def test_full_kda_std_sampled(cuda_lib):
+    _sampled(cuda_lib, synth.KDA_STD, [(0, 0), (1, 7), (2, 11), (3, 15)])
+
+
+def test_full_ckda_spread_sampled(cuda_lib):
+    _sampled(cuda_lib, synth.CKDA_SPREAD, [(0, 0), (3, 5), (7, 15)])
+
+
+def test_full_varlen_sampled(cuda_lib):
+    w = synth.varlen_workload(0)
+    _sampled(cuda_lib, w, [(0, 0), (5, 17), (16, 31)])
