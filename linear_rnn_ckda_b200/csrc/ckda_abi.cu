@@ -95,6 +95,7 @@ int ckda_chunk_fwd(const void *q, const void *k, const void *v, const void *a, c
   g.status = static_cast<int *>(workspace);
   g.workspace = workspace;
   g.workspace_bytes = workspace_bytes;
+  if (ckda::chunk_tc_supported(g)) return ckda::launch_chunk_tc(g, s);
   return ckda::launch_chunk_simt(g, s);
 }
 

@@ -32,6 +32,10 @@ struct DecodeArgs {
 // Exact fp32 SIMT chunkwise forward (any dk, dv, chunk).  Returns a CKDA_* code.
 int launch_chunk_simt(const ChunkArgs &args, cudaStream_t stream);
 
+// Tensor-core chunkwise forward (tcgen05, dk = dv = 128, chunk 64, bf16 io).
+bool chunk_tc_supported(const ChunkArgs &args);
+int launch_chunk_tc(const ChunkArgs &args, cudaStream_t stream);
+
 // One decode step.  Returns a CKDA_* code.
 int launch_decode(const DecodeArgs &args, cudaStream_t stream);
 

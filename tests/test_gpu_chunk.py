@@ -223,3 +223,76 @@ def test_full_ckda_spread_sampled(cuda_lib):
 def test_full_varlen_sampled(cuda_lib):
     w = synth.varlen_workload(0)
     _sampled(cuda_lib, w, [(0, 0), (5, 17), (16, 31)])
+
+
+# ---------------------------------------------------------------- tensor-core path
+# bf16 q/k/v/a with dk = dv = 128 and chunk 64 run on the tcgen05 kernel.
+
+
+def _bf16_raw_case(T, alpha_logit, b_logit, seed, H=2, S0=True):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((1, T, H, 128))
+    q /= np.linalg.norm(q, axis=-1, keepdims=True)
+    k = rng.standard_normal((1, T, H, 128))
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((1, T, H, 128))
+    bf = lambda x: torch.from_numpy(np.ascontiguousarray(x)).float().to(torch.bfloat16)
+    return {"q": bf(q), "k": bf(k), "v": bf(v), "a": bf(alpha_logit),
+            "b": torch.from_numpy(np.ascontiguousarray(b_logit)).float(),
+            "S0": torch.from_numpy(rng.standard_normal((1, H, 128, 128)) * 0.02).float()
+            if S0 else None, "cu_seqlens": None}
+
+
+@pytest.mark.parametrize("sg", [0, 1])
+def test_tc_degenerate_gates(cuda_lib, sg):
+    """Zero gates, +-1 gates, beta at 0 and 2 and strong decay on the bf16 d=128 path:
+    chunks whose gate products leave [2^-100, 2^100] take the exact token path."""
+    T, H = 333, 2
+    rng = np.random.default_rng(20 + sg)
+    a = rng.standard_normal((1, T, H, 128)) * 2 + (0 if sg else 3)
+    a[0, 5, 0, :] = -INF if sg == 0 else 0.0        # alpha = 0: full wipe in head 0
+    a[0, 70:75, 1, 10:20] = -INF if sg == 0 else 0.0
+    a[0, 140:150, 0, :] = INF                      # alpha = 1
+    if sg:
+        a[0, 150:160, 1, :] = -INF                 # alpha = -1
+    a[0, 200:264, 0, :32] = 1e-3 if sg else -60.0  # strong decay: products underflow
+    b = rng.standard_normal((1, T, H))
+    b[0, 7, :], b[0, 8, :] = INF, -INF
+    inp = _bf16_raw_case(T, a, b, seed=30 + sg)
+    w = synth.CKDA_SPREAD.with_(B=1, T=T, H=H, signed_gate=sg, o_dtype="f32")
+    o, S = run_gpu(cuda_lib, inp, w)
+    ro, rS = oracle_prefill(inp, sg)
+    assert rel(f64(o), ro) <= TOL_BF16 and rel(f64(S), rS) <= TOL_BF16
+
+
+def test_tc_varlen_edges(cuda_lib):
+    lens = (0, 1, 63, 64, 65, 130, 0, 7)
+    w = synth.CKDA_SPREAD.with_(B=1, H=3, seq_lens=lens, T=sum(lens), o_dtype="f32")
+    inp = synth.make_prefill(w, seed=11)
+    o, S = run_gpu(cuda_lib, inp, w)
+    ro, rS = oracle_prefill(inp, 1)
+    assert rel(f64(o), ro) <= TOL_BF16 and rel(f64(S), rS) <= TOL_BF16
+    S0 = f64(inp["S0"])
+    assert np.array_equal(f64(S)[0], S0[0]) and np.array_equal(f64(S)[6], S0[6])
+
+
+def test_tc_matches_simt(cuda_lib):
+    """The tcgen05 path (bf16 inputs) and the exact fp32 path (the same values as
+    fp32) agree within the bf16 tolerance."""
+    w = synth.KDA_STD.with_(B=2, T=257, H=2, o_dtype="f32")
+    inp = synth.make_prefill(w, seed=12)
+    o_tc, S_tc = run_gpu(cuda_lib, inp, w)
+    inp32 = {k: (v.float() if v is not None and v.dtype == torch.bfloat16 else v)
+             for k, v in inp.items()}
+    o_ex, S_ex = run_gpu(cuda_lib, inp32, w.with_(io_dtype="f32"))
+    assert rel(f64(o_tc), f64(o_ex)) <= TOL_BF16 and rel(f64(S_tc), f64(S_ex)) <= TOL_BF16
+
+
+def test_tc_state_alias_and_chunk_boundaries(cuda_lib):
+    """S_T aliasing S0 in place; T = 64, 128 and 129 exercise one, two and a ragged chunk."""
+    for T in (64, 128, 129):
+        w = synth.CKDA_SPREAD.with_(B=2, T=T, H=2, o_dtype="f32")
+        inp = synth.make_prefill(w, seed=13 + T)
+        ro, rS = oracle_prefill(inp, 1)
+        o, S = run_gpu(cuda_lib, inp, w, S0_alias=True)
+        assert rel(f64(o), ro) <= TOL_BF16 and rel(f64(S), rS) <= TOL_BF16, T
