@@ -97,7 +97,7 @@ __global__ void __launch_bounds__(kSimtThreads, 1) chunk_simt_kernel(SimtParams 
   }
 
   for (long cs = t0; cs < t1; cs += C) {
-    const int nrows = (int)std::min<long>(C, t1 - cs);
+    const int nrows = (int)(t1 - cs < C ? t1 - cs : C);
     __syncthreads();
     // ---- load q, k, raw a (rows past the sequence end: q = k = 0, alpha = 1)
     for (int e = tid; e < C * dk; e += kSimtThreads) {

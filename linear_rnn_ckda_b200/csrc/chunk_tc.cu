@@ -31,6 +31,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cstring>
 
 #include "common.cuh"
 #include "internal.h"
@@ -44,16 +45,17 @@ using namespace sm100;
 constexpr int kC = 64;      // chunk rows
 constexpr int kD = 128;     // dk = dv
 constexpr int kThreads = 256;
-constexpr int kLDA = 65;    // padded row stride of the plain fp32 scratch for the solve
 
 // shared memory map (bytes from a 1024-aligned base)
-constexpr uint32_t OFF_KQ = 0;          // [Kr;Qr] 128 rows x 128 fp32, 4 column blocks of 16 KB
-constexpr uint32_t OFF_KC = 65536;      // Kc 64 rows x 128 fp32, 4 column blocks of 8 KB
+constexpr uint32_t OFF_KQ = 0;          // [Kr;Qr] 128 rows x 128 fp32, 4 column blocks of 16 KB;
+                                        // rows 0..63 hold W once (1) has consumed Kr
+constexpr uint32_t OFF_KC = 65536;      // Kc 64 rows x 128 fp32, 4 column blocks of 8 KB;
+                                        // then the solve's A and X (plain 64 x 64 fp32 each)
 constexpr uint32_t OFF_KCT = 98304;     // Kc^T 128 rows x 64 fp32, 2 column blocks of 16 KB
-constexpr uint32_t OFF_T = 131072;      // Tm 64 x 64 fp32, 2 column blocks of 8 KB
-constexpr uint32_t OFF_P = 147456;      // P  64 x 64 fp32, 2 column blocks of 8 KB
-constexpr uint32_t OFF_STG = 163840;    // TMA staging: q, k, v, a bf16 64 x 128 (16 KB each);
-                                        // reused for the solve scratch and for W (64 x 128 fp32)
+constexpr uint32_t OFF_T = 131072;      // Tm 64 x 64 fp32, 2 column blocks of 8 KB (the solve's
+                                        // block scratch before that); T and P together
+constexpr uint32_t OFF_P = 147456;      // P  64 x 64 fp32 (2 blocks); T+P stage O for its TMA store
+constexpr uint32_t OFF_STG = 163840;    // TMA staging: q, k, v, a bf16 64 x 128 (16 KB each)
 constexpr uint32_t OFF_MISC = 229376;   // beta[64], gC[128], xch[128], barriers, tmem slot
 constexpr uint32_t kSmemUsed = OFF_MISC + 2048;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;  // + alignment slack
@@ -96,8 +98,43 @@ __device__ __forceinline__ void st_tf32(uint8_t *tile, uint32_t off, float x) {
   *reinterpret_cast<uint32_t *>(tile + off) = to_tf32(x);
 }
 
-// X = (I + A)^{-1} for a 64 x 64 strictly lower A (plain, row stride kLDA);
-// 16 x 16 diagonal blocks by forward substitution, then block rows in order.
+// Gates for the bf16 path, from their definitions with fast exponentials
+// (relative error ~1e-6, far inside the bf16-input tolerance):
+//   sigma(a) = 1 / (1 + e^{-a});  2 sigma(a) - 1 = tanh(a/2) = (1 - e^{-|a|}) / (1 + e^{-|a|})
+// with the odd Taylor series tanh(y) = y - y^3/3 + 2 y^5/15 for |a| < 0.1
+// (truncation below 2e-10 relative there), so small gates keep full precision.
+template <int SG>
+__device__ __forceinline__ float fast_alpha(float a) {
+  if (SG == 0) return __fdividef(1.f, 1.f + __expf(-a));
+  if (SG == 1) {
+    const float x = fabsf(a);
+    float t;
+    if (x < 0.1f) {
+      const float y = 0.5f * x, y2 = y * y;
+      t = y * fmaf(y2, fmaf(y2, 2.f / 15.f, -1.f / 3.f), 1.f);
+    } else {
+      const float e = __expf(-x);
+      t = __fdividef(1.f - e, 1.f + e);
+    }
+    return copysignf(t, a);
+  }
+  return a;
+}
+template <int SG>
+__device__ __forceinline__ float fast_beta(float b) {
+  if (SG == 0) return __fdividef(1.f, 1.f + __expf(-b));
+  if (SG == 1) return __fdividef(2.f, 1.f + __expf(-b));
+  return b;
+}
+
+// plain 64 x 64 fp32 scratch, columns XOR-swizzled by row so that a warp
+// touching one column of 32 consecutive rows hits 32 banks
+__device__ __forceinline__ int pidx(int r, int c) { return r * 64 + (c ^ (r & 31)); }
+
+// X = (I + A)^{-1} for a 64 x 64 strictly lower A (plain, pidx layout):
+// 16 x 16 diagonal blocks by forward substitution (one warp each), then the
+// block rows in order, X_ij = -X_ii sum_{k=j}^{i-1} A_ik X_kj, with four
+// partial sums per dot product.
 __device__ void unit_lower_inverse(const float *A, float *X, float *Y, int tid) {
   const int warp = tid >> 5, lane = tid & 31;
   if (warp < 4 && lane < 16) {
@@ -105,46 +142,52 @@ __device__ void unit_lower_inverse(const float *A, float *X, float *Y, int tid) 
     float x[16];
 #pragma unroll
     for (int r = 0; r < 16; ++r) {
-      float acc = 0.f;
+      float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-      for (int l = 0; l < r; ++l) acc = fmaf(-A[(o + r) * kLDA + o + l], x[l], acc);
-      x[r] = (r == m) ? 1.f : acc;
+      for (int l = 0; l < r; ++l) {
+        if (l & 1) a1 = fmaf(-A[pidx(o + r, o + l)], x[l], a1);
+        else a0 = fmaf(-A[pidx(o + r, o + l)], x[l], a0);
+      }
+      x[r] = (r == m) ? 1.f : a0 + a1;
     }
 #pragma unroll
-    for (int r = 0; r < 16; ++r) X[(o + r) * kLDA + o + m] = x[r];
+    for (int r = 0; r < 16; ++r) X[pidx(o + r, o + m)] = x[r];
   }
   __syncthreads();
   const int r = tid >> 4, m = tid & 15;
+#pragma unroll
   for (int i = 1; i < 4; ++i) {
     // Y_j = sum_{k=j}^{i-1} A_ik X_kj for every block j < i
-    for (int j = 0; j < i; ++j) {
-      float acc = 0.f;
-      for (int k = j; k < i; ++k) {
-        const float *Ar = A + (16 * i + r) * kLDA + 16 * k;
-        const float *Xc = X + (16 * k) * kLDA + 16 * j + m;
 #pragma unroll
-        for (int l = 0; l < 16; ++l) acc = fmaf(Ar[l], Xc[l * kLDA], acc);
+    for (int j = 0; j < i; ++j) {
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int k = j; k < i; ++k) {
+#pragma unroll
+        for (int l = 0; l < 16; ++l)
+          acc[l & 3] = fmaf(A[pidx(16 * i + r, 16 * k + l)], X[pidx(16 * k + l, 16 * j + m)], acc[l & 3]);
       }
-      Y[(j * 16 + r) * 17 + m] = acc;
+      Y[(j * 16 + r) * 17 + m] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
     }
     __syncthreads();
     // X_ij = -X_ii Y_j
-    for (int j = 0; j < i; ++j) {
-      float acc = 0.f;
-      const float *Xr = X + (16 * i + r) * kLDA + 16 * i;
 #pragma unroll
-      for (int l = 0; l < 16; ++l) acc = fmaf(-Xr[l], Y[(j * 16 + l) * 17 + m], acc);
-      X[(16 * i + r) * kLDA + 16 * j + m] = acc;
+    for (int j = 0; j < i; ++j) {
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int l = 0; l < 16; ++l)
+        acc[l & 3] = fmaf(-X[pidx(16 * i + r, 16 * i + l)], Y[(j * 16 + l) * 17 + m], acc[l & 3]);
+      X[pidx(16 * i + r, 16 * j + m)] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
     }
     __syncthreads();
   }
 }
 
-template <typename TOut>
+template <typename TOut, int SG>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_a,
-                    TcParams p) {
+                    const __grid_constant__ CUtensorMap tm_o, TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -195,6 +238,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t tma_phase = 0, mma_phase = 0;
   bool tma_pending = false, mma_pending = false, failed = false;
 
+  // one warp polls an mbarrier phase; the block then agrees on the outcome
+  auto block_wait = [&](uint64_t *bar, uint32_t parity) -> bool {
+    bool ok = true;
+    if (warp == 0) ok = mbar_wait(bar, parity, kWaitNs);
+    return __syncthreads_and(ok) != 0;
+  };
   auto issue_tma = [&](long cs) {
     mbar_arrive_expect_tx(tma_bar, 4 * 2 * 8192);
     const int row = (int)(bofs + cs);
@@ -227,12 +276,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
 
   const uint8_t *stq = sStg, *stk = sStg + 16384, *stv = sStg + 32768, *sta = sStg + 49152;
+  // strengths are loaded one chunk ahead (threads 0..63, one row each)
+  float b_next = 0.f;
+  if (tid < kC && t0 + tid < t1) b_next = p.b[(size_t)(bofs + t0 + tid) * H + h];
+  bool store_pending = false;
 
   for (long cs = t0; cs < t1; cs += kC) {
     const int nrows = (int)(t1 - cs < kC ? t1 - cs : kC);
     const bool has_next = cs + kC < t1;
+    const float b_cur = b_next;
+    if (tid < kC && cs + kC + tid < t1) b_next = p.b[(size_t)(bofs + cs + kC + tid) * H + h];
     // ---------------------------------------------------------------- A: gates and operands
-    if (!__syncthreads_and(mbar_wait(tma_bar, tma_phase, kWaitNs))) { failed = true; break; }
+    if (!block_wait(tma_bar, tma_phase)) { failed = true; break; }
     tma_phase ^= 1;
     tma_pending = false;
     const int c = tid & 127, hf = tid >> 7;
@@ -242,16 +297,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int rr = 0; rr < 32; ++rr) {
         const int r = 32 * hf + rr;
-        const float al = r < nrows ? gate_alpha(ldbf(sta, r, c), p.signed_gate) : 1.f;
-        run *= al;
+        const float al = fast_alpha<SG>(ldbf(sta, r, c));
+        run *= r < nrows ? al : 1.f;
         g[rr] = run;
       }
       if (hf == 0) sXch[c] = run;
     }
-    if (tid < kC) {
-      const int r = tid;
-      sBeta[r] = r < nrows ? gate_beta(p.b[(size_t)(bofs + cs + r) * H + h], p.signed_gate) : 0.f;
-    }
+    if (tid < kC) sBeta[tid] = tid < nrows ? fast_beta<SG>(b_cur) : 0.f;
     __syncthreads();
     bool bad = false;
     {
@@ -265,13 +317,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float gam = g[rr] * mult;
           const float ag = fabsf(gam);
           bad |= !(ag >= 0x1p-100f && ag <= 0x1p100f);
-          const float inv = __frcp_rn(gam);
-          float qv = 0.f, kv = 0.f, vv = 0.f;
-          if (r < nrows) {
-            qv = ldbf(stq, r, c);
-            kv = ldbf(stk, r, c);
-            vv = ldbf(stv, r, c);
-          }
+          const float inv = __fdividef(1.f, gam);
+          // rows past the sequence end hold another sequence's tokens or TMA fill: masked
+          const bool valid = r < nrows;
+          const float q_raw = ldbf(stq, r, c), k_raw = ldbf(stk, r, c), v_raw = ldbf(stv, r, c);
+          const float qv = valid ? q_raw : 0.f, kv = valid ? k_raw : 0.f, vv = valid ? v_raw : 0.f;
           const uint32_t kr = to_tf32(kv * gam), kc = to_tf32(kv * inv);
           *reinterpret_cast<uint32_t *>(sKQ + sw32(128, r, c)) = kr;
           st_tf32(sKQ, sw32(128, 64 + r, c), qv * gam);
@@ -279,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint32_t *>(sKCT + sw32(128, c, r)) = kc;
           krt[x] = kr;
           vt[x] = __float_as_uint(vv);
-          if (r == kC - 1) sGC[c] = gam;
+          if (rr == 31 && hf == 1) sGC[c] = gam;
         }
         // lane c of TMEM holds Kr^T[c][.] and V^T[c][.] (A operands of (2) and (3))
         tmem_st16(lane_addr + COL_KRT + 32 * hf + 16 * grp, krt);
@@ -297,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 4
       for (int rr = 0; rr < 32; ++rr) {
         const int r = 32 * hf + rr;
-        sAl[r * kD + c] = r < nrows ? gate_alpha(ldbf(sta, r, c), p.signed_gate) : 1.f;
+        sAl[r * kD + c] = r < nrows ? gate_alpha(ldbf(sta, r, c), SG) : 1.f;
       }
       __syncthreads();
       {
@@ -354,6 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---------------------------------------------------------------- (1) [A;P] = [Kr;Qr] Kc^T
     if (tid == 0) {
+      if (has_next) issue_tma(cs + kC);   // staging is free: prep has consumed it
       tc_fence_after();
 #pragma unroll
       for (int s = 0; s < 16; ++s) {
@@ -362,16 +413,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_ss(tmem + COL_AP, a, b, IDESC_N64, s > 0);
       }
       mma_commit(mma_bar);
+      if (store_pending) bulk_wait_read();  // previous O tile (over T and P) has left smem
     }
+    tma_pending = has_next;
+    store_pending = false;
     mma_pending = true;
-    if (!__syncthreads_and(mbar_wait(mma_bar, mma_phase, kWaitNs))) { failed = true; break; }
+    if (!block_wait(mma_bar, mma_phase)) { failed = true; break; }
     mma_phase ^= 1;
     mma_pending = false;
     tc_fence_after();
     // ---------------------------------------------------------------- A and P out of TMEM
-    float *sA = reinterpret_cast<float *>(sStg);          // plain [64][kLDA]
-    float *sX = sA + 64 * kLDA;                            // plain [64][kLDA]
-    float *sY = sX + 64 * kLDA;                            // [3*16][17]
+    float *sA = reinterpret_cast<float *>(sKC);           // plain [64][64], pidx layout
+    float *sX = sA + 64 * 64;                              // plain [64][64], pidx layout
+    float *sY = reinterpret_cast<float *>(sT);             // [3*16][17] block scratch
     {
       uint32_t r[32];
       tmem_ld32(lane_addr + COL_AP + 32 * half, r);
@@ -382,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int x = 0; x < 32; ++x) {
           const int j = 32 * half + x;
-          sA[t * kLDA + j] = j < t ? __uint_as_float(r[x]) * bt : 0.f;
+          sA[pidx(t, j)] = j < t ? __uint_as_float(r[x]) * bt : 0.f;
         }
       } else {
         const int t = jrow - 64;
@@ -398,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     unit_lower_inverse(sA, sX, sY, tid);
     for (int e = tid; e < kC * kC; e += kThreads) {
       const int t = e >> 6, s = e & 63;
-      st_tf32(sT, sw32(64, t, s), s <= t ? sX[t * kLDA + s] * sBeta[s] : 0.f);
+      st_tf32(sT, sw32(64, t, s), s <= t ? sX[pidx(t, s)] * sBeta[s] : 0.f);
     }
     fence_proxy_async();
     __syncthreads();
@@ -414,18 +468,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(mma_bar);
     }
     mma_pending = true;
-    if (!__syncthreads_and(mbar_wait(mma_bar, mma_phase, kWaitNs))) { failed = true; break; }
+    if (!block_wait(mma_bar, mma_phase)) { failed = true; break; }
     mma_phase ^= 1;
     mma_pending = false;
     tc_fence_after();
-    // ---------------------------------------------------------------- W (rows t, key channels) into staging
+    // ---------------------------------------------------------------- W (rows t, key channels) over Kr
     {
       uint32_t r[32];
       tmem_ld32(lane_addr + COL_W + 32 * half, r);
       tmem_wait_ld();
       const int i = jrow;
 #pragma unroll
-      for (int x = 0; x < 32; ++x) st_tf32(sStg, sw32(64, 32 * half + x, i), __uint_as_float(r[x]));
+      for (int x = 0; x < 32; ++x) st_tf32(sKQ, sw32(128, 32 * half + x, i), __uint_as_float(r[x]));
     }
     fence_proxy_async();
     tc_fence_before();
@@ -435,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
 #pragma unroll
       for (int s = 0; s < 16; ++s) {
-        const uint64_t bw = smem_desc_sw128(sbase + OFF_STG + (s >> 2) * 8192 + (s & 3) * 32, 16, 1024);
+        const uint64_t bw = smem_desc_sw128(sbase + OFF_KQ + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024);
         mma_ts(tmem + COL_U, tmem + COL_S + 8 * s, bw, IDESC_U, 1);
       }
 #pragma unroll
@@ -447,12 +501,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(mma_bar);
     }
     mma_pending = true;
-    if (!__syncthreads_and(mbar_wait(mma_bar, mma_phase, kWaitNs))) { failed = true; break; }
+    if (!block_wait(mma_bar, mma_phase)) { failed = true; break; }
     mma_phase ^= 1;
     mma_pending = false;
-    // ---------------------------------------------------------------- next chunk's loads; (5b) O^T += U^T P^T, (6) S^T += U^T Kc
+    // ---------------------------------------------------------------- (5b) O^T += U^T P^T, (6) S^T += U^T Kc
     if (tid == 0) {
-      if (has_next) issue_tma(cs + kC);   // staging (W) is free once (4) has completed
       tc_fence_after();
 #pragma unroll
       for (int s = 0; s < 8; ++s) {
@@ -466,9 +519,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       mma_commit(mma_bar);
     }
-    tma_pending = has_next;
     mma_pending = true;
-    if (!__syncthreads_and(mbar_wait(mma_bar, mma_phase, kWaitNs))) { failed = true; break; }
+    if (!block_wait(mma_bar, mma_phase)) { failed = true; break; }
     mma_phase ^= 1;
     mma_pending = false;
     tc_fence_after();
@@ -477,7 +529,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t r[32];
       tmem_ld32(lane_addr + COL_O + 32 * half, r);
       tmem_wait_ld();
-      if (o) {
+      if (o && nrows == kC) {
+        // full chunk: O [t][j] staged over T and P, written by one TMA store
+        TOut *sO = reinterpret_cast<TOut *>(sT);
+#pragma unroll
+        for (int x = 0; x < 32; ++x)
+          sO[(32 * half + x) * kD + jrow] = from_f32<TOut>(__uint_as_float(r[x]));
+        fence_proxy_async();
+      } else if (o) {
 #pragma unroll
         for (int x = 0; x < 32; ++x) {
           const int t = 32 * half + x;
@@ -498,7 +557,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     tc_fence_before();
     __syncthreads();
+    if (tid == 0 && o && nrows == kC) {
+      tma_store_3d(&tm_o, sT, 0, h, (int)(bofs + cs));
+      bulk_commit();
+      store_pending = true;
+    }
   }
+  if (tid == 0) bulk_wait_all();
 
   if (failed) {
     if (tid == 0) set_status(p.status, CKDA_ERR_TIMEOUT);
@@ -538,7 +603,8 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
-// [rows, H, 128] bf16 viewed as a 3-D tensor (channel, head, token); box 64 x 1 x 64.
+// [rows, H, 128] bf16 viewed as a 3-D tensor (channel, head, token); box 64 x 1 x 64,
+// 128-byte swizzle (the staging layout the gate threads read).
 bool make_map(CUtensorMap *map, const void *base, int H, long rows) {
   auto enc = get_encode();
   if (!enc) return false;
@@ -551,25 +617,41 @@ bool make_map(CUtensorMap *map, const void *base, int H, long rows) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <typename TOut>
+// o [rows, H, 128] (bf16 or fp32) for whole-chunk stores: box 128 x 1 x 64, no swizzle.
+bool make_out_map(CUtensorMap *map, void *base, int H, long rows, bool bf16) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  const cuuint64_t es = bf16 ? 2 : 4;
+  cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)kD * es, (cuuint64_t)H * kD * es};
+  cuuint32_t box[3] = {kD, 1, kC};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base,
+             dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename TOut, int SG>
 int launch_typed(const ChunkArgs &g, cudaStream_t stream) {
   const long rows = (long)g.B * g.T;
   if (rows == 0) {
     // no tokens: S_T = S0 (or zero) is still produced by the kernel below
   }
-  CUtensorMap mq, mk, mv, ma;
+  CUtensorMap mq, mk, mv, ma, mo;
   const long map_rows = rows > 0 ? rows : 1;
   if (!make_map(&mq, g.q, g.H, map_rows) || !make_map(&mk, g.k, g.H, map_rows) ||
       !make_map(&mv, g.v, g.H, map_rows) || !make_map(&ma, g.a, g.H, map_rows))
     return CKDA_ERR_CUDA;
+  memset(&mo, 0, sizeof(mo));
+  if (g.o && !make_out_map(&mo, g.o, g.H, map_rows, g.o_dtype == CKDA_BF16)) return CKDA_ERR_CUDA;
   TcParams p;
   p.b = g.b; p.S0 = g.S0; p.cu = g.cu_seqlens; p.o = g.o; p.S_T = g.S_T; p.status = g.status;
   p.n_seqs = g.n_seqs; p.T = g.T; p.H = g.H; p.signed_gate = g.signed_gate;
-  auto kern = chunk_tc_kernel<TOut>;
+  auto kern = chunk_tc_kernel<TOut, SG>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) !=
       cudaSuccess)
     return CKDA_ERR_CUDA;
-  kern<<<g.n_seqs * g.H, kThreads, kSmemBytes, stream>>>(mq, mk, mv, ma, p);
+  kern<<<g.n_seqs * g.H, kThreads, kSmemBytes, stream>>>(mq, mk, mv, ma, mo, p);
   return cudaGetLastError() == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
 }
 
@@ -581,7 +663,12 @@ bool chunk_tc_supported(const ChunkArgs &g) {
 
 int launch_chunk_tc(const ChunkArgs &g, cudaStream_t s) {
   if (g.n_seqs * g.H == 0) return CKDA_OK;
-  return g.o_dtype == CKDA_BF16 ? launch_typed<__nv_bfloat16>(g, s) : launch_typed<float>(g, s);
+  const bool bf = g.o_dtype == CKDA_BF16;
+  switch (g.signed_gate) {
+    case 0: return bf ? launch_typed<__nv_bfloat16, 0>(g, s) : launch_typed<float, 0>(g, s);
+    case 1: return bf ? launch_typed<__nv_bfloat16, 1>(g, s) : launch_typed<float, 1>(g, s);
+    default: return bf ? launch_typed<__nv_bfloat16, 2>(g, s) : launch_typed<float, 2>(g, s);
+  }
 }
 
 }  // namespace ckda
