@@ -119,6 +119,33 @@ int ckda_decode_step(const void *q, const void *k, const void *v, const void *a,
                      int o_dtype, void *o, void *stream);
 
 /*
+ * ckda_chunk_fwd without a caller-provided workspace.  The pages describe no
+ * such call; it exists for callers that cannot allocate device memory at all,
+ * for example a serving runtime that plans all device memory at start-up and
+ * forbids later allocations, or plain C code that links only this library
+ * and has no device allocator.  Arguments, layouts and results are those of
+ * ckda_chunk_fwd; the workspace is replaced by a fixed 4096-byte scratch array
+ * compiled into the library (every GPU that loads the library holds it until
+ * the process exits).  Sizes whose workspace would exceed 4096 bytes are
+ * rejected with CKDA_ERR_WORKSPACE.  Neither this call nor the library calls
+ * cudaMalloc or cudaFree.
+ *   - The first call on each device looks up the scratch array's device
+ *     address (cudaGetSymbolAddress) with that device current; make that
+ *     first call before any stream capture.
+ *   - Every call on a device shares the same scratch, and it keeps what the
+ *     last call left there; the status header is cleared on `stream` at the
+ *     start of each call.  Calls whose work overlaps on the GPU (different
+ *     streams without ordering) race on the scratch: serialise them.
+ *   - The device status word (bad cu_seqlens, timeouts) cannot be read back
+ *     through ckda_workspace_status, since the caller has no pointer to it.
+ * Returns CKDA_OK or a negative CKDA_ERR_* code.
+ */
+int ckda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const void *a,
+                           const float *b, const float *S0, const int32_t *cu_seqlens, int n_seqs,
+                           int B, int T, int H, int dk, int dv, int chunk, int signed_gate,
+                           int io_dtype, int o_dtype, void *o, float *S_T, void *stream);
+
+/*
  * Reads the device status word that ckda_chunk_fwd records in `workspace`
  * (CKDA_OK, CKDA_ERR_SEQLENS or CKDA_ERR_TIMEOUT) into *status.  This call
  * SYNCHRONISES `stream` (it copies 4 bytes to the host).  Returns CKDA_OK or

@@ -32,6 +32,8 @@ SIGNATURES = {
                             _i, _i, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
     "ckda_chunk_fwd_workspace_size": (ctypes.c_size_t, [_i, _i, _i, _i, _i, _i, _i]),
     "ckda_decode_step": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp]),
+    "ckda_chunk_fwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
+                                    _i, _i, _i, _vp, _vp, _vp]),
     "ckda_workspace_status": (_i, [_vp, ctypes.POINTER(_i), _vp]),
     "ckda_status_string": (ctypes.c_char_p, [_i]),
     "ckda_version": (_i, []),
