@@ -65,6 +65,33 @@ def decode_bytes(w):
     return heads * (2 * w.dk * w.dv * 4 + io * (3 * w.dk + w.dv) + 4 + ob * w.dv)
 
 
+PROFILED = os.path.join(ROOT, "profiles", "roofline_traffic.json")
+CSRC = os.path.join(ROOT, "linear_rnn_ckda_b200", "csrc")
+
+
+def source_hash(files):
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(CSRC, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(kernel):
+    """DRAM bytes per launch from the committed ncu capture of `kernel`, or None
+    when the kernel's sources changed after the capture."""
+    try:
+        with open(PROFILED) as f:
+            rec = json.load(f)[kernel]
+        if source_hash(rec["sources"]) != rec["source_sha256"]:
+            return None
+        return float(rec["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -246,6 +273,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--decode-steps", type=int, default=None,
                     help="timed decode steps (default: --steps rounded up to the 128-step cycle)")
+    ap.add_argument("--legs", default="prefill,e2e,decode",
+                    help="comma list of legs to run (prefill, e2e, decode); a profiling run can "
+                         "select one, the default runs all")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -265,6 +295,7 @@ def main():
     stream = torch.cuda.current_stream(dev)
     peaks = load_peaks()
 
+    legs = set(args.legs.split(","))
     # ------------------------------------------------------------ prefill leg
     w = PREFILL
     host = synth.make_prefill(w, seed=rank)
@@ -278,7 +309,10 @@ def main():
                       signed_gate=w.signed_gate, o=o, S_T=S_T, workspace=ws)
 
     with ClockSampler(local) as clk:
-        ms = time_loop(prefill, args.steps, args.warmup, world, stream)
+        ms = time_loop(prefill, args.steps if "prefill" in legs else 1,
+                       args.warmup if "prefill" in legs else 0, world, stream)
+    if "prefill" not in legs:
+        ms = float("nan")
     ms = max_over_ranks(ms, world)
     ms_step = ms / args.steps
     tokens = w.tokens * world
@@ -293,13 +327,15 @@ def main():
     flops = prefill_flops_per_token_head(w.dk, w.dv, w.chunk) * w.tokens * w.H
     achieved_gbs = byts / (ms_step * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": None,
+                "frac": achieved_gbs / peaks["hbm_gbs"],
+                "traffic": profiled_traffic("chunk_tc_kernel"),
                 "peak_source": peaks["source"],
                 "algorithmic_bytes_per_launch": byts, "algorithmic_flop_per_launch": flops,
                 "tensor_tflops": flops / (ms_step * 1e-3) / 1e12,
                 "tensor_frac_of_bf16": flops / (ms_step * 1e-3) / 1e12 / peaks["bf16_tflops"]}
 
     # ------------------------------------------------------------ e2e prefill (host buffers)
+    e2e = None
     pin = {k: (None if v is None else v.pin_memory()) for k, v in host.items()}
     o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
     S_host = torch.empty(S_T.shape, dtype=S_T.dtype).pin_memory()
@@ -316,33 +352,36 @@ def main():
         S_host.copy_(S_T, non_blocking=True)
 
     e2e_steps = max(3, min(args.steps, 10))
-    ms_e2e = max_over_ranks(time_loop(e2e_step, e2e_steps, 2, world, stream), world)
-    e2e = {"value": tokens * e2e_steps / (ms_e2e / 1000.0), "unit": "tokens/s",
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    if "e2e" in legs:
+        ms_e2e = max_over_ranks(time_loop(e2e_step, e2e_steps, 2, world, stream), world)
+        e2e = {"value": tokens * e2e_steps / (ms_e2e / 1000.0), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
     del dd, pin, o_host, S_host
 
     # ------------------------------------------------------------ decode leg
     wd = DECODE
-    dec_host = synth.make_decode(wd, seed=rank)
-    dq = {k: v.to(dev) for k, v in dec_host.items()}
-    S = dq["S"]
-    o_dec = torch.empty((wd.B, wd.H, wd.dv), dtype=torch.float32, device=dev)
-    counter = [0]
-
-    def decode():
-        t = counter[0] % wd.decode_steps
-        counter[0] += 1
-        ops.decode_step(dq["q"][t], dq["k"][t], dq["v"][t], dq["a"][t], dq["b"][t], S,
-                        signed_gate=wd.signed_gate, o_dtype=torch.float32, o=o_dec)
-
     dsteps = args.decode_steps or max(args.steps, 128)
-    ms_d = max_over_ranks(time_loop(decode, dsteps, args.warmup, world, stream), world)
-    dbytes = decode_bytes(wd)
-    dec_gbs = dbytes * world * dsteps / (ms_d / 1000.0) / 1e9
-    decode_obj = {"value": dec_gbs, "unit": "GB/s", "frac": dec_gbs / world / peaks["hbm_gbs"],
-                  "peak": peaks["hbm_gbs"], "ms_per_step": ms_d / dsteps, "steps": dsteps,
-                  "workload": wd.name, "algorithmic_bytes_per_step": dbytes,
-                  "state_bytes_per_step": wd.B * wd.H * wd.dk * wd.dv * 8}
+    decode_obj = None
+    if "decode" in legs:
+        dq = {k: v.to(dev) for k, v in synth.make_decode(wd, seed=rank).items()}
+        S = dq["S"]
+        o_dec = torch.empty((wd.B, wd.H, wd.dv), dtype=torch.float32, device=dev)
+        counter = [0]
+
+        def decode():
+            t = counter[0] % wd.decode_steps
+            counter[0] += 1
+            ops.decode_step(dq["q"][t], dq["k"][t], dq["v"][t], dq["a"][t], dq["b"][t], S,
+                            signed_gate=wd.signed_gate, o_dtype=torch.float32, o=o_dec)
+
+        ms_d = max_over_ranks(time_loop(decode, dsteps, args.warmup, world, stream), world)
+        dbytes = decode_bytes(wd)
+        dec_gbs = dbytes * world * dsteps / (ms_d / 1000.0) / 1e9
+        decode_obj = {"value": dec_gbs, "unit": "GB/s", "frac": dec_gbs / world / peaks["hbm_gbs"],
+                      "peak": peaks["hbm_gbs"], "ms_per_step": ms_d / dsteps, "steps": dsteps,
+                      "workload": wd.name, "algorithmic_bytes_per_step": dbytes,
+                      "state_bytes_per_step": wd.B * wd.H * wd.dk * wd.dv * 8,
+                      "traffic": profiled_traffic("decode_kernel")}
 
     # ------------------------------------------------------------ CPU baseline (oracle)
     cpu = None
