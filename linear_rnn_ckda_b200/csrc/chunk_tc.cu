@@ -56,7 +56,7 @@ constexpr uint32_t OFF_T = 131072;      // Tm 64 x 64 fp32, 2 column blocks of 8
                                         // block scratch before that); T and P together
 constexpr uint32_t OFF_P = 147456;      // P  64 x 64 fp32 (2 blocks); T+P stage O for its TMA store
 constexpr uint32_t OFF_STG = 163840;    // TMA staging: q, k, v, a bf16 64 x 128 (16 KB each)
-constexpr uint32_t OFF_MISC = 229376;   // beta[64], gC[128], xch[128], barriers, tmem slot
+constexpr uint32_t OFF_MISC = 229376;   // beta[64], gC[2][128], xch[128], barriers, tmem slot
 constexpr uint32_t kSmemUsed = OFF_MISC + 2048;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;  // + alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -131,53 +131,87 @@ __device__ __forceinline__ float fast_beta(float b) {
 // touching one column of 32 consecutive rows hits 32 banks
 __device__ __forceinline__ int pidx(int r, int c) { return r * 64 + (c ^ (r & 31)); }
 
-// X = (I + A)^{-1} for a 64 x 64 strictly lower A (plain, pidx layout):
-// 16 x 16 diagonal blocks by forward substitution (one warp each), then the
-// block rows in order, X_ij = -X_ii sum_{k=j}^{i-1} A_ik X_kj, with four
-// partial sums per dot product.
-__device__ void unit_lower_inverse(const float *A, float *X, float *Y, int tid) {
+// T = (I + A)^{-1} Diag(beta) for a 64 x 64 strictly lower A (pidx layout),
+// written as tf32 into the K-major T tile.  X (plain, stride 64) receives the
+// inverse, Y (4 KB) is scratch.  Recursive doubling on the block structure:
+//   stage 0: the eight 8 x 8 diagonal blocks by forward substitution (warp w,
+//            lane m = column m of block w);
+//   stage s = 1, 2, 3: every diagonal block of size 2b = 8 << s is finished
+//            from its two halves, X_10 = -X_11 (A_10 X_00), all such blocks at
+//            once; each product is spread over all 256 threads.
+// The strictly upper part of T is written as zeros at stage 0.
+__device__ void solve_T(const float *A, float *X, float *Y, uint8_t *sT, const float *beta, int tid) {
   const int warp = tid >> 5, lane = tid & 31;
-  if (warp < 4 && lane < 16) {
-    const int o = 16 * warp, m = lane;
-    float x[16];
+  {
+    // stage 0 (lanes 0..7 of every warp) and T's upper zeros (all threads)
+    if (lane < 8) {
+      const int o = 8 * warp, m = lane;
+      float x[8];
 #pragma unroll
-    for (int r = 0; r < 16; ++r) {
-      float a0 = 0.f, a1 = 0.f;
+      for (int r = 0; r < 8; ++r) {
+        float acc = 0.f;
 #pragma unroll
-      for (int l = 0; l < r; ++l) {
-        if (l & 1) a1 = fmaf(-A[pidx(o + r, o + l)], x[l], a1);
-        else a0 = fmaf(-A[pidx(o + r, o + l)], x[l], a0);
+        for (int l = 0; l < r; ++l) acc = fmaf(-A[pidx(o + r, o + l)], x[l], acc);
+        x[r] = (r == m) ? 1.f : acc;
       }
-      x[r] = (r == m) ? 1.f : a0 + a1;
-    }
+      const float bm = beta[o + m];
 #pragma unroll
-    for (int r = 0; r < 16; ++r) X[pidx(o + r, o + m)] = x[r];
+      for (int r = 0; r < 8; ++r) {
+        X[(o + r) * 64 + o + m] = x[r];
+        st_tf32(sT, sw32(64, o + r, o + m), r >= m ? x[r] * bm : 0.f);
+      }
+    }
+    // zeros above the 8 x 8 diagonal blocks, in T and in X (the merges read X's
+    // diagonal blocks whole)
+    for (int e = tid; e < 64 * 64; e += 256) {
+      const int t = e >> 6, s = e & 63;
+      if (s >= ((t >> 3) + 1) * 8) {
+        st_tf32(sT, sw32(64, t, s), 0.f);
+        X[t * 64 + s] = 0.f;
+      }
+    }
   }
   __syncthreads();
-  const int r = tid >> 4, m = tid & 15;
 #pragma unroll
-  for (int i = 1; i < 4; ++i) {
-    // Y_j = sum_{k=j}^{i-1} A_ik X_kj for every block j < i
-#pragma unroll
-    for (int j = 0; j < i; ++j) {
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int k = j; k < i; ++k) {
-#pragma unroll
-        for (int l = 0; l < 16; ++l)
-          acc[l & 3] = fmaf(A[pidx(16 * i + r, 16 * k + l)], X[pidx(16 * k + l, 16 * j + m)], acc[l & 3]);
+  for (int st = 1; st <= 3; ++st) {
+    const int b = 4 << st;                // half size of the blocks finished here: 8, 16, 32
+    const int tpb = (b / 2) * (b / 2);    // 2 x 2 output tiles per block
+    const int ntiles = (64 / (2 * b)) * tpb;
+    const int blk = tid / tpb, w = tid % tpb, r0 = 2 * (w / (b / 2)), c0 = 2 * (w % (b / 2));
+    const int o = blk * 2 * b;
+    float *Yb = Y + blk * b * b;
+    // phase 1: Y = A_10 X_00 (A_10: rows o+b.., columns o..; X_00: the upper diagonal block)
+    if (tid < ntiles) {
+      float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
+#pragma unroll 8
+      for (int l = 0; l < b; ++l) {
+        const float a0 = A[pidx(o + b + r0, o + l)], a1 = A[pidx(o + b + r0 + 1, o + l)];
+        const float2 xv = *reinterpret_cast<const float2 *>(X + (o + l) * 64 + o + c0);
+        y00 = fmaf(a0, xv.x, y00); y01 = fmaf(a0, xv.y, y01);
+        y10 = fmaf(a1, xv.x, y10); y11 = fmaf(a1, xv.y, y11);
       }
-      Y[(j * 16 + r) * 17 + m] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+      *reinterpret_cast<float2 *>(Yb + r0 * b + c0) = make_float2(y00, y01);
+      *reinterpret_cast<float2 *>(Yb + (r0 + 1) * b + c0) = make_float2(y10, y11);
     }
     __syncthreads();
-    // X_ij = -X_ii Y_j
-#pragma unroll
-    for (int j = 0; j < i; ++j) {
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int l = 0; l < 16; ++l)
-        acc[l & 3] = fmaf(-X[pidx(16 * i + r, 16 * i + l)], Y[(j * 16 + l) * 17 + m], acc[l & 3]);
-      X[pidx(16 * i + r, 16 * j + m)] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+    // phase 2: X_10 = -X_11 Y (X_11: the lower diagonal block, finished earlier)
+    if (tid < ntiles) {
+      float z00 = 0.f, z01 = 0.f, z10 = 0.f, z11 = 0.f;
+#pragma unroll 8
+      for (int l = 0; l < b; ++l) {
+        const float x0 = X[(o + b + r0) * 64 + o + b + l], x1 = X[(o + b + r0 + 1) * 64 + o + b + l];
+        const float2 yv = *reinterpret_cast<const float2 *>(Yb + l * b + c0);
+        z00 = fmaf(-x0, yv.x, z00); z01 = fmaf(-x0, yv.y, z01);
+        z10 = fmaf(-x1, yv.x, z10); z11 = fmaf(-x1, yv.y, z11);
+      }
+      float *X0 = X + (o + b + r0) * 64 + o + c0;
+      *reinterpret_cast<float2 *>(X0) = make_float2(z00, z01);
+      *reinterpret_cast<float2 *>(X0 + 64) = make_float2(z10, z11);
+      const float b0 = beta[o + c0], b1 = beta[o + c0 + 1];
+      st_tf32(sT, sw32(64, o + b + r0, o + c0), z00 * b0);
+      st_tf32(sT, sw32(64, o + b + r0, o + c0 + 1), z01 * b1);
+      st_tf32(sT, sw32(64, o + b + r0 + 1, o + c0), z10 * b0);
+      st_tf32(sT, sw32(64, o + b + r0 + 1, o + c0 + 1), z11 * b1);
     }
     __syncthreads();
   }
@@ -193,12 +227,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t *sKQ = sm + OFF_KQ, *sKC = sm + OFF_KC, *sKCT = sm + OFF_KCT, *sT = sm + OFF_T,
           *sP = sm + OFF_P, *sStg = sm + OFF_STG;
-  float *sBeta = reinterpret_cast<float *>(sm + OFF_MISC);
-  float *sGC = sBeta + 64;
-  float *sXch = sGC + 128;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_MISC + 1280);
+  float *sBeta = reinterpret_cast<float *>(sm + OFF_MISC);     // [64]
+  float *sGC = sBeta + 64;                                       // [2][128] G_63, double-buffered
+  float *sXch = sGC + 256;                                       // [128]
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_MISC + 1792);
   uint64_t *tma_bar = bars, *mma_bar = bars + 1;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_MISC + 1296);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_MISC + 1808);
   const uint32_t sbase = smem_u32(sm);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -231,12 +265,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int q4 = warp & 3, half = warp >> 2;
-  const uint32_t lane_addr = tmem + ((uint32_t)(32 * q4) << 16);
-  const int jrow = 32 * q4 + lane;  // TMEM lane owned by this thread
+  // TMEM lane of this thread and which half of a row it handles; the gate pass
+  // uses the same mapping (channel c = jrow, rows 32*half .. 32*half + 31).
+  const int half = warp >> 2;
+  const int jrow = 32 * (warp & 3) + lane;
+  const int c = jrow, hf = half;
+  const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
 
   uint32_t tma_phase = 0, mma_phase = 0;
-  bool tma_pending = false, mma_pending = false, failed = false;
+  bool tma_pending = false, mma_pending = false, failed = false, store_pending = false;
+
+  // descriptors of the fixed operand tiles (K-major, 128-byte swizzle)
+  const uint64_t dKQ = smem_desc_sw128(sbase + OFF_KQ, 16, 1024);
+  const uint64_t dKC = smem_desc_sw128(sbase + OFF_KC, 16, 1024);
+  const uint64_t dKCT = smem_desc_sw128(sbase + OFF_KCT, 16, 1024);
+  const uint64_t dT = smem_desc_sw128(sbase + OFF_T, 16, 1024);
+  const uint64_t dP = smem_desc_sw128(sbase + OFF_P, 16, 1024);
+  auto dadd = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (bytes >> 4); };
 
   // one warp polls an mbarrier phase; the block then agrees on the outcome
   auto block_wait = [&](uint64_t *bar, uint32_t parity) -> bool {
@@ -255,6 +300,69 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d(sStg + x * 16384 + bx * 8192, maps[x], tma_bar, bx * 64, h, row);
   };
 
+  const uint8_t *stq = sStg, *stk = sStg + 16384, *stv = sStg + 32768, *sta = sStg + 49152;
+
+  // ---- gate pass: staging (q, k, v, a of one chunk) -> Kr, Qr, Kc, Kc^T tiles, Kr^T and V^T
+  // in TMEM, beta, G_63.  Kc^T is left in kc[] for the caller to store (its tile may still be
+  // read by the previous chunk's last MMA group).  Returns whether the chunk is out of range.
+  float b_next = 0.f;
+  if (tid < kC && t0 + tid < t1) b_next = p.b[(size_t)(bofs + t0 + tid) * H + h];
+  float kc[32];
+  auto gate_pass = [&](long cs, int nrows, float *gc_out) -> bool {
+    const float b_cur = b_next;
+    if (tid < kC && cs + kC + tid < t1) b_next = p.b[(size_t)(bofs + cs + kC + tid) * H + h];
+    float g[32];
+    float run = 1.f;
+#pragma unroll
+    for (int rr = 0; rr < 32; ++rr) {
+      const int r = 32 * hf + rr;
+      const float al = fast_alpha<SG>(ldbf(sta, r, c));
+      run *= r < nrows ? al : 1.f;
+      g[rr] = run;
+    }
+    if (hf == 0) sXch[c] = run;
+    if (tid < kC) sBeta[tid] = tid < nrows ? fast_beta<SG>(b_cur) : 0.f;
+    __syncthreads();
+    bool bad = false;
+    const float mult = hf ? sXch[c] : 1.f;
+#pragma unroll
+    for (int grp = 0; grp < 2; ++grp) {
+      uint32_t krt[16], vt[16];
+#pragma unroll
+      for (int x = 0; x < 16; ++x) {
+        const int rr = 16 * grp + x, r = 32 * hf + rr;
+        const float gam = g[rr] * mult;
+        const float ag = fabsf(gam);
+        bad |= !(ag >= 0x1p-100f && ag <= 0x1p100f);
+        const float inv = __fdividef(1.f, gam);
+        // rows past the sequence end hold another sequence's tokens or TMA fill: masked
+        const bool valid = r < nrows;
+        const float q_raw = ldbf(stq, r, c), k_raw = ldbf(stk, r, c), v_raw = ldbf(stv, r, c);
+        const float qv = valid ? q_raw : 0.f, kv = valid ? k_raw : 0.f, vv = valid ? v_raw : 0.f;
+        const uint32_t kr = to_tf32(kv * gam);
+        const uint32_t kcb = to_tf32(kv * inv);
+        *reinterpret_cast<uint32_t *>(sKQ + sw32(128, r, c)) = kr;
+        st_tf32(sKQ, sw32(128, 64 + r, c), qv * gam);
+        *reinterpret_cast<uint32_t *>(sKC + sw32(64, r, c)) = kcb;
+        kc[rr] = __uint_as_float(kcb);
+        krt[x] = kr;
+        vt[x] = __float_as_uint(vv);
+        if (rr == 31 && hf == 1) gc_out[c] = gam;
+      }
+      // lane c of TMEM holds Kr^T[c][.] and V^T[c][.] (A operands of (2) and (3))
+      tmem_st16(lane_addr + COL_KRT + 32 * hf + 16 * grp, krt);
+      tmem_st16(lane_addr + COL_VT + 32 * hf + 16 * grp, vt);
+    }
+    tmem_wait_st();
+    return bad;
+  };
+  auto store_kct = [&]() {  // four consecutive t per 16-byte store
+#pragma unroll
+    for (int rr = 0; rr < 32; rr += 4)
+      *reinterpret_cast<float4 *>(sKCT + sw32(128, c, 32 * hf + rr)) =
+          make_float4(kc[rr], kc[rr + 1], kc[rr + 2], kc[rr + 3]);
+  };
+
   // ---- initial state into TMEM: thread (lane j, half) holds S^T[j][64*half .. +64) = S0[i][j]
   {
 #pragma unroll
@@ -268,149 +376,115 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     tmem_wait_st();
   }
-  if (tid == 0 && t1 > t0) {
-    issue_tma(t0);
-  }
+  if (tid == 0 && t1 > t0) issue_tma(t0);
   tma_pending = t1 > t0;
   tc_fence_before();
   __syncthreads();
 
-  const uint8_t *stq = sStg, *stk = sStg + 16384, *stv = sStg + 32768, *sta = sStg + 49152;
-  // strengths are loaded one chunk ahead (threads 0..63, one row each)
-  float b_next = 0.f;
-  if (tid < kC && t0 + tid < t1) b_next = p.b[(size_t)(bofs + t0 + tid) * H + h];
-  bool store_pending = false;
-
-  for (long cs = t0; cs < t1; cs += kC) {
-    const int nrows = (int)(t1 - cs < kC ? t1 - cs : kC);
-    const bool has_next = cs + kC < t1;
-    const float b_cur = b_next;
-    if (tid < kC && cs + kC + tid < t1) b_next = p.b[(size_t)(bofs + cs + kC + tid) * H + h];
-    // ---------------------------------------------------------------- A: gates and operands
-    if (!block_wait(tma_bar, tma_phase)) { failed = true; break; }
+  // gate pass of the first chunk
+  int gsel = 0;              // sGC buffer of the chunk being processed
+  bool slow = false;
+  if (t1 > t0) {
+    if (!block_wait(tma_bar, tma_phase)) failed = true;
     tma_phase ^= 1;
     tma_pending = false;
-    const int c = tid & 127, hf = tid >> 7;
-    float g[32];
-    {
-      float run = 1.f;
-#pragma unroll
-      for (int rr = 0; rr < 32; ++rr) {
-        const int r = 32 * hf + rr;
-        const float al = fast_alpha<SG>(ldbf(sta, r, c));
-        run *= r < nrows ? al : 1.f;
-        g[rr] = run;
-      }
-      if (hf == 0) sXch[c] = run;
+    if (!failed) {
+      const bool bad = gate_pass(t0, (int)(t1 - t0 < kC ? t1 - t0 : kC), sGC);
+      store_kct();
+      fence_proxy_async();
+      tc_fence_before();
+      slow = __syncthreads_or(bad) != 0;
     }
-    if (tid < kC) sBeta[tid] = tid < nrows ? fast_beta<SG>(b_cur) : 0.f;
-    __syncthreads();
-    bool bad = false;
-    {
-      const float mult = hf ? sXch[c] : 1.f;
-#pragma unroll
-      for (int grp = 0; grp < 2; ++grp) {
-        uint32_t krt[16], vt[16];
-#pragma unroll
-        for (int x = 0; x < 16; ++x) {
-          const int rr = 16 * grp + x, r = 32 * hf + rr;
-          const float gam = g[rr] * mult;
-          const float ag = fabsf(gam);
-          bad |= !(ag >= 0x1p-100f && ag <= 0x1p100f);
-          const float inv = __fdividef(1.f, gam);
-          // rows past the sequence end hold another sequence's tokens or TMA fill: masked
-          const bool valid = r < nrows;
-          const float q_raw = ldbf(stq, r, c), k_raw = ldbf(stk, r, c), v_raw = ldbf(stv, r, c);
-          const float qv = valid ? q_raw : 0.f, kv = valid ? k_raw : 0.f, vv = valid ? v_raw : 0.f;
-          const uint32_t kr = to_tf32(kv * gam), kc = to_tf32(kv * inv);
-          *reinterpret_cast<uint32_t *>(sKQ + sw32(128, r, c)) = kr;
-          st_tf32(sKQ, sw32(128, 64 + r, c), qv * gam);
-          *reinterpret_cast<uint32_t *>(sKC + sw32(64, r, c)) = kc;
-          *reinterpret_cast<uint32_t *>(sKCT + sw32(128, c, r)) = kc;
-          krt[x] = kr;
-          vt[x] = __float_as_uint(vv);
-          if (rr == 31 && hf == 1) sGC[c] = gam;
-        }
-        // lane c of TMEM holds Kr^T[c][.] and V^T[c][.] (A operands of (2) and (3))
-        tmem_st16(lane_addr + COL_KRT + 32 * hf + 16 * grp, krt);
-        tmem_st16(lane_addr + COL_VT + 32 * hf + 16 * grp, vt);
-      }
-      tmem_wait_st();
-    }
-    tc_fence_before();
-    fence_proxy_async();
-    const bool slow = __syncthreads_or(bad);
+  }
+
+  for (long cs = t0; cs < t1 && !failed; cs += kC) {
+    const int nrows = (int)(t1 - cs < kC ? t1 - cs : kC);
+    const bool has_next = cs + kC < t1;
+    const int nrows_next = has_next ? (int)(t1 - cs - kC < kC ? t1 - cs - kC : kC) : 0;
+    float *gc_cur = sGC + 128 * gsel, *gc_next = sGC + 128 * (gsel ^ 1);
 
     if (slow) {
       // ------------------------------------------------------------ exact token-by-token path
-      float *sAl = reinterpret_cast<float *>(sKQ);  // plain [64][128] gates
+      // state S[i][j] in smem over Kr/Qr, gates over Kc, partial sums over Kc^T
+      float *sS = reinterpret_cast<float *>(sKQ);
+      float *sAl = reinterpret_cast<float *>(sKC);
+      float *sRed = reinterpret_cast<float *>(sKCT);
 #pragma unroll 4
       for (int rr = 0; rr < 32; ++rr) {
         const int r = 32 * hf + rr;
         sAl[r * kD + c] = r < nrows ? gate_alpha(ldbf(sta, r, c), SG) : 1.f;
       }
-      __syncthreads();
-      {
-        // thread (value channel jrow, key half): s[x] = S^T[jrow][64*half + x]
-        float *sRed = sAl + kC * kD;  // [2][2][128] partial dot products
-        float s[64];
+      tc_fence_after();
 #pragma unroll
-        for (int cb = 0; cb < 2; ++cb) {
-          uint32_t r[32];
-          tmem_ld32(lane_addr + COL_S + 64 * half + 32 * cb, r);
-          tmem_wait_ld();
+      for (int cb = 0; cb < 2; ++cb) {
+        uint32_t r[32];
+        const int i0 = 64 * half + 32 * cb;
+        tmem_ld32(lane_addr + COL_S + i0, r);
+        tmem_wait_ld();
 #pragma unroll
-          for (int x = 0; x < 32; ++x) s[32 * cb + x] = __uint_as_float(r[x]);
-        }
-        for (int t = 0; t < nrows; ++t) {
-          float pk = 0.f;
-#pragma unroll
-          for (int x = 0; x < 64; ++x) {
-            const int i = 64 * half + x;
-            s[x] *= sAl[t * kD + i];
-            pk = fmaf(ldbf(stk, t, i), s[x], pk);
-          }
-          sRed[half * 128 + jrow] = pk;
-          __syncthreads();
-          const float u = sBeta[t] * (ldbf(stv, t, jrow) - (sRed[jrow] + sRed[128 + jrow]));
-          float acc = 0.f;
-#pragma unroll
-          for (int x = 0; x < 64; ++x) {
-            const int i = 64 * half + x;
-            s[x] = fmaf(ldbf(stk, t, i), u, s[x]);
-            acc = fmaf(ldbf(stq, t, i), s[x], acc);
-          }
-          sRed[256 + half * 128 + jrow] = acc;
-          __syncthreads();
-          if (half == 0 && o)
-            o[((size_t)(bofs + cs + t) * H + h) * kD + jrow] =
-                from_f32<TOut>(sRed[256 + jrow] + sRed[384 + jrow]);
-        }
-#pragma unroll
-        for (int cb = 0; cb < 2; ++cb) {
-          uint32_t r[32];
-#pragma unroll
-          for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(s[32 * cb + x]);
-          tmem_st32(lane_addr + COL_S + 64 * half + 32 * cb, r);
-        }
-        tmem_wait_st();
+        for (int x = 0; x < 32; ++x) sS[(i0 + x) * kD + jrow] = __uint_as_float(r[x]);
       }
+      __syncthreads();
+      for (int t = 0; t < nrows; ++t) {
+        float pk = 0.f;
+        for (int x = 0; x < 64; ++x) {
+          const int i = 64 * half + x;
+          const float sv = sS[i * kD + jrow] * sAl[t * kD + i];
+          sS[i * kD + jrow] = sv;
+          pk = fmaf(ldbf(stk, t, i), sv, pk);
+        }
+        sRed[half * 128 + jrow] = pk;
+        __syncthreads();
+        const float u = sBeta[t] * (ldbf(stv, t, jrow) - (sRed[jrow] + sRed[128 + jrow]));
+        float acc = 0.f;
+        for (int x = 0; x < 64; ++x) {
+          const int i = 64 * half + x;
+          const float sv = fmaf(ldbf(stk, t, i), u, sS[i * kD + jrow]);
+          sS[i * kD + jrow] = sv;
+          acc = fmaf(ldbf(stq, t, i), sv, acc);
+        }
+        sRed[256 + half * 128 + jrow] = acc;
+        __syncthreads();
+        if (half == 0 && o)
+          o[((size_t)(bofs + cs + t) * H + h) * kD + jrow] =
+              from_f32<TOut>(sRed[256 + jrow] + sRed[384 + jrow]);
+      }
+#pragma unroll
+      for (int cb = 0; cb < 2; ++cb) {
+        uint32_t r[32];
+        const int i0 = 64 * half + 32 * cb;
+#pragma unroll
+        for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(sS[(i0 + x) * kD + jrow]);
+        tmem_st32(lane_addr + COL_S + i0, r);
+      }
+      tmem_wait_st();
       tc_fence_before();
       __syncthreads();
-      if (tid == 0 && has_next) issue_tma(cs + kC);
-      tma_pending = has_next;
+      if (has_next) {
+        if (tid == 0) issue_tma(cs + kC);
+        tma_pending = true;
+        if (!block_wait(tma_bar, tma_phase)) { failed = true; break; }
+        tma_phase ^= 1;
+        tma_pending = false;
+        const bool bad = gate_pass(cs + kC, nrows_next, gc_next);
+        store_kct();
+        fence_proxy_async();
+        tc_fence_before();
+        slow = __syncthreads_or(bad) != 0;
+        gsel ^= 1;
+      }
       continue;
     }
 
     // ---------------------------------------------------------------- (1) [A;P] = [Kr;Qr] Kc^T
     if (tid == 0) {
-      if (has_next) issue_tma(cs + kC);   // staging is free: prep has consumed it
+      if (has_next) issue_tma(cs + kC);   // staging is free: the gate pass has consumed it
       tc_fence_after();
 #pragma unroll
       for (int s = 0; s < 16; ++s) {
-        const uint64_t a = smem_desc_sw128(sbase + OFF_KQ + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024);
-        const uint64_t b = smem_desc_sw128(sbase + OFF_KC + (s >> 2) * 8192 + (s & 3) * 32, 16, 1024);
-        mma_ss(tmem + COL_AP, a, b, IDESC_N64, s > 0);
+        const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
+        mma_ss(tmem + COL_AP, dadd(dKQ, off), dadd(dKC, (s >> 2) * 8192 + (s & 3) * 32), IDESC_N64,
+               s > 0);
       }
       mma_commit(mma_bar);
       if (store_pending) bulk_wait_read();  // previous O tile (over T and P) has left smem
@@ -424,8 +498,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     // ---------------------------------------------------------------- A and P out of TMEM
     float *sA = reinterpret_cast<float *>(sKC);           // plain [64][64], pidx layout
-    float *sX = sA + 64 * 64;                              // plain [64][64], pidx layout
-    float *sY = reinterpret_cast<float *>(sT);             // [3*16][17] block scratch
+    float *sX = sA + 64 * 64;                              // plain [64][64]
+    float *sY = reinterpret_cast<float *>(sKQ);           // [3][16][16] over the consumed Kr rows
     {
       uint32_t r[32];
       tmem_ld32(lane_addr + COL_AP + 32 * half, r);
@@ -449,11 +523,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncthreads();
     // ---------------------------------------------------------------- Tm = (I + A)^{-1} Diag(beta)
-    unit_lower_inverse(sA, sX, sY, tid);
-    for (int e = tid; e < kC * kC; e += kThreads) {
-      const int t = e >> 6, s = e & 63;
-      st_tf32(sT, sw32(64, t, s), s <= t ? sX[pidx(t, s)] * sBeta[s] : 0.f);
-    }
+    solve_T(sA, sX, sY, sT, sBeta, tid);
     fence_proxy_async();
     __syncthreads();
     // ---------------------------------------------------------------- (2) W^T, (3) U^T
@@ -461,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
 #pragma unroll
       for (int s = 0; s < 8; ++s) {
-        const uint64_t bt = smem_desc_sw128(sbase + OFF_T + (s >> 2) * 8192 + (s & 3) * 32, 16, 1024);
+        const uint64_t bt = dadd(dT, (s >> 2) * 8192 + (s & 3) * 32);
         mma_ts(tmem + COL_W, tmem + COL_KRT + 8 * s, bt, IDESC_N64, s > 0);
         mma_ts(tmem + COL_U, tmem + COL_VT + 8 * s, bt, IDESC_N64, s > 0);
       }
@@ -489,14 +559,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
 #pragma unroll
       for (int s = 0; s < 16; ++s) {
-        const uint64_t bw = smem_desc_sw128(sbase + OFF_KQ + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024);
-        mma_ts(tmem + COL_U, tmem + COL_S + 8 * s, bw, IDESC_U, 1);
+        const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
+        mma_ts(tmem + COL_U, tmem + COL_S + 8 * s, dadd(dKQ, off), IDESC_U, 1);
       }
 #pragma unroll
       for (int s = 0; s < 16; ++s) {
-        const uint64_t bq =
-            smem_desc_sw128(sbase + OFF_KQ + 8192 + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024);
-        mma_ts(tmem + COL_O, tmem + COL_S + 8 * s, bq, IDESC_N64, s > 0);
+        const uint32_t off = 8192 + (s >> 2) * 16384 + (s & 3) * 32;
+        mma_ts(tmem + COL_O, tmem + COL_S + 8 * s, dadd(dKQ, off), IDESC_N64, s > 0);
       }
       mma_commit(mma_bar);
     }
@@ -508,18 +577,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) {
       tc_fence_after();
 #pragma unroll
-      for (int s = 0; s < 8; ++s) {
-        const uint64_t bp = smem_desc_sw128(sbase + OFF_P + (s >> 2) * 8192 + (s & 3) * 32, 16, 1024);
-        mma_ts(tmem + COL_O, tmem + COL_U + 8 * s, bp, IDESC_N64, 1);
-      }
+      for (int s = 0; s < 8; ++s)
+        mma_ts(tmem + COL_O, tmem + COL_U + 8 * s, dadd(dP, (s >> 2) * 8192 + (s & 3) * 32),
+               IDESC_N64, 1);
 #pragma unroll
-      for (int s = 0; s < 8; ++s) {
-        const uint64_t bk = smem_desc_sw128(sbase + OFF_KCT + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024);
-        mma_ts(tmem + COL_S, tmem + COL_U + 8 * s, bk, IDESC_S, 1);
-      }
+      for (int s = 0; s < 8; ++s)
+        mma_ts(tmem + COL_S, tmem + COL_U + 8 * s, dadd(dKCT, (s >> 2) * 16384 + (s & 3) * 32),
+               IDESC_S, 1);
       mma_commit(mma_bar);
     }
     mma_pending = true;
+    // ---------------------------------------------------------------- next chunk's gate pass,
+    // overlapping (5b)/(6): Kr, Qr and Kc are free, Kc^T is not (kept in registers)
+    bool bad_next = false;
+    if (has_next) {
+      if (!block_wait(tma_bar, tma_phase)) { failed = true; break; }
+      tma_phase ^= 1;
+      tma_pending = false;
+      bad_next = gate_pass(cs + kC, nrows_next, gc_next);
+    }
     if (!block_wait(mma_bar, mma_phase)) { failed = true; break; }
     mma_phase ^= 1;
     mma_pending = false;
@@ -535,7 +611,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int x = 0; x < 32; ++x)
           sO[(32 * half + x) * kD + jrow] = from_f32<TOut>(__uint_as_float(r[x]));
-        fence_proxy_async();
       } else if (o) {
 #pragma unroll
         for (int x = 0; x < 32; ++x) {
@@ -550,26 +625,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(lane_addr + COL_S + i0, r);
         tmem_wait_ld();
 #pragma unroll
-        for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * sGC[i0 + x]);
+        for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * gc_cur[i0 + x]);
         tmem_st32(lane_addr + COL_S + i0, r);
       }
       tmem_wait_st();
     }
+    if (has_next) store_kct();
+    fence_proxy_async();
     tc_fence_before();
-    __syncthreads();
+    slow = __syncthreads_or(bad_next) != 0;
     if (tid == 0 && o && nrows == kC) {
       tma_store_3d(&tm_o, sT, 0, h, (int)(bofs + cs));
       bulk_commit();
       store_pending = true;
     }
+    gsel ^= 1;
   }
   if (tid == 0) bulk_wait_all();
 
   if (failed) {
     if (tid == 0) set_status(p.status, CKDA_ERR_TIMEOUT);
     // let in-flight copies and MMAs drain (bounded) before giving TMEM back
-    if (tma_pending) mbar_wait(tma_bar, tma_phase, kWaitNs);
-    if (mma_pending) mbar_wait(mma_bar, mma_phase, kWaitNs);
+    if (warp == 0) {
+      if (tma_pending) mbar_wait(tma_bar, tma_phase, kWaitNs);
+      if (mma_pending) mbar_wait(mma_bar, mma_phase, kWaitNs);
+    }
   } else if (p.S_T) {
     tc_fence_after();
 #pragma unroll
@@ -672,3 +752,9 @@ int launch_chunk_tc(const ChunkArgs &g, cudaStream_t s) {
 }
 
 }  // namespace ckda
+
+extern "C" int ckda_timed_solve(unsigned long long *out) {
+}
+
+extern "C" int ckda_timed_phases(unsigned long long *out) {
+}
