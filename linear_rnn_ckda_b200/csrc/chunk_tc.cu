@@ -8,25 +8,27 @@
 //   Kr = K * G,  Qr = Q * G,  Kc = K / G    (row-wise, per channel)
 //   A  = tril(Diag(beta) Kr Kc^T, -1)       P = tril(Qr Kc^T)
 //   Tm = (I + A)^{-1} Diag(beta)
-//   W  = Tm Kr,   U = Tm V - W S
+//   U  = Tm (V - Kr S)          (the WY form U = Tm V - (Tm Kr) S, regrouped)
 //   O  = Qr S + P U
 //   S' = Diag(G_63) (S + Kc^T U)
 // Everything is computed transposed so that every product has M = 128 on the
 // tensor core: the state lives in TMEM as S^T (lane = value channel j,
 // column = key channel i) and is the A operand of the state products.
 //   (1) [A;P]   = [Kr;Qr] Kc^T          M=128 (64 Kr rows + 64 Qr rows), N=64, K=128
-//   (2) W^T     = Kr^T Tm^T              A = Kr^T in TMEM (lane = key channel), K=64
-//   (3) U^T     = V^T Tm^T               A = V^T in TMEM (lane = value channel), K=64
-//   (4) U^T    -= S^T W^T                A = S^T in TMEM, K=128
-//   (5) O^T     = S^T Qr^T + U^T P^T     A from TMEM
-//   (6) S^T    += U^T Kc,  then columns scaled by G_63 (threads, in TMEM)
-// All MMAs are kind::tf32 with fp32 accumulation and K-major operands; smem
-// operands and the TMEM copies of Kr^T are rounded to tf32 (round-to-nearest)
-// when written; the state and U are read from TMEM directly.  The gate products are the signed cumulative products in
-// fp32 (the sign bit carries the gate-sign parity).  A chunk whose product
-// falls outside [2^-100, 2^100] in some channel (an exact zero gate, or
-// extreme decay) cannot use the factorisation Kr Kc^T; it is run token by
-// token, exactly, on the same TMEM-resident state (slow path).
+//   (a) [X^T|O^T] = S^T [Kr;Qr]^T       N=128 (X = Kr S, and O's first term), K=128
+//   (b) V' = V - X in fp32 (threads), kept in TMEM as tf32 hi + lo parts
+//   (c) U^T     = V'^T Tm^T              A = V'^T in TMEM (hi and lo), K=64, in two rounds
+//   (d) O^T    += U^T P^T,  S^T += U^T Kc, then S^T columns scaled by G_63 (threads, in TMEM)
+// (1) and (a) need only the chunk's inputs and S, so they are issued together
+// when the chunk starts, and (b) overlaps the solve.  All MMAs are kind::tf32
+// with fp32 accumulation and K-major operands; smem operands are rounded to
+// tf32 (round-to-nearest) when written.  TMEM operands (S, U) are read as tf32
+// directly (the low mantissa bits ignored); V' is split so that none of it is
+// lost.  The gate products are the signed cumulative products in fp32
+// (the sign bit carries the gate-sign parity).  A chunk whose product falls
+// outside [2^-100, 2^100] in some channel (an exact zero gate, or extreme
+// decay) cannot use the factorisation Kr Kc^T; it is run token by token,
+// exactly, on the same TMEM-resident state (slow path).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -44,30 +46,31 @@ using namespace sm100;
 
 constexpr int kC = 64;      // chunk rows
 constexpr int kD = 128;     // dk = dv
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;   // 16 warps: 4 per scheduler to hide latency
 
 // shared memory map (bytes from a 1024-aligned base)
-constexpr uint32_t OFF_KQ = 0;          // [Kr;Qr] 128 rows x 128 fp32, 4 column blocks of 16 KB;
-                                        // rows 0..63 hold W once (1) has consumed Kr
+constexpr uint32_t OFF_KQ = 0;          // [Kr;Qr] 128 rows x 128 fp32, 4 column blocks of 16 KB
 constexpr uint32_t OFF_KC = 65536;      // Kc 64 rows x 128 fp32, 4 column blocks of 8 KB;
-                                        // then the solve's A and X (plain 64 x 64 fp32 each)
+                                        // then the solve's A (64 x kAS) and the M tile
 constexpr uint32_t OFF_KCT = 98304;     // Kc^T 128 rows x 64 fp32, 2 column blocks of 16 KB
-constexpr uint32_t OFF_T = 131072;      // Tm 64 x 64 fp32, 2 column blocks of 8 KB (the solve's
-                                        // block scratch before that); T and P together
+constexpr uint32_t OFF_T = 131072;      // Tm 64 x 64 fp32, 2 column blocks of 8 KB; T and P together
 constexpr uint32_t OFF_P = 147456;      // P  64 x 64 fp32 (2 blocks); T+P stage O for its TMA store
+constexpr uint32_t OFF_M = OFF_KC + 18432;   // M = X2 A21, 32 x 32 tf32 (one column block)
 constexpr uint32_t OFF_STG = 163840;    // TMA staging: q, k, v, a bf16 64 x 128 (16 KB each)
-constexpr uint32_t OFF_MISC = 229376;   // beta[64], gC[2][128], xch[128], barriers, tmem slot
+constexpr uint32_t OFF_MISC = 229376;   // beta[64], gC[2][128], barriers, tmem slot
 constexpr uint32_t kSmemUsed = OFF_MISC + 2048;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;  // + alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 // TMEM columns (all 512 allocated)
-constexpr uint32_t COL_S = 0, COL_AP = 128, COL_W = 192, COL_U = 256, COL_O = 320, COL_KRT = 384,
-                   COL_VT = 448;
+// [A;P] and, once read out, the lo part of V'; X = Kr S and O adjacent (one N = 128
+// product); V^T (then the hi part of V') of two chunks at COL_VT and COL_VT + 64
+constexpr uint32_t COL_S = 0, COL_AP = 128, COL_LO = 128, COL_X = 192, COL_O = 256, COL_U = 320,
+                   COL_VT = 384;
 
-constexpr uint32_t IDESC_N64 = idesc_tf32(128, 64, false, false);        // (1), (2), (3), (5)
-constexpr uint32_t IDESC_U = idesc_tf32(128, 64, false, false, true);    // (4), B negated
-constexpr uint32_t IDESC_S = idesc_tf32(128, 128, false, false);         // (6)
+constexpr uint32_t IDESC_N64 = idesc_tf32(128, 64, false, false);         // (1), (c), O += U P^T
+constexpr uint32_t IDESC_N32_NEG = idesc_tf32(128, 32, false, false, true);  // (c) second round
+constexpr uint32_t IDESC_N128 = idesc_tf32(128, 128, false, false);       // (a), S^T += U^T Kc
 
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s bound on any single wait
 
@@ -127,93 +130,57 @@ __device__ __forceinline__ float fast_beta(float b) {
   return b;
 }
 
-// plain 64 x 64 fp32 scratch, columns XOR-swizzled by row so that a warp
-// touching one column of 32 consecutive rows hits 32 banks
-__device__ __forceinline__ int pidx(int r, int c) { return r * 64 + (c ^ (r & 31)); }
+// Row stride (floats) of the plain A array: consecutive rows start 16 bytes
+// apart modulo 128, so 32 threads writing 16 bytes of 32 different rows hit
+// every bank once per wavefront.
+constexpr int kAS = 68;
 
-// T = (I + A)^{-1} Diag(beta) for a 64 x 64 strictly lower A (pidx layout),
-// written as tf32 into the K-major T tile.  X (plain, stride 64) receives the
-// inverse, Y (4 KB) is scratch.  Recursive doubling on the block structure:
-//   stage 0: the eight 8 x 8 diagonal blocks by forward substitution (warp w,
-//            lane m = column m of block w);
-//   stage s = 1, 2, 3: every diagonal block of size 2b = 8 << s is finished
-//            from its two halves, X_10 = -X_11 (A_10 X_00), all such blocks at
-//            once; each product is spread over all 256 threads.
-// The strictly upper part of T is written as zeros at stage 0.
-__device__ void solve_T(const float *A, float *X, float *Y, uint8_t *sT, const float *beta, int tid) {
+// Tm = (I + A)^{-1} Diag(beta) for the 64 x 64 strictly lower A (plain, row
+// stride kAS, zeros on and above the diagonal).  In 32 x 32 blocks
+//   I + A = [[L1, 0], [A21, L2]],  (I + A)^{-1} = [[X1, 0], [-M X1, X2]],
+//   X1 = L1^{-1},  X2 = L2^{-1},  M = X2 A21.
+// X1, X2 and M are three independent forward substitutions (warps 0, 1, 2):
+// lane j keeps column j in registers and finishes the rows in order, reading
+// each row of the triangular factor as a broadcast; all fp32.  Written as tf32:
+// the block-diagonal part Tb = blockdiag(X1, X2) Diag(beta) into the T tile
+// (off-diagonal blocks zero) and M into its own 32 x 32 tile.  The off-diagonal
+// block of Tm is never formed: with U = Tm V' and Ub = Tb V' (rows split
+// 32 + 32), U_top = Ub_top and U_bot = Ub_bot - M U_top, a second MMA round.
+__device__ __forceinline__ void solve_T(const float *A, uint8_t *sT, uint8_t *sMt,
+                                        const float *beta, int tid) {
   const int warp = tid >> 5, lane = tid & 31;
-  {
-    // stage 0 (lanes 0..7 of every warp) and T's upper zeros (all threads)
-    if (lane < 8) {
-      const int o = 8 * warp, m = lane;
-      float x[8];
+  if (warp >= 3) return;
+  const int j = lane;
+  const int o = warp == 0 ? 0 : 32;   // the diagonal block solved by this warp
+  float x[32];
 #pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        float acc = 0.f;
+  for (int r = 0; r < 32; ++r) {
+    const float *row = A + (o + r) * kAS + o;
+    // right-hand side: column j of the identity (X1, X2) or of A21 (M)
+    float acc0 = warp == 2 ? A[(32 + r) * kAS + j] : (r == j ? 1.f : 0.f);
+    float acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
 #pragma unroll
-        for (int l = 0; l < r; ++l) acc = fmaf(-A[pidx(o + r, o + l)], x[l], acc);
-        x[r] = (r == m) ? 1.f : acc;
-      }
-      const float bm = beta[o + m];
-#pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        X[(o + r) * 64 + o + m] = x[r];
-        st_tf32(sT, sw32(64, o + r, o + m), r >= m ? x[r] * bm : 0.f);
-      }
+    for (int l4 = 0; l4 < r; l4 += 4) {
+      const float4 a = *reinterpret_cast<const float4 *>(row + l4);
+      acc0 = fmaf(-a.x, x[l4], acc0);
+      if (l4 + 1 < r) acc1 = fmaf(-a.y, x[l4 + 1], acc1);
+      if (l4 + 2 < r) acc2 = fmaf(-a.z, x[l4 + 2], acc2);
+      if (l4 + 3 < r) acc3 = fmaf(-a.w, x[l4 + 3], acc3);
     }
-    // zeros above the 8 x 8 diagonal blocks, in T and in X (the merges read X's
-    // diagonal blocks whole)
-    for (int e = tid; e < 64 * 64; e += 256) {
-      const int t = e >> 6, s = e & 63;
-      if (s >= ((t >> 3) + 1) * 8) {
-        st_tf32(sT, sw32(64, t, s), 0.f);
-        X[t * 64 + s] = 0.f;
-      }
-    }
+    x[r] = (acc0 + acc1) + (acc2 + acc3);
   }
-  __syncthreads();
+  if (warp < 2) {
+    // Tb: column o + j of the diagonal block, zeros in the same column of the other block row
+    const float bj = beta[o + j];
+    const int zr = 32 - o;
 #pragma unroll
-  for (int st = 1; st <= 3; ++st) {
-    const int b = 4 << st;                // half size of the blocks finished here: 8, 16, 32
-    const int tpb = (b / 2) * (b / 2);    // 2 x 2 output tiles per block
-    const int ntiles = (64 / (2 * b)) * tpb;
-    const int blk = tid / tpb, w = tid % tpb, r0 = 2 * (w / (b / 2)), c0 = 2 * (w % (b / 2));
-    const int o = blk * 2 * b;
-    float *Yb = Y + blk * b * b;
-    // phase 1: Y = A_10 X_00 (A_10: rows o+b.., columns o..; X_00: the upper diagonal block)
-    if (tid < ntiles) {
-      float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
-#pragma unroll 8
-      for (int l = 0; l < b; ++l) {
-        const float a0 = A[pidx(o + b + r0, o + l)], a1 = A[pidx(o + b + r0 + 1, o + l)];
-        const float2 xv = *reinterpret_cast<const float2 *>(X + (o + l) * 64 + o + c0);
-        y00 = fmaf(a0, xv.x, y00); y01 = fmaf(a0, xv.y, y01);
-        y10 = fmaf(a1, xv.x, y10); y11 = fmaf(a1, xv.y, y11);
-      }
-      *reinterpret_cast<float2 *>(Yb + r0 * b + c0) = make_float2(y00, y01);
-      *reinterpret_cast<float2 *>(Yb + (r0 + 1) * b + c0) = make_float2(y10, y11);
+    for (int r = 0; r < 32; ++r) {
+      st_tf32(sT, sw32(64, o + r, o + j), x[r] * bj);
+      *reinterpret_cast<uint32_t *>(sT + sw32(64, zr + r, o + j)) = 0u;
     }
-    __syncthreads();
-    // phase 2: X_10 = -X_11 Y (X_11: the lower diagonal block, finished earlier)
-    if (tid < ntiles) {
-      float z00 = 0.f, z01 = 0.f, z10 = 0.f, z11 = 0.f;
-#pragma unroll 8
-      for (int l = 0; l < b; ++l) {
-        const float x0 = X[(o + b + r0) * 64 + o + b + l], x1 = X[(o + b + r0 + 1) * 64 + o + b + l];
-        const float2 yv = *reinterpret_cast<const float2 *>(Yb + l * b + c0);
-        z00 = fmaf(-x0, yv.x, z00); z01 = fmaf(-x0, yv.y, z01);
-        z10 = fmaf(-x1, yv.x, z10); z11 = fmaf(-x1, yv.y, z11);
-      }
-      float *X0 = X + (o + b + r0) * 64 + o + c0;
-      *reinterpret_cast<float2 *>(X0) = make_float2(z00, z01);
-      *reinterpret_cast<float2 *>(X0 + 64) = make_float2(z10, z11);
-      const float b0 = beta[o + c0], b1 = beta[o + c0 + 1];
-      st_tf32(sT, sw32(64, o + b + r0, o + c0), z00 * b0);
-      st_tf32(sT, sw32(64, o + b + r0, o + c0 + 1), z01 * b1);
-      st_tf32(sT, sw32(64, o + b + r0 + 1, o + c0), z10 * b0);
-      st_tf32(sT, sw32(64, o + b + r0 + 1, o + c0 + 1), z11 * b1);
-    }
-    __syncthreads();
+  } else {
+#pragma unroll
+    for (int r = 0; r < 32; ++r) st_tf32(sMt, sw32(32, r, j), x[r]);
   }
 }
 
@@ -229,10 +196,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           *sP = sm + OFF_P, *sStg = sm + OFF_STG;
   float *sBeta = reinterpret_cast<float *>(sm + OFF_MISC);     // [64]
   float *sGC = sBeta + 64;                                       // [2][128] G_63, double-buffered
-  float *sXch = sGC + 256;                                       // [128]
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_MISC + 1792);
-  uint64_t *tma_bar = bars, *mma_bar = bars + 1;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_MISC + 1808);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_MISC + 1280);
+  uint64_t *tma_bar = bars, *mma_bar = bars + 1, *mma_bar2 = bars + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_MISC + 1312);
+  // [4][128] row-group products of the gate pass; T's area is free whenever the gate pass runs
+  float *sXch = reinterpret_cast<float *>(sT);
   const uint32_t sbase = smem_u32(sm);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -258,6 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     mbar_init(tma_bar, 1);
     mbar_init(mma_bar, 1);
+    mbar_init(mma_bar2, 1);
     mbar_fence_init();
   }
   if (warp == 0) tmem_alloc(tmem_slot, 512);
@@ -265,15 +234,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // TMEM lane of this thread and which half of a row it handles; the gate pass
-  // uses the same mapping (channel c = jrow, rows 32*half .. 32*half + 31).
-  const int half = warp >> 2;
+  // Thread layout: warp w reaches TMEM lanes 32*(w%4)..+31 (jrow); the four warps sharing a
+  // lane quarter split each TMEM row's columns (qg = w/4).  The gate pass uses the same
+  // mapping: channel c = jrow, rows 16*qg .. 16*qg + 15.
+  const int qg = warp >> 2;
   const int jrow = 32 * (warp & 3) + lane;
-  const int c = jrow, hf = half;
+  const int c = jrow;
   const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
 
-  uint32_t tma_phase = 0, mma_phase = 0;
-  bool tma_pending = false, mma_pending = false, failed = false, store_pending = false;
+  uint32_t tma_phase = 0, mma_phase = 0, mma2_phase = 0;
+  bool tma_pending = false, mma_pending = false, mma2_pending = false, failed = false,
+       store_pending = false;
 
   // descriptors of the fixed operand tiles (K-major, 128-byte swizzle)
   const uint64_t dKQ = smem_desc_sw128(sbase + OFF_KQ, 16, 1024);
@@ -281,6 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint64_t dKCT = smem_desc_sw128(sbase + OFF_KCT, 16, 1024);
   const uint64_t dT = smem_desc_sw128(sbase + OFF_T, 16, 1024);
   const uint64_t dP = smem_desc_sw128(sbase + OFF_P, 16, 1024);
+  const uint64_t dM = smem_desc_sw128(sbase + OFF_M, 16, 1024);
   auto dadd = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (bytes >> 4); };
 
   // one warp polls an mbarrier phase; the block then agrees on the outcome
@@ -302,78 +274,73 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const uint8_t *stq = sStg, *stk = sStg + 16384, *stv = sStg + 32768, *sta = sStg + 49152;
 
-  // ---- gate pass: staging (q, k, v, a of one chunk) -> Kr, Qr, Kc, Kc^T tiles, Kr^T and V^T
-  // in TMEM, beta, G_63.  Kc^T is left in kc[] for the caller to store (its tile may still be
-  // read by the previous chunk's last MMA group).  Returns whether the chunk is out of range.
+  // ---- gate pass: staging (q, k, v, a of one chunk) -> Kr, Qr, Kc tiles, V^T in TMEM
+  // (columns vcol..vcol+63), beta, G_63.  Kc^T is left in kc[] for the caller to store (its
+  // tile may still be read by the previous chunk's last MMA group).  Returns whether the
+  // chunk is out of range.
   float b_next = 0.f;
   if (tid < kC && t0 + tid < t1) b_next = p.b[(size_t)(bofs + t0 + tid) * H + h];
-  float kc[32];
-  auto gate_pass = [&](long cs, int nrows, float *gc_out) -> bool {
+  float kc[16];
+  auto gate_pass = [&](long cs, int nrows, float *gc_out, uint32_t vcol) -> bool {
     const float b_cur = b_next;
     if (tid < kC && cs + kC + tid < t1) b_next = p.b[(size_t)(bofs + cs + kC + tid) * H + h];
-    float g[32];
+    float g[16];
     float run = 1.f;
 #pragma unroll
-    for (int rr = 0; rr < 32; ++rr) {
-      const int r = 32 * hf + rr;
+    for (int rr = 0; rr < 16; ++rr) {
+      const int r = 16 * qg + rr;
       const float al = fast_alpha<SG>(ldbf(sta, r, c));
       run *= r < nrows ? al : 1.f;
       g[rr] = run;
     }
-    if (hf == 0) sXch[c] = run;
+    sXch[qg * 128 + c] = run;
     if (tid < kC) sBeta[tid] = tid < nrows ? fast_beta<SG>(b_cur) : 0.f;
     __syncthreads();
+    float mult = 1.f;
+#pragma unroll
+    for (int x = 0; x < 3; ++x)
+      if (x < qg) mult *= sXch[x * 128 + c];
     bool bad = false;
-    const float mult = hf ? sXch[c] : 1.f;
+    uint32_t vt[16];
 #pragma unroll
-    for (int grp = 0; grp < 2; ++grp) {
-      uint32_t krt[16], vt[16];
-#pragma unroll
-      for (int x = 0; x < 16; ++x) {
-        const int rr = 16 * grp + x, r = 32 * hf + rr;
-        const float gam = g[rr] * mult;
-        const float ag = fabsf(gam);
-        bad |= !(ag >= 0x1p-100f && ag <= 0x1p100f);
-        const float inv = __fdividef(1.f, gam);
-        // rows past the sequence end hold another sequence's tokens or TMA fill: masked
-        const bool valid = r < nrows;
-        const float q_raw = ldbf(stq, r, c), k_raw = ldbf(stk, r, c), v_raw = ldbf(stv, r, c);
-        const float qv = valid ? q_raw : 0.f, kv = valid ? k_raw : 0.f, vv = valid ? v_raw : 0.f;
-        const uint32_t kr = to_tf32(kv * gam);
-        const uint32_t kcb = to_tf32(kv * inv);
-        *reinterpret_cast<uint32_t *>(sKQ + sw32(128, r, c)) = kr;
-        st_tf32(sKQ, sw32(128, 64 + r, c), qv * gam);
-        *reinterpret_cast<uint32_t *>(sKC + sw32(64, r, c)) = kcb;
-        kc[rr] = __uint_as_float(kcb);
-        krt[x] = kr;
-        vt[x] = __float_as_uint(vv);
-        if (rr == 31 && hf == 1) gc_out[c] = gam;
-      }
-      // lane c of TMEM holds Kr^T[c][.] and V^T[c][.] (A operands of (2) and (3))
-      tmem_st16(lane_addr + COL_KRT + 32 * hf + 16 * grp, krt);
-      tmem_st16(lane_addr + COL_VT + 32 * hf + 16 * grp, vt);
+    for (int rr = 0; rr < 16; ++rr) {
+      const int r = 16 * qg + rr;
+      const float gam = g[rr] * mult;
+      const float ag = fabsf(gam);
+      bad |= !(ag >= 0x1p-100f && ag <= 0x1p100f);
+      const float inv = __fdividef(1.f, gam);
+      // rows past the sequence end hold another sequence's tokens or TMA fill: masked
+      const bool valid = r < nrows;
+      const float q_raw = ldbf(stq, r, c), k_raw = ldbf(stk, r, c), v_raw = ldbf(stv, r, c);
+      const float qv = valid ? q_raw : 0.f, kv = valid ? k_raw : 0.f, vv = valid ? v_raw : 0.f;
+      const uint32_t kcb = to_tf32(kv * inv);
+      st_tf32(sKQ, sw32(128, r, c), kv * gam);
+      st_tf32(sKQ, sw32(128, 64 + r, c), qv * gam);
+      *reinterpret_cast<uint32_t *>(sKC + sw32(64, r, c)) = kcb;
+      kc[rr] = __uint_as_float(kcb);
+      vt[rr] = __float_as_uint(vv);
+      if (rr == 15 && qg == 3) gc_out[c] = gam;
     }
+    // lane c of TMEM holds V^T[c][.] (V' = V - X is formed in place before (c))
+    tmem_st16(lane_addr + vcol + 16 * qg, vt);
     tmem_wait_st();
     return bad;
   };
   auto store_kct = [&]() {  // four consecutive t per 16-byte store
 #pragma unroll
-    for (int rr = 0; rr < 32; rr += 4)
-      *reinterpret_cast<float4 *>(sKCT + sw32(128, c, 32 * hf + rr)) =
+    for (int rr = 0; rr < 16; rr += 4)
+      *reinterpret_cast<float4 *>(sKCT + sw32(128, c, 16 * qg + rr)) =
           make_float4(kc[rr], kc[rr + 1], kc[rr + 2], kc[rr + 3]);
   };
 
-  // ---- initial state into TMEM: thread (lane j, half) holds S^T[j][64*half .. +64) = S0[i][j]
+  // ---- initial state into TMEM: thread (lane j, qg) holds S^T[j][32*qg .. +32) = S0[i][j]
   {
+    uint32_t r[32];
+    const int i0 = 32 * qg;
 #pragma unroll
-    for (int cb = 0; cb < 2; ++cb) {
-      uint32_t r[32];
-      const int i0 = 64 * half + 32 * cb;
-#pragma unroll
-      for (int x = 0; x < 32; ++x)
-        r[x] = __float_as_uint(p.S0 ? p.S0[sofs + (size_t)(i0 + x) * kD + jrow] : 0.f);
-      tmem_st32(lane_addr + COL_S + i0, r);
-    }
+    for (int x = 0; x < 32; ++x)
+      r[x] = __float_as_uint(p.S0 ? p.S0[sofs + (size_t)(i0 + x) * kD + jrow] : 0.f);
+    tmem_st32(lane_addr + COL_S + i0, r);
     tmem_wait_st();
   }
   if (tid == 0 && t1 > t0) issue_tma(t0);
@@ -389,7 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_phase ^= 1;
     tma_pending = false;
     if (!failed) {
-      const bool bad = gate_pass(t0, (int)(t1 - t0 < kC ? t1 - t0 : kC), sGC);
+      const bool bad = gate_pass(t0, (int)(t1 - t0 < kC ? t1 - t0 : kC), sGC, COL_VT);
       store_kct();
       fence_proxy_async();
       tc_fence_before();
@@ -402,23 +369,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool has_next = cs + kC < t1;
     const int nrows_next = has_next ? (int)(t1 - cs - kC < kC ? t1 - cs - kC : kC) : 0;
     float *gc_cur = sGC + 128 * gsel, *gc_next = sGC + 128 * (gsel ^ 1);
+    const uint32_t vt_cur = COL_VT + 64 * gsel, vt_next = COL_VT + 64 * (gsel ^ 1);
 
     if (slow) {
       // ------------------------------------------------------------ exact token-by-token path
-      // state S[i][j] in smem over Kr/Qr, gates over Kc, partial sums over Kc^T
+      // state S[i][j] in smem over Kr/Qr, gates over Kc, partial sums over Kc^T; thread
+      // (value channel jrow, key quarter qg) owns S[32*qg .. +32][jrow]
       float *sS = reinterpret_cast<float *>(sKQ);
       float *sAl = reinterpret_cast<float *>(sKC);
-      float *sRed = reinterpret_cast<float *>(sKCT);
+      float *sRed = reinterpret_cast<float *>(sKCT);   // [2][4][128]
+      if (tid == 0 && store_pending) bulk_wait_read();  // T/P may still feed an O store
+      store_pending = false;
 #pragma unroll 4
-      for (int rr = 0; rr < 32; ++rr) {
-        const int r = 32 * hf + rr;
+      for (int rr = 0; rr < 16; ++rr) {
+        const int r = 16 * qg + rr;
         sAl[r * kD + c] = r < nrows ? gate_alpha(ldbf(sta, r, c), SG) : 1.f;
       }
       tc_fence_after();
-#pragma unroll
-      for (int cb = 0; cb < 2; ++cb) {
+      {
         uint32_t r[32];
-        const int i0 = 64 * half + 32 * cb;
+        const int i0 = 32 * qg;
         tmem_ld32(lane_addr + COL_S + i0, r);
         tmem_wait_ld();
 #pragma unroll
@@ -427,37 +397,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncthreads();
       for (int t = 0; t < nrows; ++t) {
         float pk = 0.f;
-        for (int x = 0; x < 64; ++x) {
-          const int i = 64 * half + x;
+        for (int x = 0; x < 32; ++x) {
+          const int i = 32 * qg + x;
           const float sv = sS[i * kD + jrow] * sAl[t * kD + i];
           sS[i * kD + jrow] = sv;
           pk = fmaf(ldbf(stk, t, i), sv, pk);
         }
-        sRed[half * 128 + jrow] = pk;
+        sRed[qg * 128 + jrow] = pk;
         __syncthreads();
-        const float u = sBeta[t] * (ldbf(stv, t, jrow) - (sRed[jrow] + sRed[128 + jrow]));
+        const float ptot = (sRed[jrow] + sRed[128 + jrow]) + (sRed[256 + jrow] + sRed[384 + jrow]);
+        const float u = sBeta[t] * (ldbf(stv, t, jrow) - ptot);
         float acc = 0.f;
-        for (int x = 0; x < 64; ++x) {
-          const int i = 64 * half + x;
+        for (int x = 0; x < 32; ++x) {
+          const int i = 32 * qg + x;
           const float sv = fmaf(ldbf(stk, t, i), u, sS[i * kD + jrow]);
           sS[i * kD + jrow] = sv;
           acc = fmaf(ldbf(stq, t, i), sv, acc);
         }
-        sRed[256 + half * 128 + jrow] = acc;
+        sRed[512 + qg * 128 + jrow] = acc;
         __syncthreads();
-        if (half == 0 && o)
-          o[((size_t)(bofs + cs + t) * H + h) * kD + jrow] =
-              from_f32<TOut>(sRed[256 + jrow] + sRed[384 + jrow]);
+        if (qg == 0 && o)
+          o[((size_t)(bofs + cs + t) * H + h) * kD + jrow] = from_f32<TOut>(
+              (sRed[512 + jrow] + sRed[640 + jrow]) + (sRed[768 + jrow] + sRed[896 + jrow]));
       }
-#pragma unroll
-      for (int cb = 0; cb < 2; ++cb) {
+      {
         uint32_t r[32];
-        const int i0 = 64 * half + 32 * cb;
+        const int i0 = 32 * qg;
 #pragma unroll
         for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(sS[(i0 + x) * kD + jrow]);
         tmem_st32(lane_addr + COL_S + i0, r);
+        tmem_wait_st();
       }
-      tmem_wait_st();
       tc_fence_before();
       __syncthreads();
       if (has_next) {
@@ -466,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!block_wait(tma_bar, tma_phase)) { failed = true; break; }
         tma_phase ^= 1;
         tma_pending = false;
-        const bool bad = gate_pass(cs + kC, nrows_next, gc_next);
+        const bool bad = gate_pass(cs + kC, nrows_next, gc_next, vt_next);
         store_kct();
         fence_proxy_async();
         tc_fence_before();
@@ -476,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       continue;
     }
 
-    // ---------------------------------------------------------------- (1) [A;P] = [Kr;Qr] Kc^T
+    // ---------------------------------------------------------------- (1), then (a)
     if (tid == 0) {
       if (has_next) issue_tma(cs + kC);   // staging is free: the gate pass has consumed it
       tc_fence_after();
@@ -487,93 +457,116 @@ __global__ void __launch_bounds__(kThreads, 1)
                s > 0);
       }
       mma_commit(mma_bar);
+#pragma unroll
+      for (int s = 0; s < 16; ++s) {
+        const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
+        mma_ts(tmem + COL_X, tmem + COL_S + 8 * s, dadd(dKQ, off), IDESC_N128, s > 0);
+      }
+      mma_commit(mma_bar2);
       if (store_pending) bulk_wait_read();  // previous O tile (over T and P) has left smem
     }
     tma_pending = has_next;
     store_pending = false;
-    mma_pending = true;
+    mma_pending = mma2_pending = true;
     if (!block_wait(mma_bar, mma_phase)) { failed = true; break; }
     mma_phase ^= 1;
     mma_pending = false;
     tc_fence_after();
     // ---------------------------------------------------------------- A and P out of TMEM
-    float *sA = reinterpret_cast<float *>(sKC);           // plain [64][64], pidx layout
-    float *sX = sA + 64 * 64;                              // plain [64][64]
-    float *sY = reinterpret_cast<float *>(sKQ);           // [3][16][16] over the consumed Kr rows
+    float *sA = reinterpret_cast<float *>(sKC);           // plain [64][kAS]
     {
-      uint32_t r[32];
-      tmem_ld32(lane_addr + COL_AP + 32 * half, r);
+      uint32_t r[16];
+      tmem_ld16(lane_addr + COL_AP + 16 * qg, r);
       tmem_wait_ld();
       if (jrow < 64) {
         const int t = jrow;
         const float bt = sBeta[t];
+        float av[16];
 #pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          const int j = 32 * half + x;
-          sA[pidx(t, j)] = j < t ? __uint_as_float(r[x]) * bt : 0.f;
+        for (int x = 0; x < 16; ++x) {
+          const int j = 16 * qg + x;
+          av[x] = j < t ? __uint_as_float(r[x]) * bt : 0.f;
         }
+#pragma unroll
+        for (int y = 0; y < 4; ++y)
+          *reinterpret_cast<float4 *>(sA + t * kAS + 16 * qg + 4 * y) =
+              make_float4(av[4 * y], av[4 * y + 1], av[4 * y + 2], av[4 * y + 3]);
       } else {
         const int t = jrow - 64;
 #pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          const int j = 32 * half + x;
+        for (int x = 0; x < 16; ++x) {
+          const int j = 16 * qg + x;
           st_tf32(sP, sw32(64, t, j), j <= t ? __uint_as_float(r[x]) : 0.f);
         }
       }
     }
+    tc_fence_before();
     __syncthreads();
     // ---------------------------------------------------------------- Tm = (I + A)^{-1} Diag(beta)
-    solve_T(sA, sX, sY, sT, sBeta, tid);
-    fence_proxy_async();
-    __syncthreads();
-    // ---------------------------------------------------------------- (2) W^T, (3) U^T
-    if (tid == 0) {
+    // warps 0..2 solve; meanwhile warps 4..7 form (b) V' = V - X once (a) is done, as a
+    // round-to-nearest tf32 hi part (over V^T) and the fp32 remainder (over [A;P])
+    bool ok = true;
+    if (warp >= 4 && warp < 8) {
+      ok = mbar_wait(mma_bar2, mma2_phase, kWaitNs);
       tc_fence_after();
+      if (ok) {
+#pragma unroll 1
+        for (int qt = 0; qt < 4; ++qt) {
+          uint32_t xv[16], vv[16];
+          tmem_ld16(lane_addr + COL_X + 16 * qt, xv);
+          tmem_ld16(lane_addr + vt_cur + 16 * qt, vv);
+          tmem_wait_ld();
 #pragma unroll
-      for (int s = 0; s < 8; ++s) {
-        const uint64_t bt = dadd(dT, (s >> 2) * 8192 + (s & 3) * 32);
-        mma_ts(tmem + COL_W, tmem + COL_KRT + 8 * s, bt, IDESC_N64, s > 0);
-        mma_ts(tmem + COL_U, tmem + COL_VT + 8 * s, bt, IDESC_N64, s > 0);
+          for (int x = 0; x < 16; ++x) {
+            const float vp = __uint_as_float(vv[x]) - __uint_as_float(xv[x]);
+            const uint32_t hi = to_tf32(vp);
+            vv[x] = hi;
+            xv[x] = __float_as_uint(vp - __uint_as_float(hi));
+          }
+          tmem_st16(lane_addr + vt_cur + 16 * qt, vv);
+          tmem_st16(lane_addr + COL_LO + 16 * qt, xv);
+        }
+        tmem_wait_st();
       }
-      mma_commit(mma_bar);
-    }
-    mma_pending = true;
-    if (!block_wait(mma_bar, mma_phase)) { failed = true; break; }
-    mma_phase ^= 1;
-    mma_pending = false;
-    tc_fence_after();
-    // ---------------------------------------------------------------- W (rows t, key channels) over Kr
-    {
-      uint32_t r[32];
-      tmem_ld32(lane_addr + COL_W + 32 * half, r);
-      tmem_wait_ld();
-      const int i = jrow;
-#pragma unroll
-      for (int x = 0; x < 32; ++x) st_tf32(sKQ, sw32(128, 32 * half + x, i), __uint_as_float(r[x]));
+    } else {
+      solve_T(sA, sT, sm + OFF_M, sBeta, tid);
     }
     fence_proxy_async();
     tc_fence_before();
-    __syncthreads();
-    // ---------------------------------------------------------------- (4) U^T -= S^T W^T, (5a) O^T = S^T Qr^T
+    mma2_phase ^= 1;
+    mma2_pending = false;
+    if (!__syncthreads_and(ok)) { failed = true; break; }
+    // ---------------------------------------------------------------- (c) U^T = V'^T Tm^T
+    // round 1: U^T = V'^T Tb^T, hi and lo parts of V'
     if (tid == 0) {
       tc_fence_after();
 #pragma unroll
-      for (int s = 0; s < 16; ++s) {
-        const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
-        mma_ts(tmem + COL_U, tmem + COL_S + 8 * s, dadd(dKQ, off), IDESC_U, 1);
-      }
+      for (int s = 0; s < 8; ++s)
+        mma_ts(tmem + COL_U, tmem + vt_cur + 8 * s, dadd(dT, (s >> 2) * 8192 + (s & 3) * 32),
+               IDESC_N64, s > 0);
 #pragma unroll
-      for (int s = 0; s < 16; ++s) {
-        const uint32_t off = 8192 + (s >> 2) * 16384 + (s & 3) * 32;
-        mma_ts(tmem + COL_O, tmem + COL_S + 8 * s, dadd(dKQ, off), IDESC_N64, s > 0);
-      }
+      for (int s = 0; s < 8; ++s)
+        mma_ts(tmem + COL_U, tmem + COL_LO + 8 * s, dadd(dT, (s >> 2) * 8192 + (s & 3) * 32),
+               IDESC_N64, 1);
       mma_commit(mma_bar);
     }
     mma_pending = true;
     if (!block_wait(mma_bar, mma_phase)) { failed = true; break; }
     mma_phase ^= 1;
     mma_pending = false;
-    // ---------------------------------------------------------------- (5b) O^T += U^T P^T, (6) S^T += U^T Kc
+    // round 2: rows 32..63 of U minus M times rows 0..31 (U_top^T read from TMEM)
+    if (tid == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int s = 0; s < 4; ++s)
+        mma_ts(tmem + COL_U + 32, tmem + COL_U + 8 * s, dadd(dM, s * 32), IDESC_N32_NEG, 1);
+      mma_commit(mma_bar);
+    }
+    mma_pending = true;
+    if (!block_wait(mma_bar, mma_phase)) { failed = true; break; }
+    mma_phase ^= 1;
+    mma_pending = false;
+    // ---------------------------------------------------------------- (d) O^T += U^T P^T, S^T += U^T Kc
     if (tid == 0) {
       tc_fence_after();
 #pragma unroll
@@ -583,18 +576,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int s = 0; s < 8; ++s)
         mma_ts(tmem + COL_S, tmem + COL_U + 8 * s, dadd(dKCT, (s >> 2) * 16384 + (s & 3) * 32),
-               IDESC_S, 1);
+               IDESC_N128, 1);
       mma_commit(mma_bar);
     }
     mma_pending = true;
     // ---------------------------------------------------------------- next chunk's gate pass,
-    // overlapping (5b)/(6): Kr, Qr and Kc are free, Kc^T is not (kept in registers)
+    // overlapping (d): Kr, Qr, Kc, T and M are free, Kc^T is not (kept in registers)
     bool bad_next = false;
     if (has_next) {
       if (!block_wait(tma_bar, tma_phase)) { failed = true; break; }
       tma_phase ^= 1;
       tma_pending = false;
-      bad_next = gate_pass(cs + kC, nrows_next, gc_next);
+      bad_next = gate_pass(cs + kC, nrows_next, gc_next, vt_next);
     }
     if (!block_wait(mma_bar, mma_phase)) { failed = true; break; }
     mma_phase ^= 1;
@@ -603,31 +596,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------------- O out; S^T columns scaled by G_63
     {
       uint32_t r[32];
-      tmem_ld32(lane_addr + COL_O + 32 * half, r);
+      tmem_ld16(lane_addr + COL_O + 16 * qg, *reinterpret_cast<uint32_t(*)[16]>(r));
       tmem_wait_ld();
       if (o && nrows == kC) {
         // full chunk: O [t][j] staged over T and P, written by one TMA store
         TOut *sO = reinterpret_cast<TOut *>(sT);
 #pragma unroll
-        for (int x = 0; x < 32; ++x)
-          sO[(32 * half + x) * kD + jrow] = from_f32<TOut>(__uint_as_float(r[x]));
+        for (int x = 0; x < 16; ++x)
+          sO[(16 * qg + x) * kD + jrow] = from_f32<TOut>(__uint_as_float(r[x]));
       } else if (o) {
 #pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          const int t = 32 * half + x;
+        for (int x = 0; x < 16; ++x) {
+          const int t = 16 * qg + x;
           if (t < nrows)
             o[((size_t)(bofs + cs + t) * H + h) * kD + jrow] = from_f32<TOut>(__uint_as_float(r[x]));
         }
       }
+      const int i0 = 32 * qg;
+      tmem_ld32(lane_addr + COL_S + i0, r);
+      tmem_wait_ld();
 #pragma unroll
-      for (int cb = 0; cb < 2; ++cb) {
-        const int i0 = 64 * half + 32 * cb;
-        tmem_ld32(lane_addr + COL_S + i0, r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * gc_cur[i0 + x]);
-        tmem_st32(lane_addr + COL_S + i0, r);
-      }
+      for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * gc_cur[i0 + x]);
+      tmem_st32(lane_addr + COL_S + i0, r);
       tmem_wait_st();
     }
     if (has_next) store_kct();
@@ -649,18 +639,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {
       if (tma_pending) mbar_wait(tma_bar, tma_phase, kWaitNs);
       if (mma_pending) mbar_wait(mma_bar, mma_phase, kWaitNs);
+      if (mma2_pending) mbar_wait(mma_bar2, mma2_phase, kWaitNs);
     }
   } else if (p.S_T) {
     tc_fence_after();
+    uint32_t r[32];
+    const int i0 = 32 * qg;
+    tmem_ld32(lane_addr + COL_S + i0, r);
+    tmem_wait_ld();
 #pragma unroll
-    for (int cb = 0; cb < 2; ++cb) {
-      uint32_t r[32];
-      const int i0 = 64 * half + 32 * cb;
-      tmem_ld32(lane_addr + COL_S + i0, r);
-      tmem_wait_ld();
-#pragma unroll
-      for (int x = 0; x < 32; ++x) p.S_T[sofs + (size_t)(i0 + x) * kD + jrow] = __uint_as_float(r[x]);
-    }
+    for (int x = 0; x < 32; ++x) p.S_T[sofs + (size_t)(i0 + x) * kD + jrow] = __uint_as_float(r[x]);
   }
   tc_fence_before();
   __syncthreads();
@@ -752,9 +740,3 @@ int launch_chunk_tc(const ChunkArgs &g, cudaStream_t s) {
 }
 
 }  // namespace ckda
-
-extern "C" int ckda_timed_solve(unsigned long long *out) {
-}
-
-extern "C" int ckda_timed_phases(unsigned long long *out) {
-}
