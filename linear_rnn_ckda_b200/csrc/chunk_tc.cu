@@ -46,18 +46,21 @@ using namespace sm100;
 
 constexpr int kC = 64;      // chunk rows
 constexpr int kD = 128;     // dk = dv
-constexpr int kThreads = 512;   // 16 warps: 4 per scheduler to hide latency
+constexpr int kCompute = 512;               // 16 compute warps: 4 per scheduler
+constexpr int kThreads = kCompute + 32;     // + one warp that issues TMA loads and MMAs
+constexpr int kBarC = 1;                    // named barrier of the compute warps
 
 // shared memory map (bytes from a 1024-aligned base)
 constexpr uint32_t OFF_KQ = 0;          // [Kr;Qr] 128 rows x 128 fp32, 4 column blocks of 16 KB
 constexpr uint32_t OFF_KC = 65536;      // Kc 64 rows x 128 fp32, 4 column blocks of 8 KB;
-                                        // then the solve's A (64 x kAS) and the M tile
+                                        // then the solve's A (64 x kAS), the M tile and the
+                                        // gate pass's exchange (from +24576)
 constexpr uint32_t OFF_KCT = 98304;     // Kc^T 128 rows x 64 fp32, 2 column blocks of 16 KB
 constexpr uint32_t OFF_T = 131072;      // Tm 64 x 64 fp32, 2 column blocks of 8 KB; T and P together
 constexpr uint32_t OFF_P = 147456;      // P  64 x 64 fp32 (2 blocks); T+P stage O for its TMA store
 constexpr uint32_t OFF_M = OFF_KC + 18432;   // M = X2 A21, 32 x 32 tf32 (one column block)
 constexpr uint32_t OFF_STG = 163840;    // TMA staging: q, k, v, a bf16 64 x 128 (16 KB each)
-constexpr uint32_t OFF_MISC = 229376;   // beta[64], gC[2][128], barriers, tmem slot
+constexpr uint32_t OFF_MISC = 229376;   // beta[64], gC[2][128], barriers, tmem slot, abort flag
 constexpr uint32_t kSmemUsed = OFF_MISC + 2048;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;  // + alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -139,7 +142,7 @@ constexpr int kAS = 68;
 // stride kAS, zeros on and above the diagonal).  In 32 x 32 blocks
 //   I + A = [[L1, 0], [A21, L2]],  (I + A)^{-1} = [[X1, 0], [-M X1, X2]],
 //   X1 = L1^{-1},  X2 = L2^{-1},  M = X2 A21.
-// X1, X2 and M are three independent forward substitutions (warps 0, 1, 2):
+// X1, X2 and M are three independent forward substitutions (warps 1, 2, 3):
 // lane j keeps column j in registers and finishes the rows in order, reading
 // each row of the triangular factor as a broadcast; all fp32.  Written as tf32:
 // the block-diagonal part Tb = blockdiag(X1, X2) Diag(beta) into the T tile
@@ -148,16 +151,16 @@ constexpr int kAS = 68;
 // 32 + 32), U_top = Ub_top and U_bot = Ub_bot - M U_top, a second MMA round.
 __device__ __forceinline__ void solve_T(const float *A, uint8_t *sT, uint8_t *sMt,
                                         const float *beta, int tid) {
-  const int warp = tid >> 5, lane = tid & 31;
-  if (warp >= 3) return;
+  const int role = (tid >> 5) - 1, lane = tid & 31;   // 0: X1, 1: X2, 2: M
+  if (role < 0 || role > 2) return;
   const int j = lane;
-  const int o = warp == 0 ? 0 : 32;   // the diagonal block solved by this warp
+  const int o = role == 0 ? 0 : 32;   // the diagonal block solved by this warp
   float x[32];
 #pragma unroll
   for (int r = 0; r < 32; ++r) {
     const float *row = A + (o + r) * kAS + o;
     // right-hand side: column j of the identity (X1, X2) or of A21 (M)
-    float acc0 = warp == 2 ? A[(32 + r) * kAS + j] : (r == j ? 1.f : 0.f);
+    float acc0 = role == 2 ? A[(32 + r) * kAS + j] : (r == j ? 1.f : 0.f);
     float acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
 #pragma unroll
     for (int l4 = 0; l4 < r; l4 += 4) {
@@ -169,7 +172,7 @@ __device__ __forceinline__ void solve_T(const float *A, uint8_t *sT, uint8_t *sM
     }
     x[r] = (acc0 + acc1) + (acc2 + acc3);
   }
-  if (warp < 2) {
+  if (role < 2) {
     // Tb: column o + j of the diagonal block, zeros in the same column of the other block row
     const float bj = beta[o + j];
     const int zr = 32 - o;
@@ -197,10 +200,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   float *sBeta = reinterpret_cast<float *>(sm + OFF_MISC);     // [64]
   float *sGC = sBeta + 64;                                       // [2][128] G_63, double-buffered
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_MISC + 1280);
-  uint64_t *tma_bar = bars, *mma_bar = bars + 1, *mma_bar2 = bars + 2;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_MISC + 1312);
-  // [4][128] row-group products of the gate pass; T's area is free whenever the gate pass runs
-  float *sXch = reinterpret_cast<float *>(sT);
+  // completion (TMA or tcgen05.commit): staging, (1), (a), rounds 1/2 of (c), (d), all MMAs
+  uint64_t *bar_tma = bars, *bar_mma1 = bars + 1, *bar_a = bars + 2, *bar_r = bars + 3,
+           *bar_d = bars + 4, *bar_fin = bars + 5;
+  // compute warps -> issuer (one arrival per compute warp): a chunk's tiles are ready and
+  // it takes the fast path (rdy1) or the token-by-token path (rdy_slow); S is final and
+  // TMEM O is free (rdy2); Tm, M, P and V' are ready (rdy3)
+  uint64_t *rdy1 = bars + 6, *rdy_slow = bars + 7, *rdy2 = bars + 8, *rdy3 = bars + 9;
+  // issuer -> compute warps: a token-by-token announcement has been consumed (so the next
+  // announcement cannot be mistaken for it)
+  uint64_t *bar_ack = bars + 10;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_MISC + 1376);
+  volatile int *sAbort = reinterpret_cast<volatile int *>(sm + OFF_MISC + 1380);
   const uint32_t sbase = smem_u32(sm);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -224,9 +235,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   TOut *o = static_cast<TOut *>(p.o);
 
   if (tid == 0) {
-    mbar_init(tma_bar, 1);
-    mbar_init(mma_bar, 1);
-    mbar_init(mma_bar2, 1);
+    for (int x = 0; x < 6; ++x) mbar_init(bars + x, 1);
+    for (int x = 6; x < 10; ++x) mbar_init(bars + x, kCompute / 32);
+    mbar_init(bar_ack, 1);
+    *sAbort = 0;
     mbar_fence_init();
   }
   if (warp == 0) tmem_alloc(tmem_slot, 512);
@@ -234,17 +246,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // Thread layout: warp w reaches TMEM lanes 32*(w%4)..+31 (jrow); the four warps sharing a
-  // lane quarter split each TMEM row's columns (qg = w/4).  The gate pass uses the same
-  // mapping: channel c = jrow, rows 16*qg .. 16*qg + 15.
-  const int qg = warp >> 2;
-  const int jrow = 32 * (warp & 3) + lane;
-  const int c = jrow;
-  const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
-
-  uint32_t tma_phase = 0, mma_phase = 0, mma2_phase = 0;
-  bool tma_pending = false, mma_pending = false, mma2_pending = false, failed = false,
-       store_pending = false;
 
   // descriptors of the fixed operand tiles (K-major, 128-byte swizzle)
   const uint64_t dKQ = smem_desc_sw128(sbase + OFF_KQ, 16, 1024);
@@ -255,400 +256,450 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint64_t dM = smem_desc_sw128(sbase + OFF_M, 16, 1024);
   auto dadd = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (bytes >> 4); };
 
-  // one warp polls an mbarrier phase; the block then agrees on the outcome
-  auto block_wait = [&](uint64_t *bar, uint32_t parity) -> bool {
-    bool ok = true;
-    if (warp == 0) ok = mbar_wait(bar, parity, kWaitNs);
-    return __syncthreads_and(ok) != 0;
-  };
   auto issue_tma = [&](long cs) {
-    mbar_arrive_expect_tx(tma_bar, 4 * 2 * 8192);
+    mbar_arrive_expect_tx(bar_tma, 4 * 2 * 8192);
     const int row = (int)(bofs + cs);
     const CUtensorMap *maps[4] = {&tm_q, &tm_k, &tm_v, &tm_a};
 #pragma unroll
     for (int x = 0; x < 4; ++x)
 #pragma unroll
       for (int bx = 0; bx < 2; ++bx)
-        tma_load_3d(sStg + x * 16384 + bx * 8192, maps[x], tma_bar, bx * 64, h, row);
+        tma_load_3d(sStg + x * 16384 + bx * 8192, maps[x], bar_tma, bx * 64, h, row);
   };
 
-  const uint8_t *stq = sStg, *stk = sStg + 16384, *stv = sStg + 32768, *sta = sStg + 49152;
-
-  // ---- gate pass: staging (q, k, v, a of one chunk) -> Kr, Qr, Kc tiles, V^T in TMEM
-  // (columns vcol..vcol+63), beta, G_63.  Kc^T is left in kc[] for the caller to store (its
-  // tile may still be read by the previous chunk's last MMA group).  Returns whether the
-  // chunk is out of range.
-  float b_next = 0.f;
-  if (tid < kC && t0 + tid < t1) b_next = p.b[(size_t)(bofs + t0 + tid) * H + h];
-  float kc[16];
-  auto gate_pass = [&](long cs, int nrows, float *gc_out, uint32_t vcol) -> bool {
-    const float b_cur = b_next;
-    if (tid < kC && cs + kC + tid < t1) b_next = p.b[(size_t)(bofs + cs + kC + tid) * H + h];
-    float g[16];
-    float run = 1.f;
+  if (warp == kCompute / 32) {
+    // ================================================================ issuer (one thread)
+    // Walks the chunks in order and issues each fast chunk's products as soon as their
+    // operands are announced, so that no compute warp ever waits in an MMA issue queue.
+    if (lane == 0) {
+      uint32_t ph1 = 0, phs = 0, ph2 = 0, ph3 = 0, phr = 0;
+      bool ok = true;
+      for (long cs = t0; cs < t1 && ok; cs += kC) {
+        // which path does this chunk take?
+        bool fast = false;
+        {
+          const uint64_t w0 = globaltimer();
+          for (;;) {
+            if (mbar_try_wait(rdy1, ph1)) { fast = true; ph1 ^= 1; break; }
+            if (mbar_try_wait(rdy_slow, phs)) {
+              phs ^= 1;
+              mbar_arrive(bar_ack);
+              break;
+            }
+            if (*sAbort || globaltimer() - w0 > kWaitNs) { ok = false; break; }
+          }
+        }
+        if (!ok || !fast) continue;
+        // (1) [A;P] = [Kr;Qr] Kc^T, and the staging load of the next chunk (staging is
+        // free: this chunk's gate pass has consumed it)
+        if (cs + kC < t1) issue_tma(cs + kC);
+        tc_fence_after();
 #pragma unroll
-    for (int rr = 0; rr < 16; ++rr) {
-      const int r = 16 * qg + rr;
-      const float al = fast_alpha<SG>(ldbf(sta, r, c));
-      run *= r < nrows ? al : 1.f;
-      g[rr] = run;
+        for (int s = 0; s < 16; ++s) {
+          const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
+          mma_ss(tmem + COL_AP, dadd(dKQ, off), dadd(dKC, (s >> 2) * 8192 + (s & 3) * 32),
+                 IDESC_N64, s > 0);
+        }
+        mma_commit(bar_mma1);
+        // (a) [X^T|O^T] = S^T [Kr;Qr]^T
+        if (!(ok = mbar_wait_or_abort(rdy2, ph2, kWaitNs, sAbort))) break;
+        ph2 ^= 1;
+        tc_fence_after();
+#pragma unroll
+        for (int s = 0; s < 16; ++s) {
+          const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
+          mma_ts(tmem + COL_X, tmem + COL_S + 8 * s, dadd(dKQ, off), IDESC_N128, s > 0);
+        }
+        mma_commit(bar_a);
+        // (c) round 1: U^T = V'^T Tb^T, hi and lo parts of V'
+        if (!(ok = mbar_wait_or_abort(rdy3, ph3, kWaitNs, sAbort))) break;
+        ph3 ^= 1;
+        const uint32_t vt_cur = COL_VT + 64 * (uint32_t)(((cs - t0) / kC) & 1);
+        tc_fence_after();
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+          mma_ts(tmem + COL_U, tmem + vt_cur + 8 * s, dadd(dT, (s >> 2) * 8192 + (s & 3) * 32),
+                 IDESC_N64, s > 0);
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+          mma_ts(tmem + COL_U, tmem + COL_LO + 8 * s, dadd(dT, (s >> 2) * 8192 + (s & 3) * 32),
+                 IDESC_N64, 1);
+        mma_commit(bar_r);
+        // round 2: rows 32..63 of U minus M times rows 0..31 (U_top^T read from TMEM)
+        if (!(ok = mbar_wait_or_abort(bar_r, phr, kWaitNs, sAbort))) break;
+        phr ^= 1;
+        tc_fence_after();
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+          mma_ts(tmem + COL_U + 32, tmem + COL_U + 8 * s, dadd(dM, s * 32), IDESC_N32_NEG, 1);
+        mma_commit(bar_r);
+        // (d) O^T += U^T P^T, S^T += U^T Kc
+        if (!(ok = mbar_wait_or_abort(bar_r, phr, kWaitNs, sAbort))) break;
+        phr ^= 1;
+        tc_fence_after();
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+          mma_ts(tmem + COL_O, tmem + COL_U + 8 * s, dadd(dP, (s >> 2) * 8192 + (s & 3) * 32),
+                 IDESC_N64, 1);
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+          mma_ts(tmem + COL_S, tmem + COL_U + 8 * s, dadd(dKCT, (s >> 2) * 16384 + (s & 3) * 32),
+                 IDESC_N128, 1);
+        mma_commit(bar_d);
+      }
+      if (!ok) *sAbort = 1;
+      // every MMA issued above has finished before TMEM is released
+      mma_commit(bar_fin);
+      mbar_wait(bar_fin, 0, kWaitNs);
     }
-    sXch[qg * 128 + c] = run;
-    if (tid < kC) sBeta[tid] = tid < nrows ? fast_beta<SG>(b_cur) : 0.f;
-    __syncthreads();
-    float mult = 1.f;
-#pragma unroll
-    for (int x = 0; x < 3; ++x)
-      if (x < qg) mult *= sXch[x * 128 + c];
-    bool bad = false;
-    uint32_t vt[16];
-#pragma unroll
-    for (int rr = 0; rr < 16; ++rr) {
-      const int r = 16 * qg + rr;
-      const float gam = g[rr] * mult;
-      const float ag = fabsf(gam);
-      bad |= !(ag >= 0x1p-100f && ag <= 0x1p100f);
-      const float inv = __fdividef(1.f, gam);
-      // rows past the sequence end hold another sequence's tokens or TMA fill: masked
-      const bool valid = r < nrows;
-      const float q_raw = ldbf(stq, r, c), k_raw = ldbf(stk, r, c), v_raw = ldbf(stv, r, c);
-      const float qv = valid ? q_raw : 0.f, kv = valid ? k_raw : 0.f, vv = valid ? v_raw : 0.f;
-      const uint32_t kcb = to_tf32(kv * inv);
-      st_tf32(sKQ, sw32(128, r, c), kv * gam);
-      st_tf32(sKQ, sw32(128, 64 + r, c), qv * gam);
-      *reinterpret_cast<uint32_t *>(sKC + sw32(64, r, c)) = kcb;
-      kc[rr] = __uint_as_float(kcb);
-      vt[rr] = __float_as_uint(vv);
-      if (rr == 15 && qg == 3) gc_out[c] = gam;
-    }
-    // lane c of TMEM holds V^T[c][.] (V' = V - X is formed in place before (c))
-    tmem_st16(lane_addr + vcol + 16 * qg, vt);
-    tmem_wait_st();
-    return bad;
-  };
-  auto store_kct = [&]() {  // four consecutive t per 16-byte store
-#pragma unroll
-    for (int rr = 0; rr < 16; rr += 4)
-      *reinterpret_cast<float4 *>(sKCT + sw32(128, c, 16 * qg + rr)) =
-          make_float4(kc[rr], kc[rr + 1], kc[rr + 2], kc[rr + 3]);
-  };
+    __syncwarp();
+  } else {
+    // ================================================================ compute warps 0..15
+    // Warp w reaches TMEM lanes 32*(w%4)..+31 (jrow); the four warps sharing a lane
+    // quarter split each TMEM row's columns (qg = w/4).  The gate pass uses the same
+    // mapping: channel c = jrow, rows 16*qg .. 16*qg + 15.
+    const int qg = warp >> 2;
+    const int jrow = 32 * (warp & 3) + lane;
+    const int c = jrow;
+    const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+    uint32_t tma_ph = 0, mma1_ph = 0, a_ph = 0, d_ph = 0, ack_ph = 0;
+    bool failed = false, store_pending = false;
 
-  // ---- initial state into TMEM: thread (lane j, qg) holds S^T[j][32*qg .. +32) = S0[i][j]
-  {
-    uint32_t r[32];
-    const int i0 = 32 * qg;
+    auto csync = [&]() { bar_sync(kBarC, kCompute); };
+    // warp 0 polls a completion barrier; the compute warps then agree on the outcome
+    auto cwait = [&](uint64_t *bar, uint32_t &ph) -> bool {
+      bool ok = true;
+      if (warp == 0) ok = mbar_wait_or_abort(bar, ph, kWaitNs, sAbort);
+      ph ^= 1;
+      return bar_and(kBarC, kCompute, ok);
+    };
+    // one arrival per warp, after the whole warp's writes (each thread fenced its own)
+    auto announce = [&](uint64_t *bar) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar);
+    };
+
+    const uint8_t *stq = sStg, *stk = sStg + 16384, *stv = sStg + 32768, *sta = sStg + 49152;
+
+    // ---- gate pass: staging (q, k, v, a of one chunk) -> Kr, Qr tiles, V^T in TMEM
+    // (columns vcol..vcol+63), beta, G_63.  Kc stays in kc[] until store_kc() writes the Kc
+    // and Kc^T tiles, whose previous contents the running chunk may still be reading.
+    // Returns whether the chunk is out of range.
+    float *sXch = reinterpret_cast<float *>(sKC + 24576);   // [4][128], past the solve's data
+    float b_next = 0.f;
+    if (tid < kC && t0 + tid < t1) b_next = p.b[(size_t)(bofs + t0 + tid) * H + h];
+    float kc[16];
+    auto gate_pass = [&](long cs, int nrows, float *gc_out, uint32_t vcol) -> bool {
+      const float b_cur = b_next;
+      if (tid < kC && cs + kC + tid < t1) b_next = p.b[(size_t)(bofs + cs + kC + tid) * H + h];
+      float g[16];
+      float run = 1.f;
 #pragma unroll
-    for (int x = 0; x < 32; ++x)
-      r[x] = __float_as_uint(p.S0 ? p.S0[sofs + (size_t)(i0 + x) * kD + jrow] : 0.f);
-    tmem_st32(lane_addr + COL_S + i0, r);
-    tmem_wait_st();
-  }
-  if (tid == 0 && t1 > t0) issue_tma(t0);
-  tma_pending = t1 > t0;
-  tc_fence_before();
-  __syncthreads();
-
-  // gate pass of the first chunk
-  int gsel = 0;              // sGC buffer of the chunk being processed
-  bool slow = false;
-  if (t1 > t0) {
-    if (!block_wait(tma_bar, tma_phase)) failed = true;
-    tma_phase ^= 1;
-    tma_pending = false;
-    if (!failed) {
-      const bool bad = gate_pass(t0, (int)(t1 - t0 < kC ? t1 - t0 : kC), sGC, COL_VT);
-      store_kct();
-      fence_proxy_async();
-      tc_fence_before();
-      slow = __syncthreads_or(bad) != 0;
-    }
-  }
-
-  for (long cs = t0; cs < t1 && !failed; cs += kC) {
-    const int nrows = (int)(t1 - cs < kC ? t1 - cs : kC);
-    const bool has_next = cs + kC < t1;
-    const int nrows_next = has_next ? (int)(t1 - cs - kC < kC ? t1 - cs - kC : kC) : 0;
-    float *gc_cur = sGC + 128 * gsel, *gc_next = sGC + 128 * (gsel ^ 1);
-    const uint32_t vt_cur = COL_VT + 64 * gsel, vt_next = COL_VT + 64 * (gsel ^ 1);
-
-    if (slow) {
-      // ------------------------------------------------------------ exact token-by-token path
-      // state S[i][j] in smem over Kr/Qr, gates over Kc, partial sums over Kc^T; thread
-      // (value channel jrow, key quarter qg) owns S[32*qg .. +32][jrow]
-      float *sS = reinterpret_cast<float *>(sKQ);
-      float *sAl = reinterpret_cast<float *>(sKC);
-      float *sRed = reinterpret_cast<float *>(sKCT);   // [2][4][128]
-      if (tid == 0 && store_pending) bulk_wait_read();  // T/P may still feed an O store
-      store_pending = false;
-#pragma unroll 4
       for (int rr = 0; rr < 16; ++rr) {
         const int r = 16 * qg + rr;
-        sAl[r * kD + c] = r < nrows ? gate_alpha(ldbf(sta, r, c), SG) : 1.f;
+        const float al = fast_alpha<SG>(ldbf(sta, r, c));
+        run *= r < nrows ? al : 1.f;
+        g[rr] = run;
       }
+      sXch[qg * 128 + c] = run;
+      if (tid < kC) sBeta[tid] = tid < nrows ? fast_beta<SG>(b_cur) : 0.f;
+      csync();
+      float mult = 1.f;
+#pragma unroll
+      for (int x = 0; x < 3; ++x)
+        if (x < qg) mult *= sXch[x * 128 + c];
+      bool bad = false;
+      uint32_t vt[16];
+#pragma unroll
+      for (int rr = 0; rr < 16; ++rr) {
+        const int r = 16 * qg + rr;
+        const float gam = g[rr] * mult;
+        const float ag = fabsf(gam);
+        bad |= !(ag >= 0x1p-100f && ag <= 0x1p100f);
+        const float inv = __fdividef(1.f, gam);
+        // rows past the sequence end hold another sequence's tokens or TMA fill: masked
+        const bool valid = r < nrows;
+        const float q_raw = ldbf(stq, r, c), k_raw = ldbf(stk, r, c), v_raw = ldbf(stv, r, c);
+        const float qv = valid ? q_raw : 0.f, kv = valid ? k_raw : 0.f, vv = valid ? v_raw : 0.f;
+        st_tf32(sKQ, sw32(128, r, c), kv * gam);
+        st_tf32(sKQ, sw32(128, 64 + r, c), qv * gam);
+        kc[rr] = __uint_as_float(to_tf32(kv * inv));
+        vt[rr] = __float_as_uint(vv);
+        if (rr == 15 && qg == 3) gc_out[c] = gam;
+      }
+      // lane c of TMEM holds V^T[c][.] (V' = V - X is formed in place before (c))
+      tmem_st16(lane_addr + vcol + 16 * qg, vt);
+      tmem_wait_st();
+      return bad;
+    };
+    auto store_kc = [&]() {  // Kc (row t, channel c); Kc^T (row c, four t per 16-byte store)
+#pragma unroll
+      for (int rr = 0; rr < 16; ++rr)
+        *reinterpret_cast<float *>(sKC + sw32(64, 16 * qg + rr, c)) = kc[rr];
+#pragma unroll
+      for (int rr = 0; rr < 16; rr += 4)
+        *reinterpret_cast<float4 *>(sKCT + sw32(128, c, 16 * qg + rr)) =
+            make_float4(kc[rr], kc[rr + 1], kc[rr + 2], kc[rr + 3]);
+    };
+    // tiles of the next chunk written: tell the issuer which path it takes
+    auto announce_chunk = [&](bool is_slow) {
+      fence_proxy_async();
+      tc_fence_before();
+      announce(is_slow ? rdy_slow : rdy1);
+    };
+
+    // ---- initial state into TMEM: thread (lane j, qg) holds S^T[j][32*qg .. +32) = S0[i][j]
+    {
+      uint32_t r[32];
+      const int i0 = 32 * qg;
+#pragma unroll
+      for (int x = 0; x < 32; ++x)
+        r[x] = __float_as_uint(p.S0 ? p.S0[sofs + (size_t)(i0 + x) * kD + jrow] : 0.f);
+      tmem_st32(lane_addr + COL_S + i0, r);
+      tmem_wait_st();
+    }
+    if (tid == 0 && t1 > t0) issue_tma(t0);
+    csync();
+
+    // gate pass of the first chunk
+    int gsel = 0;              // sGC / V^T buffer of the chunk being processed
+    bool slow = false;
+    if (t1 > t0) {
+      if (!cwait(bar_tma, tma_ph)) {
+        failed = true;
+      } else {
+        const bool bad = gate_pass(t0, (int)(t1 - t0 < kC ? t1 - t0 : kC), sGC, COL_VT);
+        store_kc();
+        slow = bar_or(kBarC, kCompute, bad);
+        announce_chunk(slow);
+        if (!slow) announce(rdy2);
+      }
+    }
+
+    for (long cs = t0; cs < t1 && !failed; cs += kC) {
+      const int nrows = (int)(t1 - cs < kC ? t1 - cs : kC);
+      const bool has_next = cs + kC < t1;
+      const int nrows_next = has_next ? (int)(t1 - cs - kC < kC ? t1 - cs - kC : kC) : 0;
+      float *gc_cur = sGC + 128 * gsel, *gc_next = sGC + 128 * (gsel ^ 1);
+      const uint32_t vt_cur = COL_VT + 64 * gsel, vt_next = COL_VT + 64 * (gsel ^ 1);
+
+      if (slow) {
+        // ------------------------------------------------------------ exact token-by-token path
+        // state S[i][j] in smem over Kr/Qr, gates over Kc, partial sums over Kc^T; thread
+        // (value channel jrow, key quarter qg) owns S[32*qg .. +32][jrow]
+        float *sS = reinterpret_cast<float *>(sKQ);
+        float *sAl = reinterpret_cast<float *>(sKC);
+        float *sRed = reinterpret_cast<float *>(sKCT);   // [2][4][128]
+        if (tid == 0 && store_pending) bulk_wait_read();  // T/P may still feed an O store
+        store_pending = false;
+#pragma unroll 4
+        for (int rr = 0; rr < 16; ++rr) {
+          const int r = 16 * qg + rr;
+          sAl[r * kD + c] = r < nrows ? gate_alpha(ldbf(sta, r, c), SG) : 1.f;
+        }
+        tc_fence_after();
+        {
+          uint32_t r[32];
+          const int i0 = 32 * qg;
+          tmem_ld32(lane_addr + COL_S + i0, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int x = 0; x < 32; ++x) sS[(i0 + x) * kD + jrow] = __uint_as_float(r[x]);
+        }
+        csync();
+        for (int t = 0; t < nrows; ++t) {
+          float pk = 0.f;
+          for (int x = 0; x < 32; ++x) {
+            const int i = 32 * qg + x;
+            const float sv = sS[i * kD + jrow] * sAl[t * kD + i];
+            sS[i * kD + jrow] = sv;
+            pk = fmaf(ldbf(stk, t, i), sv, pk);
+          }
+          sRed[qg * 128 + jrow] = pk;
+          csync();
+          const float ptot =
+              (sRed[jrow] + sRed[128 + jrow]) + (sRed[256 + jrow] + sRed[384 + jrow]);
+          const float u = sBeta[t] * (ldbf(stv, t, jrow) - ptot);
+          float acc = 0.f;
+          for (int x = 0; x < 32; ++x) {
+            const int i = 32 * qg + x;
+            const float sv = fmaf(ldbf(stk, t, i), u, sS[i * kD + jrow]);
+            sS[i * kD + jrow] = sv;
+            acc = fmaf(ldbf(stq, t, i), sv, acc);
+          }
+          sRed[512 + qg * 128 + jrow] = acc;
+          csync();
+          if (qg == 0 && o)
+            o[((size_t)(bofs + cs + t) * H + h) * kD + jrow] = from_f32<TOut>(
+                (sRed[512 + jrow] + sRed[640 + jrow]) + (sRed[768 + jrow] + sRed[896 + jrow]));
+        }
+        {
+          uint32_t r[32];
+          const int i0 = 32 * qg;
+#pragma unroll
+          for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(sS[(i0 + x) * kD + jrow]);
+          tmem_st32(lane_addr + COL_S + i0, r);
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        csync();
+        if (has_next) {
+          if (tid == 0) issue_tma(cs + kC);
+          if (!cwait(bar_tma, tma_ph)) { failed = true; break; }
+          const bool bad = gate_pass(cs + kC, nrows_next, gc_next, vt_next);
+          store_kc();
+          slow = bar_or(kBarC, kCompute, bad);
+          if (!cwait(bar_ack, ack_ph)) { failed = true; break; }   // this chunk's announcement seen
+          announce_chunk(slow);
+          if (!slow) announce(rdy2);
+          gsel ^= 1;
+        }
+        continue;
+      }
+
+      // ---------------------------------------------------------------- (1)
+      // issued by the issuer once this chunk was announced
+      if (tid == 0 && store_pending) bulk_wait_read();  // previous O tile (over T and P) has left
+      store_pending = false;
+      if (!cwait(bar_mma1, mma1_ph)) { failed = true; break; }
       tc_fence_after();
+      // ---------------------------------------------------------------- A and P out of TMEM
+      float *sA = reinterpret_cast<float *>(sKC);           // plain [64][kAS]
+      {
+        uint32_t r[16];
+        tmem_ld16(lane_addr + COL_AP + 16 * qg, r);
+        tmem_wait_ld();
+        if (jrow < 64) {
+          const int t = jrow;
+          const float bt = sBeta[t];
+          float av[16];
+#pragma unroll
+          for (int x = 0; x < 16; ++x) {
+            const int j = 16 * qg + x;
+            av[x] = j < t ? __uint_as_float(r[x]) * bt : 0.f;
+          }
+#pragma unroll
+          for (int y = 0; y < 4; ++y)
+            *reinterpret_cast<float4 *>(sA + t * kAS + 16 * qg + 4 * y) =
+                make_float4(av[4 * y], av[4 * y + 1], av[4 * y + 2], av[4 * y + 3]);
+        } else {
+          const int t = jrow - 64;
+#pragma unroll
+          for (int x = 0; x < 16; ++x) {
+            const int j = 16 * qg + x;
+            st_tf32(sP, sw32(64, t, j), j <= t ? __uint_as_float(r[x]) : 0.f);
+          }
+        }
+      }
+      tc_fence_before();
+      csync();
+      // ---------------------------------------------------------------- Tm = (I + A)^{-1} Diag(beta)
+      // warps 1..3 solve; meanwhile warps 4..7 form (b) V' = V - X once (a) is done, as a
+      // round-to-nearest tf32 hi part (over V^T) and the fp32 remainder (over [A;P])
+      bool ok = true;
+      if (warp >= 4 && warp < 8) {
+        ok = mbar_wait_or_abort(bar_a, a_ph, kWaitNs, sAbort);
+        tc_fence_after();
+        if (ok) {
+#pragma unroll 1
+          for (int qt = 0; qt < 4; ++qt) {
+            uint32_t xv[16], vv[16];
+            tmem_ld16(lane_addr + COL_X + 16 * qt, xv);
+            tmem_ld16(lane_addr + vt_cur + 16 * qt, vv);
+            tmem_wait_ld();
+#pragma unroll
+            for (int x = 0; x < 16; ++x) {
+              const float vp = __uint_as_float(vv[x]) - __uint_as_float(xv[x]);
+              const uint32_t hi = to_tf32(vp);
+              vv[x] = hi;
+              xv[x] = __float_as_uint(vp - __uint_as_float(hi));
+            }
+            tmem_st16(lane_addr + vt_cur + 16 * qt, vv);
+            tmem_st16(lane_addr + COL_LO + 16 * qt, xv);
+          }
+          tmem_wait_st();
+        }
+      } else {
+        solve_T(sA, sT, sm + OFF_M, sBeta, tid);
+      }
+      a_ph ^= 1;
+      fence_proxy_async();
+      tc_fence_before();
+      if (!bar_and(kBarC, kCompute, ok)) { failed = true; break; }
+      announce(rdy3);
+      // ---------------------------------------------------------------- next chunk's gate pass,
+      // overlapping (c) and (d): Kr, Qr are free ((a) is done); Kc and Kc^T are stored
+      // after (d)
+      bool bad_next = false;
+      if (has_next) {
+        if (!cwait(bar_tma, tma_ph)) { failed = true; break; }
+        bad_next = gate_pass(cs + kC, nrows_next, gc_next, vt_next);
+      }
+      if (!cwait(bar_d, d_ph)) { failed = true; break; }
+      tc_fence_after();
+      if (has_next) {
+        store_kc();
+        slow = bar_or(kBarC, kCompute, bad_next);
+        announce_chunk(slow);   // (1) of the next chunk runs under this chunk's read-out
+      }
+      // ---------------------------------------------------------------- O out; S^T columns scaled by G_63
       {
         uint32_t r[32];
+        tmem_ld16(lane_addr + COL_O + 16 * qg, *reinterpret_cast<uint32_t(*)[16]>(r));
+        tmem_wait_ld();
+        if (o && nrows == kC) {
+          // full chunk: O [t][j] staged over T and P, written by one TMA store
+          TOut *sO = reinterpret_cast<TOut *>(sT);
+#pragma unroll
+          for (int x = 0; x < 16; ++x)
+            sO[(16 * qg + x) * kD + jrow] = from_f32<TOut>(__uint_as_float(r[x]));
+        } else if (o) {
+#pragma unroll
+          for (int x = 0; x < 16; ++x) {
+            const int t = 16 * qg + x;
+            if (t < nrows)
+              o[((size_t)(bofs + cs + t) * H + h) * kD + jrow] =
+                  from_f32<TOut>(__uint_as_float(r[x]));
+          }
+        }
         const int i0 = 32 * qg;
         tmem_ld32(lane_addr + COL_S + i0, r);
         tmem_wait_ld();
 #pragma unroll
-        for (int x = 0; x < 32; ++x) sS[(i0 + x) * kD + jrow] = __uint_as_float(r[x]);
-      }
-      __syncthreads();
-      for (int t = 0; t < nrows; ++t) {
-        float pk = 0.f;
-        for (int x = 0; x < 32; ++x) {
-          const int i = 32 * qg + x;
-          const float sv = sS[i * kD + jrow] * sAl[t * kD + i];
-          sS[i * kD + jrow] = sv;
-          pk = fmaf(ldbf(stk, t, i), sv, pk);
-        }
-        sRed[qg * 128 + jrow] = pk;
-        __syncthreads();
-        const float ptot = (sRed[jrow] + sRed[128 + jrow]) + (sRed[256 + jrow] + sRed[384 + jrow]);
-        const float u = sBeta[t] * (ldbf(stv, t, jrow) - ptot);
-        float acc = 0.f;
-        for (int x = 0; x < 32; ++x) {
-          const int i = 32 * qg + x;
-          const float sv = fmaf(ldbf(stk, t, i), u, sS[i * kD + jrow]);
-          sS[i * kD + jrow] = sv;
-          acc = fmaf(ldbf(stq, t, i), sv, acc);
-        }
-        sRed[512 + qg * 128 + jrow] = acc;
-        __syncthreads();
-        if (qg == 0 && o)
-          o[((size_t)(bofs + cs + t) * H + h) * kD + jrow] = from_f32<TOut>(
-              (sRed[512 + jrow] + sRed[640 + jrow]) + (sRed[768 + jrow] + sRed[896 + jrow]));
-      }
-      {
-        uint32_t r[32];
-        const int i0 = 32 * qg;
-#pragma unroll
-        for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(sS[(i0 + x) * kD + jrow]);
+        for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * gc_cur[i0 + x]);
         tmem_st32(lane_addr + COL_S + i0, r);
         tmem_wait_st();
       }
+      fence_proxy_async();
       tc_fence_before();
-      __syncthreads();
-      if (has_next) {
-        if (tid == 0) issue_tma(cs + kC);
-        tma_pending = true;
-        if (!block_wait(tma_bar, tma_phase)) { failed = true; break; }
-        tma_phase ^= 1;
-        tma_pending = false;
-        const bool bad = gate_pass(cs + kC, nrows_next, gc_next, vt_next);
-        store_kct();
-        fence_proxy_async();
-        tc_fence_before();
-        slow = __syncthreads_or(bad) != 0;
-        gsel ^= 1;
+      if (has_next && !slow) announce(rdy2);   // S final, TMEM O free: (a) may run
+      csync();
+      if (tid == 0 && o && nrows == kC) {
+        tma_store_3d(&tm_o, sT, 0, h, (int)(bofs + cs));
+        bulk_commit();
+        store_pending = true;
       }
-      continue;
+      gsel ^= 1;
     }
+    if (tid == 0) bulk_wait_all();
 
-    // ---------------------------------------------------------------- (1), then (a)
-    if (tid == 0) {
-      if (has_next) issue_tma(cs + kC);   // staging is free: the gate pass has consumed it
-      tc_fence_after();
-#pragma unroll
-      for (int s = 0; s < 16; ++s) {
-        const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
-        mma_ss(tmem + COL_AP, dadd(dKQ, off), dadd(dKC, (s >> 2) * 8192 + (s & 3) * 32), IDESC_N64,
-               s > 0);
+    if (failed) {
+      if (tid == 0) {
+        set_status(p.status, CKDA_ERR_TIMEOUT);
+        *sAbort = 1;
       }
-      mma_commit(mma_bar);
-#pragma unroll
-      for (int s = 0; s < 16; ++s) {
-        const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
-        mma_ts(tmem + COL_X, tmem + COL_S + 8 * s, dadd(dKQ, off), IDESC_N128, s > 0);
-      }
-      mma_commit(mma_bar2);
-      if (store_pending) bulk_wait_read();  // previous O tile (over T and P) has left smem
-    }
-    tma_pending = has_next;
-    store_pending = false;
-    mma_pending = mma2_pending = true;
-    if (!block_wait(mma_bar, mma_phase)) { failed = true; break; }
-    mma_phase ^= 1;
-    mma_pending = false;
-    tc_fence_after();
-    // ---------------------------------------------------------------- A and P out of TMEM
-    float *sA = reinterpret_cast<float *>(sKC);           // plain [64][kAS]
-    {
-      uint32_t r[16];
-      tmem_ld16(lane_addr + COL_AP + 16 * qg, r);
-      tmem_wait_ld();
-      if (jrow < 64) {
-        const int t = jrow;
-        const float bt = sBeta[t];
-        float av[16];
-#pragma unroll
-        for (int x = 0; x < 16; ++x) {
-          const int j = 16 * qg + x;
-          av[x] = j < t ? __uint_as_float(r[x]) * bt : 0.f;
-        }
-#pragma unroll
-        for (int y = 0; y < 4; ++y)
-          *reinterpret_cast<float4 *>(sA + t * kAS + 16 * qg + 4 * y) =
-              make_float4(av[4 * y], av[4 * y + 1], av[4 * y + 2], av[4 * y + 3]);
-      } else {
-        const int t = jrow - 64;
-#pragma unroll
-        for (int x = 0; x < 16; ++x) {
-          const int j = 16 * qg + x;
-          st_tf32(sP, sw32(64, t, j), j <= t ? __uint_as_float(r[x]) : 0.f);
-        }
-      }
-    }
-    tc_fence_before();
-    __syncthreads();
-    // ---------------------------------------------------------------- Tm = (I + A)^{-1} Diag(beta)
-    // warps 0..2 solve; meanwhile warps 4..7 form (b) V' = V - X once (a) is done, as a
-    // round-to-nearest tf32 hi part (over V^T) and the fp32 remainder (over [A;P])
-    bool ok = true;
-    if (warp >= 4 && warp < 8) {
-      ok = mbar_wait(mma_bar2, mma2_phase, kWaitNs);
+      // a staging load may still be in flight: let it land (bounded) before leaving
+      if (tid == 0) mbar_wait(bar_tma, tma_ph, kWaitNs);
+    } else if (p.S_T) {
       tc_fence_after();
-      if (ok) {
-#pragma unroll 1
-        for (int qt = 0; qt < 4; ++qt) {
-          uint32_t xv[16], vv[16];
-          tmem_ld16(lane_addr + COL_X + 16 * qt, xv);
-          tmem_ld16(lane_addr + vt_cur + 16 * qt, vv);
-          tmem_wait_ld();
-#pragma unroll
-          for (int x = 0; x < 16; ++x) {
-            const float vp = __uint_as_float(vv[x]) - __uint_as_float(xv[x]);
-            const uint32_t hi = to_tf32(vp);
-            vv[x] = hi;
-            xv[x] = __float_as_uint(vp - __uint_as_float(hi));
-          }
-          tmem_st16(lane_addr + vt_cur + 16 * qt, vv);
-          tmem_st16(lane_addr + COL_LO + 16 * qt, xv);
-        }
-        tmem_wait_st();
-      }
-    } else {
-      solve_T(sA, sT, sm + OFF_M, sBeta, tid);
-    }
-    fence_proxy_async();
-    tc_fence_before();
-    mma2_phase ^= 1;
-    mma2_pending = false;
-    if (!__syncthreads_and(ok)) { failed = true; break; }
-    // ---------------------------------------------------------------- (c) U^T = V'^T Tm^T
-    // round 1: U^T = V'^T Tb^T, hi and lo parts of V'
-    if (tid == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int s = 0; s < 8; ++s)
-        mma_ts(tmem + COL_U, tmem + vt_cur + 8 * s, dadd(dT, (s >> 2) * 8192 + (s & 3) * 32),
-               IDESC_N64, s > 0);
-#pragma unroll
-      for (int s = 0; s < 8; ++s)
-        mma_ts(tmem + COL_U, tmem + COL_LO + 8 * s, dadd(dT, (s >> 2) * 8192 + (s & 3) * 32),
-               IDESC_N64, 1);
-      mma_commit(mma_bar);
-    }
-    mma_pending = true;
-    if (!block_wait(mma_bar, mma_phase)) { failed = true; break; }
-    mma_phase ^= 1;
-    mma_pending = false;
-    // round 2: rows 32..63 of U minus M times rows 0..31 (U_top^T read from TMEM)
-    if (tid == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int s = 0; s < 4; ++s)
-        mma_ts(tmem + COL_U + 32, tmem + COL_U + 8 * s, dadd(dM, s * 32), IDESC_N32_NEG, 1);
-      mma_commit(mma_bar);
-    }
-    mma_pending = true;
-    if (!block_wait(mma_bar, mma_phase)) { failed = true; break; }
-    mma_phase ^= 1;
-    mma_pending = false;
-    // ---------------------------------------------------------------- (d) O^T += U^T P^T, S^T += U^T Kc
-    if (tid == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int s = 0; s < 8; ++s)
-        mma_ts(tmem + COL_O, tmem + COL_U + 8 * s, dadd(dP, (s >> 2) * 8192 + (s & 3) * 32),
-               IDESC_N64, 1);
-#pragma unroll
-      for (int s = 0; s < 8; ++s)
-        mma_ts(tmem + COL_S, tmem + COL_U + 8 * s, dadd(dKCT, (s >> 2) * 16384 + (s & 3) * 32),
-               IDESC_N128, 1);
-      mma_commit(mma_bar);
-    }
-    mma_pending = true;
-    // ---------------------------------------------------------------- next chunk's gate pass,
-    // overlapping (d): Kr, Qr, Kc, T and M are free, Kc^T is not (kept in registers)
-    bool bad_next = false;
-    if (has_next) {
-      if (!block_wait(tma_bar, tma_phase)) { failed = true; break; }
-      tma_phase ^= 1;
-      tma_pending = false;
-      bad_next = gate_pass(cs + kC, nrows_next, gc_next, vt_next);
-    }
-    if (!block_wait(mma_bar, mma_phase)) { failed = true; break; }
-    mma_phase ^= 1;
-    mma_pending = false;
-    tc_fence_after();
-    // ---------------------------------------------------------------- O out; S^T columns scaled by G_63
-    {
       uint32_t r[32];
-      tmem_ld16(lane_addr + COL_O + 16 * qg, *reinterpret_cast<uint32_t(*)[16]>(r));
-      tmem_wait_ld();
-      if (o && nrows == kC) {
-        // full chunk: O [t][j] staged over T and P, written by one TMA store
-        TOut *sO = reinterpret_cast<TOut *>(sT);
-#pragma unroll
-        for (int x = 0; x < 16; ++x)
-          sO[(16 * qg + x) * kD + jrow] = from_f32<TOut>(__uint_as_float(r[x]));
-      } else if (o) {
-#pragma unroll
-        for (int x = 0; x < 16; ++x) {
-          const int t = 16 * qg + x;
-          if (t < nrows)
-            o[((size_t)(bofs + cs + t) * H + h) * kD + jrow] = from_f32<TOut>(__uint_as_float(r[x]));
-        }
-      }
       const int i0 = 32 * qg;
       tmem_ld32(lane_addr + COL_S + i0, r);
       tmem_wait_ld();
 #pragma unroll
-      for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * gc_cur[i0 + x]);
-      tmem_st32(lane_addr + COL_S + i0, r);
-      tmem_wait_st();
+      for (int x = 0; x < 32; ++x)
+        p.S_T[sofs + (size_t)(i0 + x) * kD + jrow] = __uint_as_float(r[x]);
     }
-    if (has_next) store_kct();
-    fence_proxy_async();
-    tc_fence_before();
-    slow = __syncthreads_or(bad_next) != 0;
-    if (tid == 0 && o && nrows == kC) {
-      tma_store_3d(&tm_o, sT, 0, h, (int)(bofs + cs));
-      bulk_commit();
-      store_pending = true;
-    }
-    gsel ^= 1;
-  }
-  if (tid == 0) bulk_wait_all();
-
-  if (failed) {
-    if (tid == 0) set_status(p.status, CKDA_ERR_TIMEOUT);
-    // let in-flight copies and MMAs drain (bounded) before giving TMEM back
-    if (warp == 0) {
-      if (tma_pending) mbar_wait(tma_bar, tma_phase, kWaitNs);
-      if (mma_pending) mbar_wait(mma_bar, mma_phase, kWaitNs);
-      if (mma2_pending) mbar_wait(mma_bar2, mma2_phase, kWaitNs);
-    }
-  } else if (p.S_T) {
-    tc_fence_after();
-    uint32_t r[32];
-    const int i0 = 32 * qg;
-    tmem_ld32(lane_addr + COL_S + i0, r);
-    tmem_wait_ld();
-#pragma unroll
-    for (int x = 0; x < 32; ++x) p.S_T[sofs + (size_t)(i0 + x) * kD + jrow] = __uint_as_float(r[x]);
   }
   tc_fence_before();
   __syncthreads();
