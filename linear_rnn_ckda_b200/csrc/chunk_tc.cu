@@ -18,7 +18,7 @@
 //   (a) [X^T|O^T] = S^T [Kr;Qr]^T       N=128 (X = Kr S, and O's first term), K=128
 //   (b) V' = V - X in fp32 (threads), kept in TMEM as tf32 hi + lo parts
 //   (c) U^T     = V'^T Tm^T              A = V'^T in TMEM (hi and lo), K=64, in two rounds
-//   (d) O^T    += U^T P^T,  S^T += U^T Kc, then S^T columns scaled by G_63 (threads, in TMEM)
+//   (d) [O^T|S^T] += U^T [P;Kc^T]^T     N=192, then S^T columns scaled by G_63 (threads)
 // (1) and (a) need only the chunk's inputs and S, so they are issued together
 // when the chunk starts, and (b) overlaps the solve.  All MMAs are kind::tf32
 // with fp32 accumulation and K-major operands; smem operands are rounded to
@@ -55,10 +55,11 @@ constexpr uint32_t OFF_KQ = 0;          // [Kr;Qr] 128 rows x 128 fp32, 4 column
 constexpr uint32_t OFF_KC = 65536;      // Kc 64 rows x 128 fp32, 4 column blocks of 8 KB;
                                         // then the solve's A (64 x kAS), the M tile and the
                                         // gate pass's exchange (from +24576)
-constexpr uint32_t OFF_KCT = 98304;     // Kc^T 128 rows x 64 fp32, 2 column blocks of 16 KB
-constexpr uint32_t OFF_T = 131072;      // Tm 64 x 64 fp32, 2 column blocks of 8 KB; T and P together
-constexpr uint32_t OFF_P = 147456;      // P  64 x 64 fp32 (2 blocks); T+P stage O for its TMA store
 constexpr uint32_t OFF_M = OFF_KC + 18432;   // M = X2 A21, 32 x 32 tf32 (one column block)
+constexpr uint32_t OFF_PK = 98304;      // [P; Kc^T]: 64 + 128 rows x 64 fp32, the B operand of
+                                        // (d); each 32-column block holds P's 64 rows and then
+                                        // Kc^T's 128 rows (24 KB)
+constexpr uint32_t OFF_T = 147456;      // Tm 64 x 64 fp32, 2 column blocks of 8 KB; bf16 O staging
 constexpr uint32_t OFF_STG = 163840;    // TMA staging: q, k, v, a bf16 64 x 128 (16 KB each)
 constexpr uint32_t OFF_MISC = 229376;   // beta[64], gC[2][128], barriers, tmem slot, abort flag
 constexpr uint32_t kSmemUsed = OFF_MISC + 2048;
@@ -66,14 +67,16 @@ constexpr uint32_t kSmemBytes = kSmemUsed + 1024;  // + alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 // TMEM columns (all 512 allocated)
-// [A;P] and, once read out, the lo part of V'; X = Kr S and O adjacent (one N = 128
-// product); V^T (then the hi part of V') of two chunks at COL_VT and COL_VT + 64
-constexpr uint32_t COL_S = 0, COL_AP = 128, COL_LO = 128, COL_X = 192, COL_O = 256, COL_U = 320,
-                   COL_VT = 384;
+// [A;P] and, once read out, the lo part of V'; X, O and S adjacent so that (a) writes
+// [X|O] and (d) writes [O|S] as single products; V^T (then the hi part of V') of two
+// chunks in COL_VT0 and COL_VT1
+constexpr uint32_t COL_U = 0, COL_VT0 = 64, COL_AP = 128, COL_LO = 128, COL_X = 192, COL_O = 256,
+                   COL_S = 320, COL_VT1 = 448;
 
 constexpr uint32_t IDESC_N64 = idesc_tf32(128, 64, false, false);         // (1), (c), O += U P^T
 constexpr uint32_t IDESC_N32_NEG = idesc_tf32(128, 32, false, false, true);  // (c) second round
-constexpr uint32_t IDESC_N128 = idesc_tf32(128, 128, false, false);       // (a), S^T += U^T Kc
+constexpr uint32_t IDESC_N128 = idesc_tf32(128, 128, false, false);       // (a)
+constexpr uint32_t IDESC_N192 = idesc_tf32(128, 192, false, false);       // (d)
 
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s bound on any single wait
 
@@ -99,6 +102,11 @@ __device__ __forceinline__ uint32_t swbf(int r, int c) {
 }
 __device__ __forceinline__ float ldbf(const uint8_t *tile, int r, int c) {
   return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(tile + swbf(r, c)));
+}
+// byte offset of fp32 element (r, c) of the [P; Kc^T] tile (r < 64: P, else Kc^T row r - 64)
+__device__ __forceinline__ uint32_t swpk(int r, int c) {
+  return (uint32_t)((c >> 5) * 24576 + r * 128 + ((((c & 31) >> 2) ^ (r & 7)) << 4) +
+                    ((c & 3) << 2));
 }
 __device__ __forceinline__ void st_tf32(uint8_t *tile, uint32_t off, float x) {
   *reinterpret_cast<uint32_t *>(tile + off) = to_tf32(x);
@@ -195,8 +203,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t *sKQ = sm + OFF_KQ, *sKC = sm + OFF_KC, *sKCT = sm + OFF_KCT, *sT = sm + OFF_T,
-          *sP = sm + OFF_P, *sStg = sm + OFF_STG;
+  uint8_t *sKQ = sm + OFF_KQ, *sKC = sm + OFF_KC, *sPK = sm + OFF_PK, *sT = sm + OFF_T,
+          *sStg = sm + OFF_STG;
   float *sBeta = reinterpret_cast<float *>(sm + OFF_MISC);     // [64]
   float *sGC = sBeta + 64;                                       // [2][128] G_63, double-buffered
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_MISC + 1280);
@@ -250,9 +258,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // descriptors of the fixed operand tiles (K-major, 128-byte swizzle)
   const uint64_t dKQ = smem_desc_sw128(sbase + OFF_KQ, 16, 1024);
   const uint64_t dKC = smem_desc_sw128(sbase + OFF_KC, 16, 1024);
-  const uint64_t dKCT = smem_desc_sw128(sbase + OFF_KCT, 16, 1024);
+  const uint64_t dPK = smem_desc_sw128(sbase + OFF_PK, 16, 1024);
   const uint64_t dT = smem_desc_sw128(sbase + OFF_T, 16, 1024);
-  const uint64_t dP = smem_desc_sw128(sbase + OFF_P, 16, 1024);
   const uint64_t dM = smem_desc_sw128(sbase + OFF_M, 16, 1024);
   auto dadd = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (bytes >> 4); };
 
@@ -314,7 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // (c) round 1: U^T = V'^T Tb^T, hi and lo parts of V'
         if (!(ok = mbar_wait_or_abort(rdy3, ph3, kWaitNs, sAbort))) break;
         ph3 ^= 1;
-        const uint32_t vt_cur = COL_VT + 64 * (uint32_t)(((cs - t0) / kC) & 1);
+        const uint32_t vt_cur = (((cs - t0) / kC) & 1) ? COL_VT1 : COL_VT0;
         tc_fence_after();
 #pragma unroll
         for (int s = 0; s < 8; ++s)
@@ -333,18 +340,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < 4; ++s)
           mma_ts(tmem + COL_U + 32, tmem + COL_U + 8 * s, dadd(dM, s * 32), IDESC_N32_NEG, 1);
         mma_commit(bar_r);
-        // (d) O^T += U^T P^T, S^T += U^T Kc
+        // (d) [O^T|S^T] += U^T [P;Kc^T]^T
         if (!(ok = mbar_wait_or_abort(bar_r, phr, kWaitNs, sAbort))) break;
         phr ^= 1;
         tc_fence_after();
 #pragma unroll
         for (int s = 0; s < 8; ++s)
-          mma_ts(tmem + COL_O, tmem + COL_U + 8 * s, dadd(dP, (s >> 2) * 8192 + (s & 3) * 32),
-                 IDESC_N64, 1);
-#pragma unroll
-        for (int s = 0; s < 8; ++s)
-          mma_ts(tmem + COL_S, tmem + COL_U + 8 * s, dadd(dKCT, (s >> 2) * 16384 + (s & 3) * 32),
-                 IDESC_N128, 1);
+          mma_ts(tmem + COL_O, tmem + COL_U + 8 * s, dadd(dPK, (s >> 2) * 24576 + (s & 3) * 32),
+                 IDESC_N192, 1);
         mma_commit(bar_d);
       }
       if (!ok) *sAbort = 1;
@@ -363,6 +366,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int c = jrow;
     const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
     uint32_t tma_ph = 0, mma1_ph = 0, a_ph = 0, d_ph = 0, ack_ph = 0;
+    // bf16 O (16 KB per chunk) is staged in T's tile and written by one TMA store;
+    // fp32 O is written directly from registers
+    constexpr bool kTmaStoreO = sizeof(TOut) == 2;
     bool failed = false, store_pending = false;
 
     auto csync = [&]() { bar_sync(kBarC, kCompute); };
@@ -384,43 +390,64 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- gate pass: staging (q, k, v, a of one chunk) -> Kr, Qr tiles, V^T in TMEM
     // (columns vcol..vcol+63), beta, G_63.  Kc stays in kc[] until store_kc() writes the Kc
     // and Kc^T tiles, whose previous contents the running chunk may still be reading.
-    // Returns whether the chunk is out of range.
-    float *sXch = reinterpret_cast<float *>(sKC + 24576);   // [4][128], past the solve's data
+    // Returns whether the chunk is out of range.  Range: for KDA and CKDA every |alpha| <= 1,
+    // so |G_t| never grows within the chunk and the last row decides (a NaN gate propagates
+    // to it); raw gates are checked at every row.
+    float *sXch = reinterpret_cast<float *>(sKC + 24576);    // [4][128], past the solve's data
+    float *sXchI = reinterpret_cast<float *>(sKC + 26624);   // [4][128] inverse products (KDA)
     float b_next = 0.f;
     if (tid < kC && t0 + tid < t1) b_next = p.b[(size_t)(bofs + t0 + tid) * H + h];
     float kc[16];
-    auto gate_pass = [&](long cs, int nrows, float *gc_out, uint32_t vcol) -> bool {
-      const float b_cur = b_next;
-      if (tid < kC && cs + kC + tid < t1) b_next = p.b[(size_t)(bofs + cs + kC + tid) * H + h];
-      float g[16];
-      float run = 1.f;
+    auto gate_core = [&](int nrows, float *gc_out, uint32_t vcol) -> bool {
+      float g[16], ig[16];
+      float run = 1.f, irun = 1.f;
 #pragma unroll
       for (int rr = 0; rr < 16; ++rr) {
         const int r = 16 * qg + rr;
-        const float al = fast_alpha<SG>(ldbf(sta, r, c));
-        run *= r < nrows ? al : 1.f;
+        const float a = ldbf(sta, r, c);
+        float al, ial = 1.f;
+        if (SG == 0) {
+          // sigma(a) and its inverse 1 + e^{-a} from one exponential
+          const float e = __expf(-a);
+          ial = 1.f + e;
+          al = __fdividef(1.f, ial);
+        } else {
+          al = fast_alpha<SG>(a);
+        }
+        if (r >= nrows) al = ial = 1.f;
+        run *= al;
         g[rr] = run;
+        if (SG == 0) {
+          irun *= ial;
+          ig[rr] = irun;
+        }
       }
       sXch[qg * 128 + c] = run;
-      if (tid < kC) sBeta[tid] = tid < nrows ? fast_beta<SG>(b_cur) : 0.f;
+      if (SG == 0) sXchI[qg * 128 + c] = irun;
       csync();
-      float mult = 1.f;
+      float mult = 1.f, imult = 1.f;
 #pragma unroll
       for (int x = 0; x < 3; ++x)
-        if (x < qg) mult *= sXch[x * 128 + c];
+        if (x < qg) {
+          mult *= sXch[x * 128 + c];
+          if (SG == 0) imult *= sXchI[x * 128 + c];
+        }
       bool bad = false;
       uint32_t vt[16];
 #pragma unroll
       for (int rr = 0; rr < 16; ++rr) {
         const int r = 16 * qg + rr;
         const float gam = g[rr] * mult;
-        const float ag = fabsf(gam);
-        bad |= !(ag >= 0x1p-100f && ag <= 0x1p100f);
-        const float inv = __fdividef(1.f, gam);
-        // rows past the sequence end hold another sequence's tokens or TMA fill: masked
-        const bool valid = r < nrows;
-        const float q_raw = ldbf(stq, r, c), k_raw = ldbf(stk, r, c), v_raw = ldbf(stv, r, c);
-        const float qv = valid ? q_raw : 0.f, kv = valid ? k_raw : 0.f, vv = valid ? v_raw : 0.f;
+        if (SG == 2 || (rr == 15 && qg == 3)) {
+          const float ag = fabsf(gam);
+          bad |= !(ag >= 0x1p-100f && ag <= 0x1p100f);
+        }
+        const float inv = SG == 0 ? ig[rr] * imult : __fdividef(1.f, gam);
+        float qv = ldbf(stq, r, c), kv = ldbf(stk, r, c), vv = ldbf(stv, r, c);
+        if (r >= nrows) {
+          // rows past the sequence end hold another sequence's tokens or TMA fill
+          qv = kv = vv = 0.f;
+        }
         st_tf32(sKQ, sw32(128, r, c), kv * gam);
         st_tf32(sKQ, sw32(128, 64 + r, c), qv * gam);
         kc[rr] = __uint_as_float(to_tf32(kv * inv));
@@ -432,13 +459,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_st();
       return bad;
     };
+    auto gate_pass = [&](long cs, int nrows, float *gc_out, uint32_t vcol) -> bool {
+      const float b_cur = b_next;
+      if (tid < kC && cs + kC + tid < t1) b_next = p.b[(size_t)(bofs + cs + kC + tid) * H + h];
+      if (tid < kC) sBeta[tid] = tid < nrows ? fast_beta<SG>(b_cur) : 0.f;
+      return gate_core(nrows, gc_out, vcol);
+    };
     auto store_kc = [&]() {  // Kc (row t, channel c); Kc^T (row c, four t per 16-byte store)
 #pragma unroll
       for (int rr = 0; rr < 16; ++rr)
         *reinterpret_cast<float *>(sKC + sw32(64, 16 * qg + rr, c)) = kc[rr];
 #pragma unroll
       for (int rr = 0; rr < 16; rr += 4)
-        *reinterpret_cast<float4 *>(sKCT + sw32(128, c, 16 * qg + rr)) =
+        *reinterpret_cast<float4 *>(sPK + swpk(64 + c, 16 * qg + rr)) =
             make_float4(kc[rr], kc[rr + 1], kc[rr + 2], kc[rr + 3]);
     };
     // tiles of the next chunk written: tell the issuer which path it takes
@@ -468,7 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!cwait(bar_tma, tma_ph)) {
         failed = true;
       } else {
-        const bool bad = gate_pass(t0, (int)(t1 - t0 < kC ? t1 - t0 : kC), sGC, COL_VT);
+        const bool bad = gate_pass(t0, (int)(t1 - t0 < kC ? t1 - t0 : kC), sGC, COL_VT0);
         store_kc();
         slow = bar_or(kBarC, kCompute, bad);
         announce_chunk(slow);
@@ -481,16 +514,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool has_next = cs + kC < t1;
       const int nrows_next = has_next ? (int)(t1 - cs - kC < kC ? t1 - cs - kC : kC) : 0;
       float *gc_cur = sGC + 128 * gsel, *gc_next = sGC + 128 * (gsel ^ 1);
-      const uint32_t vt_cur = COL_VT + 64 * gsel, vt_next = COL_VT + 64 * (gsel ^ 1);
+      const uint32_t vt_cur = gsel ? COL_VT1 : COL_VT0, vt_next = gsel ? COL_VT0 : COL_VT1;
 
       if (slow) {
         // ------------------------------------------------------------ exact token-by-token path
-        // state S[i][j] in smem over Kr/Qr, gates over Kc, partial sums over Kc^T; thread
+        // state S[i][j] in smem over Kr/Qr, gates over Kc, partial sums over [P;Kc^T]; thread
         // (value channel jrow, key quarter qg) owns S[32*qg .. +32][jrow]
         float *sS = reinterpret_cast<float *>(sKQ);
         float *sAl = reinterpret_cast<float *>(sKC);
-        float *sRed = reinterpret_cast<float *>(sKCT);   // [2][4][128]
-        if (tid == 0 && store_pending) bulk_wait_read();  // T/P may still feed an O store
+        float *sRed = reinterpret_cast<float *>(sPK);    // [2][4][128]
+        if (tid == 0 && store_pending) bulk_wait_read();  // T may still feed an O store
         store_pending = false;
 #pragma unroll 4
         for (int rr = 0; rr < 16; ++rr) {
@@ -559,7 +592,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       // ---------------------------------------------------------------- (1)
       // issued by the issuer once this chunk was announced
-      if (tid == 0 && store_pending) bulk_wait_read();  // previous O tile (over T and P) has left
+      if (tid == 0 && store_pending) bulk_wait_read();  // previous O tile (over T) has left
       store_pending = false;
       if (!cwait(bar_mma1, mma1_ph)) { failed = true; break; }
       tc_fence_after();
@@ -587,7 +620,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int x = 0; x < 16; ++x) {
             const int j = 16 * qg + x;
-            st_tf32(sP, sw32(64, t, j), j <= t ? __uint_as_float(r[x]) : 0.f);
+            st_tf32(sPK, swpk(t, j), j <= t ? __uint_as_float(r[x]) : 0.f);
           }
         }
       }
@@ -647,8 +680,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t r[32];
         tmem_ld16(lane_addr + COL_O + 16 * qg, *reinterpret_cast<uint32_t(*)[16]>(r));
         tmem_wait_ld();
-        if (o && nrows == kC) {
-          // full chunk: O [t][j] staged over T and P, written by one TMA store
+        if (kTmaStoreO && o && nrows == kC) {
+          // full chunk: O [t][j] staged over T, written by one TMA store
           TOut *sO = reinterpret_cast<TOut *>(sT);
 #pragma unroll
           for (int x = 0; x < 16; ++x)
@@ -674,7 +707,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       if (has_next && !slow) announce(rdy2);   // S final, TMEM O free: (a) may run
       csync();
-      if (tid == 0 && o && nrows == kC) {
+      if (kTmaStoreO && tid == 0 && o && nrows == kC) {
         tma_store_3d(&tm_o, sT, 0, h, (int)(bofs + cs));
         bulk_commit();
         store_pending = true;
