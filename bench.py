@@ -37,6 +37,7 @@ from linear_rnn_ckda_b200 import synth  # noqa: E402
 
 PREFILL = synth.KDA_STD
 DECODE = synth.DECODE
+SPREAD = synth.CKDA_SPREAD
 
 # Algorithmic counts per unit (d = dk = dv = 128, chunk C = 64):
 #   prefill FLOP per token-head = 6 d^2 + C (3 dk + 2 dv) + C^2 / 3
@@ -273,9 +274,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--decode-steps", type=int, default=None,
                     help="timed decode steps (default: --steps rounded up to the 128-step cycle)")
-    ap.add_argument("--legs", default="prefill,e2e,decode",
-                    help="comma list of legs to run (prefill, e2e, decode); a profiling run can "
-                         "select one, the default runs all")
+    ap.add_argument("--legs", default="prefill,e2e,ckda,decode",
+                    help="comma list of legs to run (prefill, e2e, ckda, decode); a profiling "
+                         "run can select one, the default runs all")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -358,6 +359,44 @@ def main():
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
     del dd, pin, o_host, S_host
 
+    # ------------------------------------------------------------ CKDA legs
+    # the same kernel in signed-gate (CKDA) mode: on the KDA shapes and inputs (the throughput
+    # ratio the pages quote as 96-97%), and on the CKDA spread-init workload
+    ckda = None
+    if "ckda" in legs:
+        csteps = max(3, min(args.steps, 10))
+
+        def prefill_ckda():
+            ops.chunk_fwd(d["q"], d["k"], d["v"], d["a"], d["b"], None, None, chunk=w.chunk,
+                          signed_gate=1, o=o, S_T=S_T, workspace=ws)
+
+        ms_k = max_over_ranks(time_loop(prefill, csteps, args.warmup, world, stream), world)
+        ms_c = max_over_ranks(time_loop(prefill_ckda, csteps, args.warmup, world, stream), world)
+        if ops.workspace_status(ws) != 0:
+            raise RuntimeError("device status after the CKDA leg")
+        ws_ = SPREAD
+        hs = synth.make_prefill(ws_, seed=rank)
+        ds = {k: (None if v is None else v.to(dev)) for k, v in hs.items()}
+        os_ = torch.empty((ws_.B, ws_.T, ws_.H, ws_.dv), dtype=torch.bfloat16, device=dev)
+        Ss = torch.empty((ws_.n_seqs, ws_.H, ws_.dk, ws_.dv), dtype=torch.float32, device=dev)
+        wss = ops.new_workspace(ws_.B, ws_.T, ws_.H, ws_.dk, ws_.dv, ws_.chunk, 0, dev)
+
+        def spread():
+            ops.chunk_fwd(ds["q"], ds["k"], ds["v"], ds["a"], ds["b"], ds["S0"], None,
+                          chunk=ws_.chunk, signed_gate=ws_.signed_gate, o=os_, S_T=Ss,
+                          workspace=wss)
+
+        ms_s = max_over_ranks(time_loop(spread, csteps, args.warmup, world, stream), world)
+        if ops.workspace_status(wss) != 0:
+            raise RuntimeError("device status after the CKDA spread leg")
+        ckda = {"workload": w.name, "steps": csteps,
+                "kda_ms_per_step": ms_k / csteps, "ckda_ms_per_step": ms_c / csteps,
+                "ckda_over_kda_throughput": ms_k / ms_c,
+                "spread": {"workload": ws_.name, "ms_per_step": ms_s / csteps,
+                           "tokens_per_s": ws_.tokens * world * csteps / (ms_s / 1000.0),
+                           "hbm_gbs": prefill_bytes(ws_) * world * csteps / (ms_s / 1000.0) / 1e9}}
+        del ds, os_, Ss, wss
+
     # ------------------------------------------------------------ decode leg
     wd = DECODE
     dsteps = args.decode_steps or max(args.steps, 128)
@@ -403,7 +442,8 @@ def main():
                        "chunk": w.chunk, "signed_gate": w.signed_gate, "io_dtype": w.io_dtype,
                        "o_dtype": w.o_dtype, "state_dtype": "f32",
                        "l2": "inputs larger than L2 (q,k,v,a 268 MB + o 67 MB per step)"},
-            "roofline": roofline, "decode": decode_obj, "cpu_baseline": cpu, "e2e": e2e,
+            "roofline": roofline, "decode": decode_obj, "ckda": ckda, "cpu_baseline": cpu,
+            "e2e": e2e,
             "gpu_launches": args.steps, "clocks": clocks, "peaks_source": peaks["source"],
         }
         print(json.dumps(line), flush=True)

@@ -287,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         {
           const uint64_t w0 = globaltimer();
           for (;;) {
-            if (mbar_try_wait(rdy1, ph1)) { fast = true; ph1 ^= 1; break; }
+            if (mbar_try_wait_sleep(rdy1, ph1, 2000)) { fast = true; ph1 ^= 1; break; }
             if (mbar_try_wait(rdy_slow, phs)) {
               phs ^= 1;
               mbar_arrive(bar_ack);
