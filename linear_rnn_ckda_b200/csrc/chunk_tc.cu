@@ -17,7 +17,7 @@
 //   (1) [A;P]   = [Kr;Qr] Kc^T          M=128 (64 Kr rows + 64 Qr rows), N=64, K=128
 //   (a) [X^T|O^T] = S^T [Kr;Qr]^T       N=128 (X = Kr S, and O's first term), K=128
 //   (b) V' = V - X in fp32 (threads), kept in TMEM as tf32 hi + lo parts
-//   (c) U^T     = V'^T Tm^T              A = V'^T in TMEM (hi and lo), K=64, in two rounds
+//   (c) U^T     = V'^T Tm^T              A = V'^T in TMEM (hi and lo), K=64, then three rounds
 //   (d) [O^T|S^T] += U^T [P;Kc^T]^T     N=192, then S^T columns scaled by G_63 (threads)
 // (1) and (a) need only the chunk's inputs and S, so they are issued together
 // when the chunk starts, and (b) overlaps the solve.  All MMAs are kind::tf32
@@ -53,9 +53,11 @@ constexpr int kBarC = 1;                    // named barrier of the compute warp
 // shared memory map (bytes from a 1024-aligned base)
 constexpr uint32_t OFF_KQ = 0;          // [Kr;Qr] 128 rows x 128 fp32, 4 column blocks of 16 KB
 constexpr uint32_t OFF_KC = 65536;      // Kc 64 rows x 128 fp32, 4 column blocks of 8 KB;
-                                        // then the solve's A (64 x kAS), the M tile and the
-                                        // gate pass's exchange (from +24576)
-constexpr uint32_t OFF_M = OFF_KC + 18432;   // M = X2 A21, 32 x 32 tf32 (one column block)
+                                        // then the solve's A (64 x kAS), the R tiles and the
+                                        // gate pass's exchange
+constexpr uint32_t OFF_R2 = OFF_KC + 18432;    // [M10; M20; M30]: 48 rows, K = 16 of 32
+constexpr uint32_t OFF_R34 = OFF_KC + 24576;   // [M21; M31; M32]: 48 rows, K = 16 of 32
+constexpr uint32_t OFF_XCH = OFF_KC + 30720;   // gate pass exchange [4][128] fp32
 constexpr uint32_t OFF_PK = 98304;      // [P; Kc^T]: 64 + 128 rows x 64 fp32, the B operand of
                                         // (d); each 32-column block holds P's 64 rows and then
                                         // Kc^T's 128 rows (24 KB)
@@ -74,7 +76,9 @@ constexpr uint32_t COL_U = 0, COL_VT0 = 64, COL_AP = 128, COL_LO = 128, COL_X = 
                    COL_S = 320, COL_VT1 = 448;
 
 constexpr uint32_t IDESC_N64 = idesc_tf32(128, 64, false, false);         // (1), (c), O += U P^T
-constexpr uint32_t IDESC_N32_NEG = idesc_tf32(128, 32, false, false, true);  // (c) second round
+constexpr uint32_t IDESC_N48_NEG = idesc_tf32(128, 48, false, false, true);  // (c) round 2
+constexpr uint32_t IDESC_N32_NEG = idesc_tf32(128, 32, false, false, true);  // (c) round 3
+constexpr uint32_t IDESC_N16_NEG = idesc_tf32(128, 16, false, false, true);  // (c) round 4
 constexpr uint32_t IDESC_N128 = idesc_tf32(128, 128, false, false);       // (a)
 constexpr uint32_t IDESC_N192 = idesc_tf32(128, 192, false, false);       // (d)
 
@@ -146,52 +150,60 @@ __device__ __forceinline__ float fast_beta(float b) {
 // every bank once per wavefront.
 constexpr int kAS = 68;
 
-// Tm = (I + A)^{-1} Diag(beta) for the 64 x 64 strictly lower A (plain, row
-// stride kAS, zeros on and above the diagonal).  In 32 x 32 blocks
-//   I + A = [[L1, 0], [A21, L2]],  (I + A)^{-1} = [[X1, 0], [-M X1, X2]],
-//   X1 = L1^{-1},  X2 = L2^{-1},  M = X2 A21.
-// X1, X2 and M are three independent forward substitutions (warps 1, 2, 3):
-// lane j keeps column j in registers and finishes the rows in order, reading
-// each row of the triangular factor as a broadcast; all fp32.  Written as tf32:
-// the block-diagonal part Tb = blockdiag(X1, X2) Diag(beta) into the T tile
-// (off-diagonal blocks zero) and M into its own 32 x 32 tile.  The off-diagonal
-// block of Tm is never formed: with U = Tm V' and Ub = Tb V' (rows split
-// 32 + 32), U_top = Ub_top and U_bot = Ub_bot - M U_top, a second MMA round.
-__device__ __forceinline__ void solve_T(const float *A, uint8_t *sT, uint8_t *sMt,
-                                        const float *beta, int tid) {
-  const int role = (tid >> 5) - 1, lane = tid & 31;   // 0: X1, 1: X2, 2: M
-  if (role < 0 || role > 2) return;
-  const int j = lane;
-  const int o = role == 0 ? 0 : 32;   // the diagonal block solved by this warp
-  float x[32];
+// Tm = (I + A)^{-1} Diag(beta) for the 64 x 64 strictly lower A (plain, row stride kAS,
+// zeros on and above the diagonal), in 16 x 16 blocks i, j = 0..3 with diagonal blocks
+// D_i = I + A_ii.  Block forward substitution of (I + A) U = Diag(beta) V' gives
+//   U_i = Ub_i - sum_{j<i} M_ij U_j,   Ub = Tb V',  Tb = blockdiag(X_i) Diag(beta),
+//   X_i = D_i^{-1},  M_ij = X_i A_ij,
+// so the solve needs only ten independent 16-row forward substitutions: X_0..X_3 (right-hand
+// sides the identity) and the six M_ij (right-hand sides the columns of A_ij).  Half a warp
+// takes one of them (lane = column, kept in registers, rows finished in order, each row of
+// D_i read as a broadcast; all fp32), two per warp over warps w0..w0+4.  Written as tf32:
+// Tb into the T tile (zeros off the diagonal blocks), [M10; M20; M30] and [M21; M31; M32]
+// into two 48-row tiles (K = 16 of each 32-wide row used).  The MMA rounds then apply the
+// M_ij as each U_j becomes final.
+__device__ __forceinline__ void solve_T(const float *A, uint8_t *sT, uint8_t *sR2, uint8_t *sR34,
+                                        const float *beta, int task2, int lane) {
+  // task: 0..3 X_i;  4..9 M_ij in the order (1,0) (2,0) (3,0) (2,1) (3,1) (3,2)
+  const int task = 2 * task2 + (lane >> 4), jj = lane & 15;
+  constexpr int kI[10] = {0, 1, 2, 3, 1, 2, 3, 2, 3, 3};
+  constexpr int kJ[10] = {0, 1, 2, 3, 0, 0, 0, 1, 1, 2};
+  int bi = 0, bj = 0;
 #pragma unroll
-  for (int r = 0; r < 32; ++r) {
+  for (int x = 0; x < 10; ++x)
+    if (x == task) {
+      bi = kI[x];
+      bj = kJ[x];
+    }
+  const bool is_x = task < 4;
+  const int o = 16 * bi;
+  float xv[16];
+#pragma unroll
+  for (int r = 0; r < 16; ++r) {
     const float *row = A + (o + r) * kAS + o;
-    // right-hand side: column j of the identity (X1, X2) or of A21 (M)
-    float acc0 = role == 2 ? A[(32 + r) * kAS + j] : (r == j ? 1.f : 0.f);
+    float acc0 = is_x ? (r == jj ? 1.f : 0.f) : A[(o + r) * kAS + 16 * bj + jj];
     float acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
 #pragma unroll
     for (int l4 = 0; l4 < r; l4 += 4) {
       const float4 a = *reinterpret_cast<const float4 *>(row + l4);
-      acc0 = fmaf(-a.x, x[l4], acc0);
-      if (l4 + 1 < r) acc1 = fmaf(-a.y, x[l4 + 1], acc1);
-      if (l4 + 2 < r) acc2 = fmaf(-a.z, x[l4 + 2], acc2);
-      if (l4 + 3 < r) acc3 = fmaf(-a.w, x[l4 + 3], acc3);
+      acc0 = fmaf(-a.x, xv[l4], acc0);
+      if (l4 + 1 < r) acc1 = fmaf(-a.y, xv[l4 + 1], acc1);
+      if (l4 + 2 < r) acc2 = fmaf(-a.z, xv[l4 + 2], acc2);
+      if (l4 + 3 < r) acc3 = fmaf(-a.w, xv[l4 + 3], acc3);
     }
-    x[r] = (acc0 + acc1) + (acc2 + acc3);
+    xv[r] = (acc0 + acc1) + (acc2 + acc3);
   }
-  if (role < 2) {
-    // Tb: column o + j of the diagonal block, zeros in the same column of the other block row
-    const float bj = beta[o + j];
-    const int zr = 32 - o;
+  if (is_x) {
+    // column o + jj of Tb: this block's rows, zeros in the other three block rows
+    const float bj_ = beta[o + jj];
 #pragma unroll
-    for (int r = 0; r < 32; ++r) {
-      st_tf32(sT, sw32(64, o + r, o + j), x[r] * bj);
-      *reinterpret_cast<uint32_t *>(sT + sw32(64, zr + r, o + j)) = 0u;
-    }
+    for (int r = 0; r < 64; ++r) st_tf32(sT, sw32(64, r, o + jj), (r >> 4) == bi ? xv[r & 15] * bj_ : 0.f);
   } else {
+    // row n of R2 = rows of U updated by U_0 (blocks 1..3); R34 = blocks 2, 3 by U_1, 3 by U_2
+    uint8_t *tile = bj == 0 ? sR2 : sR34;
+    const int base = bj == 0 ? 16 * (bi - 1) : (bj == 1 ? 16 * (bi - 2) : 32);
 #pragma unroll
-    for (int r = 0; r < 32; ++r) st_tf32(sMt, sw32(32, r, j), x[r]);
+    for (int r = 0; r < 16; ++r) st_tf32(tile, sw32(48, base + r, jj), xv[r]);
   }
 }
 
@@ -260,7 +272,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint64_t dKC = smem_desc_sw128(sbase + OFF_KC, 16, 1024);
   const uint64_t dPK = smem_desc_sw128(sbase + OFF_PK, 16, 1024);
   const uint64_t dT = smem_desc_sw128(sbase + OFF_T, 16, 1024);
-  const uint64_t dM = smem_desc_sw128(sbase + OFF_M, 16, 1024);
+  const uint64_t dR2 = smem_desc_sw128(sbase + OFF_R2, 16, 1024);
+  const uint64_t dR34 = smem_desc_sw128(sbase + OFF_R34, 16, 1024);
   auto dadd = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (bytes >> 4); };
 
   auto issue_tma = [&](long cs) {
@@ -332,13 +345,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ts(tmem + COL_U, tmem + COL_LO + 8 * s, dadd(dT, (s >> 2) * 8192 + (s & 3) * 32),
                  IDESC_N64, 1);
         mma_commit(bar_r);
-        // round 2: rows 32..63 of U minus M times rows 0..31 (U_top^T read from TMEM)
+        // rounds 2, 3, 4: U_i -= M_ij U_j for the blocks j = 0, 1, 2 as each becomes final
+        // (U_j^T read from TMEM, K = 16)
         if (!(ok = mbar_wait_or_abort(bar_r, phr, kWaitNs, sAbort))) break;
         phr ^= 1;
         tc_fence_after();
 #pragma unroll
-        for (int s = 0; s < 4; ++s)
-          mma_ts(tmem + COL_U + 32, tmem + COL_U + 8 * s, dadd(dM, s * 32), IDESC_N32_NEG, 1);
+        for (int s = 0; s < 2; ++s)
+          mma_ts(tmem + COL_U + 16, tmem + COL_U + 8 * s, dadd(dR2, s * 32), IDESC_N48_NEG, 1);
+        mma_commit(bar_r);
+        if (!(ok = mbar_wait_or_abort(bar_r, phr, kWaitNs, sAbort))) break;
+        phr ^= 1;
+        tc_fence_after();
+#pragma unroll
+        for (int s = 0; s < 2; ++s)
+          mma_ts(tmem + COL_U + 32, tmem + COL_U + 16 + 8 * s, dadd(dR34, s * 32), IDESC_N32_NEG,
+                 1);
+        mma_commit(bar_r);
+        if (!(ok = mbar_wait_or_abort(bar_r, phr, kWaitNs, sAbort))) break;
+        phr ^= 1;
+        tc_fence_after();
+#pragma unroll
+        for (int s = 0; s < 2; ++s)
+          mma_ts(tmem + COL_U + 48, tmem + COL_U + 32 + 8 * s, dadd(dR34, 4096 + s * 32),
+                 IDESC_N16_NEG, 1);
         mma_commit(bar_r);
         // (d) [O^T|S^T] += U^T [P;Kc^T]^T
         if (!(ok = mbar_wait_or_abort(bar_r, phr, kWaitNs, sAbort))) break;
@@ -393,12 +423,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Returns whether the chunk is out of range.  Range: for KDA and CKDA every |alpha| <= 1,
     // so |G_t| never grows within the chunk and the last row decides (a NaN gate propagates
     // to it); raw gates are checked at every row.
-    float *sXch = reinterpret_cast<float *>(sKC + 24576);    // [4][128], past the solve's data
-    float *sXchI = reinterpret_cast<float *>(sKC + 26624);   // [4][128] inverse products (KDA)
+    // [4][128] products of the row groups' gates (KDA: of their inverses), past the solve's data
+    float *sXch = reinterpret_cast<float *>(sm + OFF_XCH);
     float b_next = 0.f;
     if (tid < kC && t0 + tid < t1) b_next = p.b[(size_t)(bofs + t0 + tid) * H + h];
     float kc[16];
-    auto gate_core = [&](int nrows, float *gc_out, uint32_t vcol) -> bool {
+    auto gate_core = [&](float *gc_out, uint32_t vcol) -> bool {
       float g[16], ig[16];
       float run = 1.f, irun = 1.f;
 #pragma unroll
@@ -414,7 +444,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           al = fast_alpha<SG>(a);
         }
-        if (r >= nrows) al = ial = 1.f;
         run *= al;
         g[rr] = run;
         if (SG == 0) {
@@ -422,16 +451,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           ig[rr] = irun;
         }
       }
-      sXch[qg * 128 + c] = run;
-      if (SG == 0) sXchI[qg * 128 + c] = irun;
+      sXch[qg * 128 + c] = SG == 0 ? irun : run;
       csync();
       float mult = 1.f, imult = 1.f;
 #pragma unroll
       for (int x = 0; x < 3; ++x)
         if (x < qg) {
-          mult *= sXch[x * 128 + c];
-          if (SG == 0) imult *= sXchI[x * 128 + c];
+          if (SG == 0)
+            imult *= sXch[x * 128 + c];
+          else
+            mult *= sXch[x * 128 + c];
         }
+      if (SG == 0) mult = __fdividef(1.f, imult);
       bool bad = false;
       uint32_t vt[16];
 #pragma unroll
@@ -443,11 +474,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           bad |= !(ag >= 0x1p-100f && ag <= 0x1p100f);
         }
         const float inv = SG == 0 ? ig[rr] * imult : __fdividef(1.f, gam);
-        float qv = ldbf(stq, r, c), kv = ldbf(stk, r, c), vv = ldbf(stv, r, c);
-        if (r >= nrows) {
-          // rows past the sequence end hold another sequence's tokens or TMA fill
-          qv = kv = vv = 0.f;
-        }
+        const float qv = ldbf(stq, r, c), kv = ldbf(stk, r, c), vv = ldbf(stv, r, c);
         st_tf32(sKQ, sw32(128, r, c), kv * gam);
         st_tf32(sKQ, sw32(128, 64 + r, c), qv * gam);
         kc[rr] = __uint_as_float(to_tf32(kv * inv));
@@ -463,7 +490,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float b_cur = b_next;
       if (tid < kC && cs + kC + tid < t1) b_next = p.b[(size_t)(bofs + cs + kC + tid) * H + h];
       if (tid < kC) sBeta[tid] = tid < nrows ? fast_beta<SG>(b_cur) : 0.f;
-      return gate_core(nrows, gc_out, vcol);
+      if (nrows < kC) {
+        // Rows past the sequence end hold another sequence's tokens or TMA fill.  They are
+        // overwritten in the staging copy with q = k = v = 0 and a gate of exactly 1
+        // (a = 100 gives sigma(a) = 2 sigma(a) - 1 = 1 in fp32; raw gates take a = 1), so
+        // the pass needs no per-row masking.
+        const uint32_t afill = SG == 2 ? 0x3F803F80u : 0x42C842C8u;   // bf16 pairs 1.0, 100.0
+        const int nt = (kC - nrows) * 16;   // 16-byte pieces of one array: 8 per row and box
+        for (int e = tid; e < 4 * nt; e += kCompute) {
+          const int x = e / nt, rem = e - x * nt;
+          const int row = nrows + (rem >> 4), piece = rem & 15;
+          const uint32_t f = x == 3 ? afill : 0u;
+          *reinterpret_cast<uint4 *>(sStg + x * 16384 + (piece >> 3) * 8192 + row * 128 +
+                                     (piece & 7) * 16) = make_uint4(f, f, f, f);
+        }
+        csync();
+      }
+      return gate_core(gc_out, vcol);
     };
     auto store_kc = [&]() {  // Kc (row t, channel c); Kc^T (row c, four t per 16-byte store)
 #pragma unroll
@@ -627,7 +670,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       csync();
       // ---------------------------------------------------------------- Tm = (I + A)^{-1} Diag(beta)
-      // warps 1..3 solve; meanwhile warps 4..7 form (b) V' = V - X once (a) is done, as a
+      // warps 8..12 solve; meanwhile warps 4..7 form (b) V' = V - X once (a) is done, as a
       // round-to-nearest tf32 hi part (over V^T) and the fp32 remainder (over [A;P])
       bool ok = true;
       if (warp >= 4 && warp < 8) {
@@ -653,7 +696,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_st();
         }
       } else {
-        solve_T(sA, sT, sm + OFF_M, sBeta, tid);
+        if (warp >= 8 && warp < 13) solve_T(sA, sT, sm + OFF_R2, sm + OFF_R34, sBeta, warp - 8, lane);
       }
       a_ph ^= 1;
       fence_proxy_async();
