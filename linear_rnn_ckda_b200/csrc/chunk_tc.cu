@@ -230,8 +230,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   // issuer -> compute warps: a token-by-token announcement has been consumed (so the next
   // announcement cannot be mistaken for it)
   uint64_t *bar_ack = bars + 10;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_MISC + 1376);
-  volatile int *sAbort = reinterpret_cast<volatile int *>(sm + OFF_MISC + 1380);
+  // the last round of (c) is done: the R tiles in Kc's area have been read
+  uint64_t *bar_r4 = bars + 11;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_MISC + 1392);
+  volatile int *sAbort = reinterpret_cast<volatile int *>(sm + OFF_MISC + 1396);
   const uint32_t sbase = smem_u32(sm);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -258,6 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int x = 0; x < 6; ++x) mbar_init(bars + x, 1);
     for (int x = 6; x < 10; ++x) mbar_init(bars + x, kCompute / 32);
     mbar_init(bar_ack, 1);
+    mbar_init(bar_r4, 1);
     *sAbort = 0;
     mbar_fence_init();
   }
@@ -370,6 +373,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ts(tmem + COL_U + 48, tmem + COL_U + 32 + 8 * s, dadd(dR34, 4096 + s * 32),
                  IDESC_N16_NEG, 1);
         mma_commit(bar_r);
+        mma_commit(bar_r4);
         // (d) [O^T|S^T] += U^T [P;Kc^T]^T
         if (!(ok = mbar_wait_or_abort(bar_r, phr, kWaitNs, sAbort))) break;
         phr ^= 1;
@@ -395,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int jrow = 32 * (warp & 3) + lane;
     const int c = jrow;
     const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
-    uint32_t tma_ph = 0, mma1_ph = 0, a_ph = 0, d_ph = 0, ack_ph = 0;
+    uint32_t tma_ph = 0, mma1_ph = 0, a_ph = 0, d_ph = 0, ack_ph = 0, r4_ph = 0;
     // bf16 O (16 KB per chunk) is staged in T's tile and written by one TMA store;
     // fp32 O is written directly from registers
     constexpr bool kTmaStoreO = sizeof(TOut) == 2;
@@ -508,14 +512,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       return gate_core(gc_out, vcol);
     };
-    auto store_kc = [&]() {  // Kc (row t, channel c); Kc^T (row c, four t per 16-byte store)
+    auto store_kc_tile = [&]() {  // Kc (row t, channel c)
 #pragma unroll
       for (int rr = 0; rr < 16; ++rr)
         *reinterpret_cast<float *>(sKC + sw32(64, 16 * qg + rr, c)) = kc[rr];
+    };
+    auto store_kct_tile = [&]() {  // Kc^T (row c, four t per 16-byte store)
 #pragma unroll
       for (int rr = 0; rr < 16; rr += 4)
         *reinterpret_cast<float4 *>(sPK + swpk(64 + c, 16 * qg + rr)) =
             make_float4(kc[rr], kc[rr + 1], kc[rr + 2], kc[rr + 3]);
+    };
+    auto store_kc = [&]() {
+      store_kc_tile();
+      store_kct_tile();
     };
     // tiles of the next chunk written: tell the issuer which path it takes
     auto announce_chunk = [&](bool is_slow) {
@@ -711,13 +721,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!cwait(bar_tma, tma_ph)) { failed = true; break; }
         bad_next = gate_pass(cs + kC, nrows_next, gc_next, vt_next);
       }
+      // the next chunk's Kc tile once (c) is done with the R tiles; then (1) of the next
+      // chunk can run under this chunk's (d) and read-out.  Kc^T waits for (d).
+      if (!cwait(bar_r4, r4_ph)) { failed = true; break; }
+      if (has_next) {
+        store_kc_tile();
+        slow = bar_or(kBarC, kCompute, bad_next);
+        announce_chunk(slow);
+      }
       if (!cwait(bar_d, d_ph)) { failed = true; break; }
       tc_fence_after();
-      if (has_next) {
-        store_kc();
-        slow = bar_or(kBarC, kCompute, bad_next);
-        announce_chunk(slow);   // (1) of the next chunk runs under this chunk's read-out
-      }
+      if (has_next) store_kct_tile();
       // ---------------------------------------------------------------- O out; S^T columns scaled by G_63
       {
         uint32_t r[32];
@@ -742,7 +756,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(lane_addr + COL_S + i0, r);
         tmem_wait_ld();
 #pragma unroll
-        for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * gc_cur[i0 + x]);
+        for (int x = 0; x < 32; x += 4) {
+          const float4 gv = *reinterpret_cast<const float4 *>(gc_cur + i0 + x);
+          r[x] = __float_as_uint(__uint_as_float(r[x]) * gv.x);
+          r[x + 1] = __float_as_uint(__uint_as_float(r[x + 1]) * gv.y);
+          r[x + 2] = __float_as_uint(__uint_as_float(r[x + 2]) * gv.z);
+          r[x + 3] = __float_as_uint(__uint_as_float(r[x + 3]) * gv.w);
+        }
         tmem_st32(lane_addr + COL_S + i0, r);
         tmem_wait_st();
       }
