@@ -53,11 +53,10 @@ constexpr int kBarC = 1;                    // named barrier of the compute warp
 // shared memory map (bytes from a 1024-aligned base)
 constexpr uint32_t OFF_KQ = 0;          // [Kr;Qr] 128 rows x 128 fp32, 4 column blocks of 16 KB
 constexpr uint32_t OFF_KC = 65536;      // Kc 64 rows x 128 fp32, 4 column blocks of 8 KB;
-                                        // then the solve's A (64 x kAS), the R tiles and the
-                                        // gate pass's exchange
+                                        // then the solve's A (64 x kAS) (or the gate pass's
+                                        // exchange) and the R tiles
 constexpr uint32_t OFF_R2 = OFF_KC + 18432;    // [M10; M20; M30]: 48 rows, K = 16 of 32
 constexpr uint32_t OFF_R34 = OFF_KC + 24576;   // [M21; M31; M32]: 48 rows, K = 16 of 32
-constexpr uint32_t OFF_XCH = OFF_KC + 30720;   // gate pass exchange [4][128] fp32
 constexpr uint32_t OFF_PK = 98304;      // [P; Kc^T]: 64 + 128 rows x 64 fp32, the B operand of
                                         // (d); each 32-column block holds P's 64 rows and then
                                         // Kc^T's 128 rows (24 KB)
@@ -427,66 +426,102 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Returns whether the chunk is out of range.  Range: for KDA and CKDA every |alpha| <= 1,
     // so |G_t| never grows within the chunk and the last row decides (a NaN gate propagates
     // to it); raw gates are checked at every row.
-    // [4][128] products of the row groups' gates (KDA: of their inverses), past the solve's data
-    float *sXch = reinterpret_cast<float *>(sm + OFF_XCH);
     float b_next = 0.f;
     if (tid < kC && t0 + tid < t1) b_next = p.b[(size_t)(bofs + t0 + tid) * H + h];
     float kc[16];
+    // The gate pass proper works on channel pairs: thread (pair pc = tid % 64, row group
+    // rg = tid / 64) takes channels 2pc, 2pc + 1 of rows 8rg .. 8rg + 7, reading bf16 pairs
+    // and writing 8-byte pairs.  V^T keeps the one-channel-per-lane mapping TMEM needs.
+    const int pc = tid & 63, rg = tid >> 6, ch0 = 2 * pc;
+    float *sXp = reinterpret_cast<float *>(sKC);   // [8][128] row-group products (the solve's A
+                                                   // is dead whenever a gate pass runs)
+    auto ldbf2 = [&](const uint8_t *tile, int r, float &x0, float &x1) {
+      const uint32_t u = *reinterpret_cast<const uint32_t *>(tile + swbf(r, ch0));
+      x0 = __uint_as_float(u << 16);
+      x1 = __uint_as_float(u & 0xFFFF0000u);
+    };
+    auto gate2 = [&](float a, float &al, float &ial) {
+      if (SG == 0) {
+        // sigma(a) and its inverse 1 + e^{-a} from one exponential
+        const float e = __expf(-a);
+        ial = 1.f + e;
+        al = __fdividef(1.f, ial);
+      } else {
+        ial = 1.f;
+        al = fast_alpha<SG>(a);
+      }
+    };
     auto gate_core = [&](float *gc_out, uint32_t vcol) -> bool {
-      float g[16], ig[16];
-      float run = 1.f, irun = 1.f;
+      {
+        // lane c of TMEM holds V^T[c][.] (V' = V - X is formed in place before (c))
+        uint32_t vt[16];
 #pragma unroll
-      for (int rr = 0; rr < 16; ++rr) {
-        const int r = 16 * qg + rr;
-        const float a = ldbf(sta, r, c);
-        float al, ial = 1.f;
+        for (int rr = 0; rr < 16; ++rr) vt[rr] = __float_as_uint(ldbf(stv, 16 * qg + rr, c));
+        tmem_st16(lane_addr + vcol + 16 * qg, vt);
+      }
+      float g[16], ig[16];   // [row][channel of the pair]
+      float run0 = 1.f, run1 = 1.f, irun0 = 1.f, irun1 = 1.f;
+#pragma unroll
+      for (int rr = 0; rr < 8; ++rr) {
+        float a0, a1, al0, al1, ial0, ial1;
+        ldbf2(sta, 8 * rg + rr, a0, a1);
+        gate2(a0, al0, ial0);
+        gate2(a1, al1, ial1);
+        run0 *= al0;
+        run1 *= al1;
+        g[2 * rr] = run0;
+        g[2 * rr + 1] = run1;
         if (SG == 0) {
-          // sigma(a) and its inverse 1 + e^{-a} from one exponential
-          const float e = __expf(-a);
-          ial = 1.f + e;
-          al = __fdividef(1.f, ial);
-        } else {
-          al = fast_alpha<SG>(a);
-        }
-        run *= al;
-        g[rr] = run;
-        if (SG == 0) {
-          irun *= ial;
-          ig[rr] = irun;
+          irun0 *= ial0;
+          irun1 *= ial1;
+          ig[2 * rr] = irun0;
+          ig[2 * rr + 1] = irun1;
         }
       }
-      sXch[qg * 128 + c] = SG == 0 ? irun : run;
+      *reinterpret_cast<float2 *>(sXp + rg * 128 + ch0) =
+          SG == 0 ? make_float2(irun0, irun1) : make_float2(run0, run1);
       csync();
-      float mult = 1.f, imult = 1.f;
+      // products of the earlier row groups (KDA: of the inverses)
+      float m0 = 1.f, m1 = 1.f;
 #pragma unroll
-      for (int x = 0; x < 3; ++x)
-        if (x < qg) {
-          if (SG == 0)
-            imult *= sXch[x * 128 + c];
-          else
-            mult *= sXch[x * 128 + c];
+      for (int x = 0; x < 7; ++x)
+        if (x < rg) {
+          const float2 v = *reinterpret_cast<const float2 *>(sXp + x * 128 + ch0);
+          m0 *= v.x;
+          m1 *= v.y;
         }
-      if (SG == 0) mult = __fdividef(1.f, imult);
-      bool bad = false;
-      uint32_t vt[16];
-#pragma unroll
-      for (int rr = 0; rr < 16; ++rr) {
-        const int r = 16 * qg + rr;
-        const float gam = g[rr] * mult;
-        if (SG == 2 || (rr == 15 && qg == 3)) {
-          const float ag = fabsf(gam);
-          bad |= !(ag >= 0x1p-100f && ag <= 0x1p100f);
-        }
-        const float inv = SG == 0 ? ig[rr] * imult : __fdividef(1.f, gam);
-        const float qv = ldbf(stq, r, c), kv = ldbf(stk, r, c), vv = ldbf(stv, r, c);
-        st_tf32(sKQ, sw32(128, r, c), kv * gam);
-        st_tf32(sKQ, sw32(128, 64 + r, c), qv * gam);
-        kc[rr] = __uint_as_float(to_tf32(kv * inv));
-        vt[rr] = __float_as_uint(vv);
-        if (rr == 15 && qg == 3) gc_out[c] = gam;
+      float mult0, mult1, imult0 = 1.f, imult1 = 1.f;
+      if (SG == 0) {
+        imult0 = m0;
+        imult1 = m1;
+        mult0 = __fdividef(1.f, m0);
+        mult1 = __fdividef(1.f, m1);
+      } else {
+        mult0 = m0;
+        mult1 = m1;
       }
-      // lane c of TMEM holds V^T[c][.] (V' = V - X is formed in place before (c))
-      tmem_st16(lane_addr + vcol + 16 * qg, vt);
+      bool bad = false;
+#pragma unroll
+      for (int rr = 0; rr < 8; ++rr) {
+        const int r = 8 * rg + rr;
+        const float gam0 = g[2 * rr] * mult0, gam1 = g[2 * rr + 1] * mult1;
+        if (SG == 2 || (rr == 7 && rg == 7)) {
+          const float ag0 = fabsf(gam0), ag1 = fabsf(gam1);
+          bad |= !(ag0 >= 0x1p-100f && ag0 <= 0x1p100f && ag1 >= 0x1p-100f && ag1 <= 0x1p100f);
+        }
+        const float inv0 = SG == 0 ? ig[2 * rr] * imult0 : __fdividef(1.f, gam0);
+        const float inv1 = SG == 0 ? ig[2 * rr + 1] * imult1 : __fdividef(1.f, gam1);
+        float q0, q1, k0, k1;
+        ldbf2(stq, r, q0, q1);
+        ldbf2(stk, r, k0, k1);
+        *reinterpret_cast<uint2 *>(sKQ + sw32(128, r, ch0)) =
+            make_uint2(to_tf32(k0 * gam0), to_tf32(k1 * gam1));
+        *reinterpret_cast<uint2 *>(sKQ + sw32(128, 64 + r, ch0)) =
+            make_uint2(to_tf32(q0 * gam0), to_tf32(q1 * gam1));
+        kc[2 * rr] = __uint_as_float(to_tf32(k0 * inv0));
+        kc[2 * rr + 1] = __uint_as_float(to_tf32(k1 * inv1));
+        if (rr == 7 && rg == 7) *reinterpret_cast<float2 *>(gc_out + ch0) = make_float2(gam0, gam1);
+      }
       tmem_wait_st();
       return bad;
     };
@@ -512,16 +547,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       return gate_core(gc_out, vcol);
     };
-    auto store_kc_tile = [&]() {  // Kc (row t, channel c)
+    auto store_kc_tile = [&]() {  // Kc (row t, channel pair)
 #pragma unroll
-      for (int rr = 0; rr < 16; ++rr)
-        *reinterpret_cast<float *>(sKC + sw32(64, 16 * qg + rr, c)) = kc[rr];
+      for (int rr = 0; rr < 8; ++rr)
+        *reinterpret_cast<float2 *>(sKC + sw32(64, 8 * rg + rr, ch0)) =
+            make_float2(kc[2 * rr], kc[2 * rr + 1]);
     };
-    auto store_kct_tile = [&]() {  // Kc^T (row c, four t per 16-byte store)
+    auto store_kct_tile = [&]() {  // Kc^T (rows 2pc and 2pc + 1, four t per 16-byte store)
 #pragma unroll
-      for (int rr = 0; rr < 16; rr += 4)
-        *reinterpret_cast<float4 *>(sPK + swpk(64 + c, 16 * qg + rr)) =
-            make_float4(kc[rr], kc[rr + 1], kc[rr + 2], kc[rr + 3]);
+      for (int e = 0; e < 2; ++e)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf)
+          *reinterpret_cast<float4 *>(sPK + swpk(64 + ch0 + e, 8 * rg + 4 * hf)) =
+              make_float4(kc[8 * hf + e], kc[8 * hf + 2 + e], kc[8 * hf + 4 + e], kc[8 * hf + 6 + e]);
     };
     auto store_kc = [&]() {
       store_kc_tile();
