@@ -115,28 +115,8 @@ __device__ __forceinline__ void st_tf32(uint8_t *tile, uint32_t off, float x) {
   *reinterpret_cast<uint32_t *>(tile + off) = to_tf32(x);
 }
 
-// Gates for the bf16 path, from their definitions with fast exponentials
-// (relative error ~1e-6, far inside the bf16-input tolerance):
-//   sigma(a) = 1 / (1 + e^{-a});  2 sigma(a) - 1 = tanh(a/2) = (1 - e^{-|a|}) / (1 + e^{-|a|})
-// with the odd Taylor series tanh(y) = y - y^3/3 + 2 y^5/15 for |a| < 0.1
-// (truncation below 2e-10 relative there), so small gates keep full precision.
-template <int SG>
-__device__ __forceinline__ float fast_alpha(float a) {
-  if (SG == 0) return __fdividef(1.f, 1.f + __expf(-a));
-  if (SG == 1) {
-    const float x = fabsf(a);
-    float t;
-    if (x < 0.1f) {
-      const float y = 0.5f * x, y2 = y * y;
-      t = y * fmaf(y2, fmaf(y2, 2.f / 15.f, -1.f / 3.f), 1.f);
-    } else {
-      const float e = __expf(-x);
-      t = __fdividef(1.f - e, 1.f + e);
-    }
-    return copysignf(t, a);
-  }
-  return a;
-}
+// beta for the bf16 path from its definition with a fast exponential (relative error ~1e-6,
+// far inside the bf16-input tolerance): sigma(b) (KDA), 2 sigma(b) (CKDA), b (raw)
 template <int SG>
 __device__ __forceinline__ float fast_beta(float b) {
   if (SG == 0) return __fdividef(1.f, 1.f + __expf(-b));
@@ -433,22 +413,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     // rg = tid / 64) takes channels 2pc, 2pc + 1 of rows 8rg .. 8rg + 7, reading bf16 pairs
     // and writing 8-byte pairs.  V^T keeps the one-channel-per-lane mapping TMEM needs.
     const int pc = tid & 63, rg = tid >> 6, ch0 = 2 * pc;
-    float *sXp = reinterpret_cast<float *>(sKC);   // [8][128] row-group products (the solve's A
-                                                   // is dead whenever a gate pass runs)
+    float *sXp = reinterpret_cast<float *>(sKC);   // [8][128][2] row-group products of the gates
+                                                   // and of their inverses (the solve's A is
+                                                   // dead whenever a gate pass runs)
     auto ldbf2 = [&](const uint8_t *tile, int r, float &x0, float &x1) {
       const uint32_t u = *reinterpret_cast<const uint32_t *>(tile + swbf(r, ch0));
       x0 = __uint_as_float(u << 16);
       x1 = __uint_as_float(u & 0xFFFF0000u);
     };
+    // the gate and (KDA, CKDA) its inverse, so that the second part needs no reciprocal:
+    //   KDA   sigma(a) = 1 / (1 + e^{-a}), inverse 1 + e^{-a}
+    //   CKDA  2 sigma(a) - 1 = tanh(a/2) = sign(a) (1 - e^{-|a|}) / (1 + e^{-|a|}), inverse the
+    //         ratio upside down; both from one reciprocal r = 1 / (num den) (num r = 1 / den,
+    //         den r = 1 / num).  For small |a| the difference 1 - e^{-|a|} cancels: the gate's
+    //         error stays at fp32 rounding level in absolute terms; an exactly zero gate stays 0.
     auto gate2 = [&](float a, float &al, float &ial) {
       if (SG == 0) {
-        // sigma(a) and its inverse 1 + e^{-a} from one exponential
         const float e = __expf(-a);
         ial = 1.f + e;
         al = __fdividef(1.f, ial);
+      } else if (SG == 1) {
+        const float e = __expf(-fabsf(a));
+        const float num = 1.f - e, den = 1.f + e;
+        const float r = __fdividef(1.f, num * den);
+        al = copysignf(num * (num * r), a);
+        ial = copysignf(den * (den * r), a);
       } else {
         ial = 1.f;
-        al = fast_alpha<SG>(a);
+        al = a;
       }
     };
     auto gate_core = [&](float *gc_out, uint32_t vcol) -> bool {
@@ -471,35 +463,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         run1 *= al1;
         g[2 * rr] = run0;
         g[2 * rr + 1] = run1;
-        if (SG == 0) {
+        if (SG != 2) {
           irun0 *= ial0;
           irun1 *= ial1;
           ig[2 * rr] = irun0;
           ig[2 * rr + 1] = irun1;
         }
       }
-      *reinterpret_cast<float2 *>(sXp + rg * 128 + ch0) =
-          SG == 0 ? make_float2(irun0, irun1) : make_float2(run0, run1);
+      *reinterpret_cast<float4 *>(sXp + (rg * 128 + ch0) * 2) = make_float4(run0, irun0, run1, irun1);
       csync();
-      // products of the earlier row groups (KDA: of the inverses)
-      float m0 = 1.f, m1 = 1.f;
+      // products of the earlier row groups (of the gates and of their inverses)
+      float mult0 = 1.f, mult1 = 1.f, imult0 = 1.f, imult1 = 1.f;
 #pragma unroll
       for (int x = 0; x < 7; ++x)
         if (x < rg) {
-          const float2 v = *reinterpret_cast<const float2 *>(sXp + x * 128 + ch0);
-          m0 *= v.x;
-          m1 *= v.y;
+          const float4 v = *reinterpret_cast<const float4 *>(sXp + (x * 128 + ch0) * 2);
+          mult0 *= v.x;
+          imult0 *= v.y;
+          mult1 *= v.z;
+          imult1 *= v.w;
         }
-      float mult0, mult1, imult0 = 1.f, imult1 = 1.f;
-      if (SG == 0) {
-        imult0 = m0;
-        imult1 = m1;
-        mult0 = __fdividef(1.f, m0);
-        mult1 = __fdividef(1.f, m1);
-      } else {
-        mult0 = m0;
-        mult1 = m1;
-      }
       bool bad = false;
 #pragma unroll
       for (int rr = 0; rr < 8; ++rr) {
@@ -509,8 +492,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float ag0 = fabsf(gam0), ag1 = fabsf(gam1);
           bad |= !(ag0 >= 0x1p-100f && ag0 <= 0x1p100f && ag1 >= 0x1p-100f && ag1 <= 0x1p100f);
         }
-        const float inv0 = SG == 0 ? ig[2 * rr] * imult0 : __fdividef(1.f, gam0);
-        const float inv1 = SG == 0 ? ig[2 * rr + 1] * imult1 : __fdividef(1.f, gam1);
+        const float inv0 = SG != 2 ? ig[2 * rr] * imult0 : __fdividef(1.f, gam0);
+        const float inv1 = SG != 2 ? ig[2 * rr + 1] * imult1 : __fdividef(1.f, gam1);
         float q0, q1, k0, k1;
         ldbf2(stq, r, q0, q1);
         ldbf2(stk, r, k0, k1);
