@@ -138,7 +138,7 @@ constexpr int kAS = 68;
 // sides the identity) and the six M_ij (right-hand sides the columns of A_ij).  Half a warp
 // takes one of them (lane = column, kept in registers, rows finished in order, each row of
 // D_i read as a broadcast; all fp32), two per warp over warps w0..w0+4.  Written as tf32:
-// Tb into the T tile (zeros off the diagonal blocks), [M10; M20; M30] and [M21; M31; M32]
+// Tb into the T tile (its zero blocks by solve_T_zeros), [M10; M20; M30] and [M21; M31; M32]
 // into two 48-row tiles (K = 16 of each 32-wide row used).  The MMA rounds then apply the
 // M_ij as each U_j becomes final.
 __device__ __forceinline__ void solve_T(const float *A, uint8_t *sT, uint8_t *sR2, uint8_t *sR34,
@@ -156,15 +156,28 @@ __device__ __forceinline__ void solve_T(const float *A, uint8_t *sT, uint8_t *sR
     }
   const bool is_x = task < 4;
   const int o = 16 * bi;
+  // right-hand sides up front (column jj of I or of A_ij); each row of D_i is fetched one
+  // step ahead of its use, so the loads stay off the dependent chain
+  float rhs[16];
+#pragma unroll
+  for (int r = 0; r < 16; ++r) rhs[r] = is_x ? (r == jj ? 1.f : 0.f) : A[(o + r) * kAS + 16 * bj + jj];
   float xv[16];
+  float4 nx[4];
 #pragma unroll
   for (int r = 0; r < 16; ++r) {
-    const float *row = A + (o + r) * kAS + o;
-    float acc0 = is_x ? (r == jj ? 1.f : 0.f) : A[(o + r) * kAS + 16 * bj + jj];
-    float acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+    float4 cur[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) cur[q] = nx[q];
+    if (r + 1 < 16) {
+      const float *row1 = A + (o + r + 1) * kAS + o;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (4 * q < r + 1) nx[q] = *reinterpret_cast<const float4 *>(row1 + 4 * q);
+    }
+    float acc0 = rhs[r], acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
 #pragma unroll
     for (int l4 = 0; l4 < r; l4 += 4) {
-      const float4 a = *reinterpret_cast<const float4 *>(row + l4);
+      const float4 a = cur[l4 >> 2];
       acc0 = fmaf(-a.x, xv[l4], acc0);
       if (l4 + 1 < r) acc1 = fmaf(-a.y, xv[l4 + 1], acc1);
       if (l4 + 2 < r) acc2 = fmaf(-a.z, xv[l4 + 2], acc2);
@@ -173,16 +186,27 @@ __device__ __forceinline__ void solve_T(const float *A, uint8_t *sT, uint8_t *sR
     xv[r] = (acc0 + acc1) + (acc2 + acc3);
   }
   if (is_x) {
-    // column o + jj of Tb: this block's rows, zeros in the other three block rows
+    // column o + jj of Tb's diagonal block (the zero blocks: solve_T_zeros)
     const float bj_ = beta[o + jj];
 #pragma unroll
-    for (int r = 0; r < 64; ++r) st_tf32(sT, sw32(64, r, o + jj), (r >> 4) == bi ? xv[r & 15] * bj_ : 0.f);
+    for (int r = 0; r < 16; ++r) st_tf32(sT, sw32(64, o + r, o + jj), xv[r] * bj_);
   } else {
     // row n of R2 = rows of U updated by U_0 (blocks 1..3); R34 = blocks 2, 3 by U_1, 3 by U_2
     uint8_t *tile = bj == 0 ? sR2 : sR34;
     const int base = bj == 0 ? 16 * (bi - 1) : (bj == 1 ? 16 * (bi - 2) : 32);
 #pragma unroll
     for (int r = 0; r < 16; ++r) st_tf32(tile, sw32(48, base + r, jj), xv[r]);
+  }
+}
+
+// The twelve off-diagonal 16 x 16 blocks of Tb are zero: 768 16-byte pieces, six per thread
+// of a 128-thread group (t = 0..127), written while other warps run the substitutions.
+__device__ __forceinline__ void solve_T_zeros(uint8_t *sT, int t) {
+#pragma unroll
+  for (int k = 0; k < 6; ++k) {
+    const int e = t + 128 * k, r = e / 12, q = e - 12 * (e / 12), rb = r >> 4;
+    const int c4 = q < 4 * rb ? q : q + 4;   // 4-column piece, skipping the diagonal block
+    *reinterpret_cast<uint4 *>(sT + sw32(64, r, 4 * c4)) = make_uint4(0u, 0u, 0u, 0u);
   }
 }
 
@@ -728,6 +752,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else {
         if (warp >= 8 && warp < 13) solve_T(sA, sT, sm + OFF_R2, sm + OFF_R34, sBeta, warp - 8, lane);
+        if (warp < 4) solve_T_zeros(sT, tid);
       }
       a_ph ^= 1;
       fence_proxy_async();
