@@ -37,6 +37,18 @@ __global__ void __launch_bounds__(kDecodeThreads)
   const int hl = warp / kWarpsPerHead;
   const int head = blockIdx.x * kHeadsPerBlock + hl;
   const int gtid = threadIdx.x - hl * kWarpsPerHead * 32;  // thread index within the head group
+  const int cq = lane & 3, r0 = lane >> 2;
+  const int col = (warp % kWarpsPerHead) * 16 + cq * 4;
+  float *Sh = S + (size_t)head * DK * DV;
+
+  // The state loads go first: they do not depend on the staging below and stay in flight
+  // across it.
+  float4 st[kRows];
+  if (head < n_heads) {
+#pragma unroll
+    for (int m = 0; m < kRows; ++m)
+      st[m] = *reinterpret_cast<const float4 *>(Sh + (size_t)(r0 + 8 * m) * DV + col);
+  }
 
   // Stage q, k and the activated gate for this head group.
   if (head < n_heads) {
@@ -50,15 +62,6 @@ __global__ void __launch_bounds__(kDecodeThreads)
   }
   __syncthreads();
   if (head >= n_heads) return;
-
-  const int cq = lane & 3, r0 = lane >> 2;
-  const int col = (warp % kWarpsPerHead) * 16 + cq * 4;
-  float *Sh = S + (size_t)head * DK * DV;
-
-  float4 st[kRows];
-#pragma unroll
-  for (int m = 0; m < kRows; ++m)
-    st[m] = *reinterpret_cast<const float4 *>(Sh + (size_t)(r0 + 8 * m) * DV + col);
 
   // S' = Diag(alpha) S and p = S'^T k (partial over this thread's rows)
   float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;

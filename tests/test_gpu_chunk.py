@@ -296,3 +296,21 @@ def test_tc_state_alias_and_chunk_boundaries(cuda_lib):
         ro, rS = oracle_prefill(inp, 1)
         o, S = run_gpu(cuda_lib, inp, w, S0_alias=True)
         assert rel(f64(o), ro) <= TOL_BF16 and rel(f64(S), rS) <= TOL_BF16, T
+
+
+@pytest.mark.parametrize("sg", [0, 1])
+def test_tc_small_gate_logits(cuda_lib, sg):
+    """Gate logits near zero on the bf16 d=128 path (CKDA gates of either sign and size
+    below 0.05, KDA gates near 1/2), mixed into large ones so that the chunks stay on the
+    factorised path: the gates' products must still match the oracle."""
+    T, H = 300, 2
+    rng = np.random.default_rng(40 + sg)
+    a = rng.standard_normal((1, T, H, 128)) + np.where(rng.random((1, T, H, 128)) < 0.5, 3.0, -3.0)
+    small = rng.random((1, T, H, 128)) < 0.1
+    a[small] = rng.uniform(-0.1, 0.1, size=int(small.sum()))
+    b = rng.standard_normal((1, T, H))
+    inp = _bf16_raw_case(T, a, b, seed=50 + sg)
+    w = synth.CKDA_SPREAD.with_(B=1, T=T, H=H, signed_gate=sg, o_dtype="f32")
+    o, S = run_gpu(cuda_lib, inp, w)
+    ro, rS = oracle_prefill(inp, sg)
+    assert rel(f64(o), ro) <= TOL_BF16 and rel(f64(S), rS) <= TOL_BF16
