@@ -18,6 +18,10 @@
  *   1  CKDA  alpha = 2 sigma(a) - 1 in [-1,1], beta = 2 sigma(b) in [0,2]
  *            (CKDA review, "Method steps", step 1: both ranges widen together)
  *   2  raw   a holds alpha and b holds beta directly (tests and special cases)
+ *   3  gate range only:      alpha = 2 sigma(a) - 1,  beta = sigma(b)
+ *   4  strength range only:  alpha = sigma(a),        beta = 2 sigma(b)
+ *            (3 and 4: the single-range variants of the CKDA review, "Experimental
+ *            results", Figure 6)
  * Logits of +-inf are legal and exact: alpha = 0, +-1 and beta = 0, 1, 2.
  *
  * Conventions for every entry point:

@@ -117,10 +117,9 @@ __device__ __forceinline__ void st_tf32(uint8_t *tile, uint32_t off, float x) {
 
 // beta for the bf16 path from its definition with a fast exponential (relative error ~1e-6,
 // far inside the bf16-input tolerance): sigma(b) (KDA), 2 sigma(b) (CKDA), b (raw)
-template <int SG>
-__device__ __forceinline__ float fast_beta(float b) {
-  if (SG == 0) return __fdividef(1.f, 1.f + __expf(-b));
-  if (SG == 1) return __fdividef(2.f, 1.f + __expf(-b));
+__device__ __forceinline__ float fast_beta(float b, int form) {
+  if (form == 0) return __fdividef(1.f, 1.f + __expf(-b));
+  if (form == 1) return __fdividef(2.f, 1.f + __expf(-b));
   return b;
 }
 
@@ -535,7 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto gate_pass = [&](long cs, int nrows, float *gc_out, uint32_t vcol) -> bool {
       const float b_cur = b_next;
       if (tid < kC && cs + kC + tid < t1) b_next = p.b[(size_t)(bofs + cs + kC + tid) * H + h];
-      if (tid < kC) sBeta[tid] = tid < nrows ? fast_beta<SG>(b_cur) : 0.f;
+      if (tid < kC) sBeta[tid] = tid < nrows ? fast_beta(b_cur, beta_form(p.signed_gate)) : 0.f;
       if (nrows < kC) {
         // Rows past the sequence end hold another sequence's tokens or TMA fill.  They are
         // overwritten in the staging copy with q = k = v = 0 and a gate of exactly 1
@@ -925,7 +924,8 @@ bool chunk_tc_supported(const ChunkArgs &g) {
 int launch_chunk_tc(const ChunkArgs &g, cudaStream_t s) {
   if (g.n_seqs * g.H == 0) return CKDA_OK;
   const bool bf = g.o_dtype == CKDA_BF16;
-  switch (g.signed_gate) {
+  // the kernel is specialised on the gate's form; the strength's form is read at run time
+  switch (alpha_form(g.signed_gate)) {
     case 0: return bf ? launch_typed<__nv_bfloat16, 0>(g, s) : launch_typed<float, 0>(g, s);
     case 1: return bf ? launch_typed<__nv_bfloat16, 1>(g, s) : launch_typed<float, 1>(g, s);
     default: return bf ? launch_typed<__nv_bfloat16, 2>(g, s) : launch_typed<float, 2>(g, s);

@@ -68,7 +68,7 @@ int ckda_chunk_fwd(const void *q, const void *k, const void *v, const void *a, c
   if (!q || !k || !v || !a || !b) return CKDA_ERR_NULL;
   if (!valid_dim(dk) || !valid_dim(dv) || B < 0 || T < 0 || H <= 0) return CKDA_ERR_DIM;
   if (chunk != 16 && chunk != 32 && chunk != 64) return CKDA_ERR_CHUNK;
-  if (signed_gate < 0 || signed_gate > 2 || (io_dtype != CKDA_F32 && io_dtype != CKDA_BF16) ||
+  if (signed_gate < 0 || signed_gate > 4 || (io_dtype != CKDA_F32 && io_dtype != CKDA_BF16) ||
       (o_dtype != CKDA_F32 && o_dtype != CKDA_BF16))
     return CKDA_ERR_DTYPE;
   int N = B;
@@ -105,7 +105,7 @@ int ckda_decode_step(const void *q, const void *k, const void *v, const void *a,
   if (!q || !k || !v || !a || !b || !S) return CKDA_ERR_NULL;
   if (!valid_dim(dk) || !valid_dim(dv) || B < 0 || H <= 0) return CKDA_ERR_DIM;
   if ((long long)B * H > (1LL << 31) - 1) return CKDA_ERR_DIM;
-  if (signed_gate < 0 || signed_gate > 2 || (io_dtype != CKDA_F32 && io_dtype != CKDA_BF16) ||
+  if (signed_gate < 0 || signed_gate > 4 || (io_dtype != CKDA_F32 && io_dtype != CKDA_BF16) ||
       (o_dtype != CKDA_F32 && o_dtype != CKDA_BF16))
     return CKDA_ERR_DTYPE;
   const uintptr_t in_sz = io_dtype == CKDA_BF16 ? 2 : 4, out_sz = o_dtype == CKDA_BF16 ? 2 : 4;

@@ -31,17 +31,30 @@ __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
   return __float2bfloat16_rn(x);
 }
 
-// Linear gate value alpha (decode path).  Exact at +-inf: KDA 1/0, CKDA +-1.
+// Gate forms: signed_gate 0 (KDA) widens no range and 1 (CKDA) both; 3 widens the gate range
+// alone and 4 the strength range alone (the single-range variants of the CKDA review's
+// Figure 6); 2 passes raw values.  The gate is sigma / 2 sigma - 1 / raw for alpha_form
+// 0 / 1 / 2, the strength sigma / 2 sigma / raw for beta_form 0 / 1 / 2.
+__host__ __device__ __forceinline__ constexpr int alpha_form(int signed_gate) {
+  return signed_gate == 3 ? 1 : (signed_gate == 4 ? 0 : signed_gate);
+}
+__host__ __device__ __forceinline__ constexpr int beta_form(int signed_gate) {
+  return signed_gate == 3 ? 0 : (signed_gate == 4 ? 1 : signed_gate);
+}
+
+// Linear gate value alpha (decode path).  Exact at +-inf: sigma 1/0, 2 sigma - 1 +-1.
 __device__ __forceinline__ float gate_alpha(float a, int signed_gate) {
-  if (signed_gate == 0) return 1.0f / (1.0f + expf(-a));
-  if (signed_gate == 1) return tanhf(0.5f * a);  // 2 sigma(a) - 1 == tanh(a/2)
+  const int f = alpha_form(signed_gate);
+  if (f == 0) return 1.0f / (1.0f + expf(-a));
+  if (f == 1) return tanhf(0.5f * a);  // 2 sigma(a) - 1 == tanh(a/2)
   return a;
 }
 
-// Strength beta.  Exact at +-inf: KDA 1/0, CKDA 2/0.
+// Strength beta.  Exact at +-inf: sigma 1/0, 2 sigma 2/0.
 __device__ __forceinline__ float gate_beta(float b, int signed_gate) {
-  if (signed_gate == 0) return 1.0f / (1.0f + expf(-b));
-  if (signed_gate == 1) return 2.0f / (1.0f + expf(-b));
+  const int f = beta_form(signed_gate);
+  if (f == 0) return 1.0f / (1.0f + expf(-b));
+  if (f == 1) return 2.0f / (1.0f + expf(-b));
   return b;
 }
 
@@ -51,13 +64,14 @@ __device__ __forceinline__ float gate_beta(float b, int signed_gate) {
 //   raw : log |a|;                            zero iff a == 0
 __device__ __forceinline__ void gate_log2(float a, int signed_gate, float &log2abs, bool &is_zero,
                                           bool &is_neg) {
-  if (signed_gate == 0) {
+  const int f = alpha_form(signed_gate);
+  if (f == 0) {
     is_neg = false;
     is_zero = (a == -INFINITY);
     const float x = -a;  // softplus(x) = max(x, 0) + log1p(exp(-|x|))
     const float sp = fmaxf(x, 0.0f) + log1pf(expf(-fabsf(x)));
     log2abs = is_zero ? 0.0f : -sp * kInvLn2;
-  } else if (signed_gate == 1) {
+  } else if (f == 1) {
     is_neg = (a < 0.0f);
     is_zero = (a == 0.0f);
     const float x = fabsf(a);

@@ -12,6 +12,8 @@
  *   alpha_t = sigma(a_t)            beta_t = sigma(b_t)       (KDA,  signed_gate = 0)
  *   alpha_t = 2 sigma(a_t) - 1      beta_t = 2 sigma(b_t)     (CKDA, signed_gate = 1)
  *   alpha_t = a_t                   beta_t = b_t              (raw,  signed_gate = 2)
+ *   alpha_t = 2 sigma(a_t) - 1      beta_t = sigma(b_t)       (gate range only, 3)
+ *   alpha_t = sigma(a_t)            beta_t = 2 sigma(b_t)     (strength range only, 4)
  *
  *   S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
  *   o_t = S_t^T q_t
@@ -53,20 +55,33 @@
 /* sigma(x) = 1 / (1 + e^{-x}); exact 1 at +inf and 0 at -inf. */
 static double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
 
-/* Gate activation, "Method steps" step 1 of the CKDA review. */
+/*
+ * Gate activation, "Method steps" step 1 of the CKDA review (both ranges widened),
+ * and the single-range variants of its "Experimental results" (Figure 6): the gate
+ * range alone (3) or the strength range alone (4).  Per form: the gate is
+ * sigma (0, 4), 2 sigma - 1 (1, 3) or the raw value (2); the strength is sigma
+ * (0, 3), 2 sigma (1, 4) or the raw value (2).
+ */
+static int alpha_form(int signed_gate) {
+    return signed_gate == 3 ? 1 : (signed_gate == 4 ? 0 : signed_gate);
+}
+static int beta_form(int signed_gate) {
+    return signed_gate == 3 ? 0 : (signed_gate == 4 ? 1 : signed_gate);
+}
 static void gate_values(const double *a, double b, int n, int signed_gate,
                         double *alpha, double *beta) {
+    const int af = alpha_form(signed_gate), bf = beta_form(signed_gate);
     for (int i = 0; i < n; ++i) {
-        if (signed_gate == 0)
+        if (af == 0)
             alpha[i] = sigmoid(a[i]);
-        else if (signed_gate == 1)
+        else if (af == 1)
             alpha[i] = 2.0 * sigmoid(a[i]) - 1.0;
         else
             alpha[i] = a[i];
     }
-    if (signed_gate == 0)
+    if (bf == 0)
         *beta = sigmoid(b);
-    else if (signed_gate == 1)
+    else if (bf == 1)
         *beta = 2.0 * sigmoid(b);
     else
         *beta = b;
@@ -185,7 +200,7 @@ int oracle_ckda_fwd(const double *q, const double *k, const double *v, const dou
                     double *o, double *S_T, int n_threads) {
     if (!q || !k || !v || !a || !b) return ORACLE_ERR_ARG;
     if (B < 0 || T < 0 || H <= 0 || dk <= 0 || dv <= 0) return ORACLE_ERR_ARG;
-    if (signed_gate < 0 || signed_gate > 2) return ORACLE_ERR_ARG;
+    if (signed_gate < 0 || signed_gate > 4) return ORACLE_ERR_ARG;
     int N = B;
     if (cu_seqlens) {
         if (B != 1 || n_seqs < 0) return ORACLE_ERR_ARG;
@@ -231,7 +246,7 @@ int oracle_decode_step(const double *q, const double *k, const double *v, const 
                        int signed_gate, double *o) {
     if (!q || !k || !v || !a || !b || !S) return ORACLE_ERR_ARG;
     if (B < 0 || H <= 0 || dk <= 0 || dv <= 0) return ORACLE_ERR_ARG;
-    if (signed_gate < 0 || signed_gate > 2) return ORACLE_ERR_ARG;
+    if (signed_gate < 0 || signed_gate > 4) return ORACLE_ERR_ARG;
     double *alpha = (double *)malloc(sizeof(double) * (size_t)dk);
     double *p = (double *)malloc(sizeof(double) * (size_t)dv);
     if (!alpha || !p) { free(alpha); free(p); return ORACLE_ERR_NOMEM; }
@@ -266,7 +281,7 @@ int oracle_ckda_fwd_explicit(const double *q, const double *k, const double *v,
                              const double *a, const double *b, const double *S0,
                              int T, int dk, int dv, int signed_gate, double *o, double *S_T) {
     if (!q || !k || !v || !a || !b || !S_T) return ORACLE_ERR_ARG;
-    if (T < 0 || dk <= 0 || dv <= 0 || signed_gate < 0 || signed_gate > 2) return ORACLE_ERR_ARG;
+    if (T < 0 || dk <= 0 || dv <= 0 || signed_gate < 0 || signed_gate > 4) return ORACLE_ERR_ARG;
     double *A = (double *)malloc(sizeof(double) * (size_t)dk * dk);
     double *S = (double *)malloc(sizeof(double) * (size_t)dk * dv);
     double *N = (double *)malloc(sizeof(double) * (size_t)dk * dv);

@@ -14,6 +14,8 @@ on a mismatch, so the same checks run on the real oracle
   [LA]    CyFA blog, section 2.1 (linear attention S_t = S_{t-1} + k v^T)
   [DR]    CyFA blog, section 2.2 (delta rule S_t = S_{t-1} + k (v - S^T k)^T)
   [CHUNK] CyFA blog, section 5.5 (chunk = 1 and chunk = 64 must agree)
+  [FIG6]  "Complex KDA" review, "Experimental results", Figure 6 (the gate range or the
+          strength range widened alone)
 """
 from __future__ import annotations
 
@@ -78,6 +80,33 @@ def pin_gate_activation(orc):
     assert be1[0] == 0.0 and be1[-1] == 2.0 and be1[4] == 1.0
     assert al0[0] == 0.0 and al0[-1] == 1.0 and al0[4] == 0.5
     assert np.array_equal(al2, a) and np.array_equal(be2, a)
+
+
+def pin_single_range_variants(orc):
+    """[FIG6]: signed_gate 3 widens the gate range alone (alpha = 2 sigma(a) - 1 = tanh(a/2),
+    beta = sigma(b)), 4 the strength range alone (alpha = sigma(a), beta = 2 sigma(b)).  The
+    gates against tanh closed forms, and a whole forward in each form against the raw form
+    fed with those closed forms."""
+    a = np.array([-INF, -30.0, -3.0, -0.7, 0.0, 1e-9, 0.7, 3.0, 30.0, INF])
+    th = np.tanh(a / 2)
+    al3, be3 = orc.gates(a, a, 3)
+    al4, be4 = orc.gates(a, a, 4)
+    assert np.allclose(al3, th, rtol=1e-13, atol=1e-15)
+    assert np.allclose(be3, (1 + th) / 2, rtol=1e-13, atol=1e-15)
+    assert np.allclose(al4, (1 + th) / 2, rtol=1e-13, atol=1e-15)
+    assert np.allclose(be4, 1 + th, rtol=1e-13, atol=1e-15)
+    assert al3[0] == -1.0 and al3[-1] == 1.0 and be3[0] == 0.0 and be3[-1] == 1.0
+    assert al4[0] == 0.0 and al4[-1] == 1.0 and be4[0] == 0.0 and be4[-1] == 2.0
+    rng = np.random.default_rng(61)
+    T, dk, dv = 23, 5, 3
+    q, k, v = _unit(rng, T, dk), _unit(rng, T, dk), rng.standard_normal((T, dv))
+    la, lb = rng.standard_normal((T, dk)) * 2, rng.standard_normal(T) * 2
+    S0 = rng.standard_normal((dk, dv))
+    sig = lambda x: (1 + np.tanh(x / 2)) / 2
+    for sg, alpha, beta in ((3, np.tanh(la / 2), sig(lb)), (4, sig(la), 1 + np.tanh(lb / 2))):
+        o, S = _one(orc, q, k, v, la, lb, S0, signed_gate=sg)
+        ro, rS = _one(orc, q, k, v, alpha, beta, S0, signed_gate=2)
+        assert _rel(o, ro) < 1e-12 and _rel(S, rS) < 1e-12, sg
 
 
 # ------------------------------------------------------- closed-form cases

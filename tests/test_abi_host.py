@@ -91,7 +91,7 @@ def _dec(lib, **kw):
     (dict(dk=24), -2), (dict(dv=256), -2), (dict(H=0), -2), (dict(T=-1), -2), (dict(B=-1), -2),
     (dict(cu=P, B=2, n_seqs=1), -2),
     (dict(chunk=128), -3), (dict(chunk=8), -3),
-    (dict(sg=3), -4), (dict(io=2), -4), (dict(od=-1), -4),
+    (dict(sg=5), -4), (dict(io=2), -4), (dict(od=-1), -4),
     (dict(k=MIS), -5), (dict(o=MIS), -5), (dict(S0=MIS), -5), (dict(S_T=MIS), -5),
     (dict(b=ODD), -5), (dict(cu=ODD), -5),
     (dict(ws=None), -7), (dict(wsb=16), -7), (dict(ws=ctypes.c_void_p((1 << 20) + 16)), -7),

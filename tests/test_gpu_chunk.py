@@ -314,3 +314,14 @@ def test_tc_small_gate_logits(cuda_lib, sg):
     o, S = run_gpu(cuda_lib, inp, w)
     ro, rS = oracle_prefill(inp, sg)
     assert rel(f64(o), ro) <= TOL_BF16 and rel(f64(S), rS) <= TOL_BF16
+
+
+@pytest.mark.parametrize("signed_gate", [3, 4], ids=["gate_range", "strength_range"])
+def test_single_range_variants(cuda_lib, signed_gate):
+    """The gate range or the strength range widened alone (CKDA review, Figure 6) on both
+    prefill paths: exact fp32 (d=64, chunk 32) and tensor-core bf16 (d=128, chunk 64)."""
+    w32 = synth.CKDA_SPREAD.with_(B=2, T=150, H=2, dk=64, dv=64, chunk=32,
+                                  signed_gate=signed_gate, io_dtype="f32", o_dtype="f32")
+    check(cuda_lib, w32, seed=7, tol=TOL_FP32)
+    wtc = synth.CKDA_SPREAD.with_(B=2, T=300, H=3, signed_gate=signed_gate, o_dtype="f32")
+    check(cuda_lib, wtc, seed=8)

@@ -112,3 +112,17 @@ def test_full_decode_sampled(cuda_lib):
     gS = f64(S).reshape(w.B * w.H, w.dk, w.dv)[heads]
     assert rel(go, ro) <= TOL_BF16
     assert rel(gS, rS) <= TOL_BF16
+
+
+@pytest.mark.parametrize("signed_gate", [3, 4], ids=["gate_range", "strength_range"])
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_decode_single_range_variants(cuda_lib, signed_gate, io):
+    """The gate range or the strength range widened alone (CKDA review, Figure 6)."""
+    w = synth.DECODE.with_(B=2, H=5, signed_gate=signed_gate, gate="spread", strength="spread",
+                           io_dtype=io, o_dtype="f32")
+    inp = synth.make_decode(w, seed=5, steps=24)
+    o, S = run_steps(cuda_lib, inp, signed_gate)
+    ro, rS = oracle_steps(inp, signed_gate)
+    tol = TOL_FP32 if io == "f32" else TOL_BF16
+    assert rel(f64(o).reshape(ro.shape[0], -1), ro.reshape(ro.shape[0], -1)) <= tol
+    assert rel(f64(S).reshape(rS.shape), rS) <= tol
