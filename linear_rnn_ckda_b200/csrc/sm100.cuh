@@ -295,10 +295,12 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar) {
       : "memory");
 }
 
+// fp32 -> tf32, round to nearest with ties away from zero (the rounding of cvt.rna.tf32):
+// tf32 keeps the top 10 of the 23 mantissa bits, so add half of the dropped 13-bit unit to
+// the magnitude bits and clear them (a carry moves into the exponent as it should).
+// Integer arithmetic, so it issues on the integer pipe beside the fp32 work.
 __device__ __forceinline__ uint32_t to_tf32(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-  return r;
+  return (__float_as_uint(x) + 0x1000u) & 0xFFFFE000u;
 }
 
 }  // namespace sm100
