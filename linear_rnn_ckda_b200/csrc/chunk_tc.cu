@@ -480,8 +480,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int rr = 0; rr < 8; ++rr) {
         float a0, a1, al0, al1, ial0, ial1;
         ldbf2(sta, 8 * rg + rr, a0, a1);
-        gate2(a0, al0, ial0);
-        gate2(a1, al1, ial1);
+        if (SG == 1) {
+          // the pair's CKDA ratios in packed fp32 pairs (same arithmetic as gate2)
+          const uint64_t one = f2pk(1.f, 1.f);
+          const uint64_t e = f2pk(__expf(-fabsf(a0)), __expf(-fabsf(a1)));
+          const uint64_t num = f2sub(one, e), den = f2add(one, e);
+          float p0, p1;
+          f2up(f2mul(num, den), p0, p1);
+          const uint64_t rr2 = f2pk(__fdividef(1.f, p0), __fdividef(1.f, p1));
+          float m0, m1, n0, n1;
+          f2up(f2mul(num, f2mul(num, rr2)), m0, m1);
+          f2up(f2mul(den, f2mul(den, rr2)), n0, n1);
+          al0 = copysignf(m0, a0);
+          al1 = copysignf(m1, a1);
+          ial0 = copysignf(n0, a0);
+          ial1 = copysignf(n1, a1);
+        } else {
+          gate2(a0, al0, ial0);
+          gate2(a1, al1, ial1);
+        }
         run0 *= al0;
         run1 *= al1;
         g[2 * rr] = run0;
