@@ -487,14 +487,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t num = f2sub(one, e), den = f2add(one, e);
           float p0, p1;
           f2up(f2mul(num, den), p0, p1);
-          const uint64_t rr2 = f2pk(__fdividef(1.f, p0), __fdividef(1.f, p1));
-          float m0, m1, n0, n1;
-          f2up(f2mul(num, f2mul(num, rr2)), m0, m1);
-          f2up(f2mul(den, f2mul(den, rr2)), n0, n1);
-          al0 = copysignf(m0, a0);
-          al1 = copysignf(m1, a1);
-          ial0 = copysignf(n0, a0);
-          ial1 = copysignf(n1, a1);
+          // the gate's sign rides on the shared reciprocal: num^2 r and den^2 r take it
+          const uint64_t rr2 = f2pk(copysignf(__fdividef(1.f, p0), a0),
+                                    copysignf(__fdividef(1.f, p1), a1));
+          f2up(f2mul(num, f2mul(num, rr2)), al0, al1);
+          f2up(f2mul(den, f2mul(den, rr2)), ial0, ial1);
         } else {
           gate2(a0, al0, ial0);
           gate2(a1, al1, ial1);
