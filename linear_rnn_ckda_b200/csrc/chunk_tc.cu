@@ -727,11 +727,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             *reinterpret_cast<float4 *>(sA + t * kAS + 16 * qg + 4 * y) =
                 make_float4(av[4 * y], av[4 * y + 1], av[4 * y + 2], av[4 * y + 3]);
         } else {
+          // four consecutive columns of row t per 16-byte store (one store per row and
+          // 16-byte piece keeps the 32 rows of a warp on distinct bank groups)
           const int t = jrow - 64;
 #pragma unroll
-          for (int x = 0; x < 16; ++x) {
-            const int j = 16 * qg + x;
-            st_tf32(sPK, swpk(t, j), j <= t ? __uint_as_float(r[x]) : 0.f);
+          for (int y = 0; y < 4; ++y) {
+            uint32_t w4[4];
+#pragma unroll
+            for (int z = 0; z < 4; ++z) {
+              const int x = 4 * y + z, j = 16 * qg + x;
+              w4[z] = to_tf32(j <= t ? __uint_as_float(r[x]) : 0.f);
+            }
+            *reinterpret_cast<uint4 *>(sPK + swpk(t, 16 * qg + 4 * y)) =
+                make_uint4(w4[0], w4[1], w4[2], w4[3]);
           }
         }
       }
