@@ -574,12 +574,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             make_float2(kc[2 * rr], kc[2 * rr + 1]);
     };
     auto store_kct_tile = [&]() {  // Kc^T (rows 2pc and 2pc + 1, four t per 16-byte store)
+      // the first store of a lane takes row 2pc + ((pc >> 2) & 1), the second the other one,
+      // so the 32 rows of one store instruction fall on all eight 16-byte bank groups
+      const int e0 = (pc >> 2) & 1;
 #pragma unroll
-      for (int e = 0; e < 2; ++e)
+      for (int k = 0; k < 2; ++k) {
+        const int e = e0 ^ k;
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf)
+        for (int hf = 0; hf < 2; ++hf) {
+          const float x0 = e ? kc[8 * hf + 1] : kc[8 * hf], x1 = e ? kc[8 * hf + 3] : kc[8 * hf + 2];
+          const float x2 = e ? kc[8 * hf + 5] : kc[8 * hf + 4], x3 = e ? kc[8 * hf + 7] : kc[8 * hf + 6];
           *reinterpret_cast<float4 *>(sPK + swpk(64 + ch0 + e, 8 * rg + 4 * hf)) =
-              make_float4(kc[8 * hf + e], kc[8 * hf + 2 + e], kc[8 * hf + 4 + e], kc[8 * hf + 6 + e]);
+              make_float4(x0, x1, x2, x3);
+        }
+      }
     };
     auto store_kc = [&]() {
       store_kc_tile();
