@@ -40,7 +40,7 @@
  *     No entry point aborts, throws or traps; device-side checks (offsets in
  *     cu_seqlens, bounded waits) set a status word in the workspace that
  *     ckda_workspace_status() reads back.
- *   - NaN or Inf in q, k, v give undefined values but no fault.
+ *   - NaN or Inf in q, k, v, and NaN in a or b, give undefined values but no fault.
  */
 #ifndef CKDA_H
 #define CKDA_H

@@ -448,8 +448,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     //   KDA   sigma(a) = 1 / (1 + e^{-a}), inverse 1 + e^{-a}
     //   CKDA  2 sigma(a) - 1 = tanh(a/2) = sign(a) (1 - e^{-|a|}) / (1 + e^{-|a|}), inverse the
     //         ratio upside down; both from one reciprocal r = 1 / (num den) (num r = 1 / den,
-    //         den r = 1 / num).  For small |a| the difference 1 - e^{-|a|} cancels: the gate's
-    //         error stays at fp32 rounding level in absolute terms; an exactly zero gate stays 0.
+    //         den r = 1 / num).  Small |a|: 1 - e^{-|a|} cancels, an error at fp32 rounding level
+    //         in absolute terms.  a = 0 gives 0 or NaN (0 inf): either fails the range check.
     auto gate2 = [&](float a, float &al, float &ial) {
       if (SG == 0) {
         const float e = __expf(-a);
