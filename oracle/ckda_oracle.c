@@ -35,6 +35,14 @@
  * The recurrence has no 1/sqrt(dk) scale on q (none appears on the pages);
  * o_t uses the state after token t's update.
  *
+ * Backward (oracle_ckda_bwd): the gradients of L = sum dO . o + sum dS_T . S_T
+ * with respect to q, k, v, a, b and S0, by the chain rule taken through the
+ * same token steps in reverse order (states recomputed from checkpoints).  The
+ * pages give no backward formulas; they measure the kernels forward plus
+ * backward ("Complex KDA" review, Figure 5), and the reverse pass here is the
+ * plain derivative of the forward above, pinned by finite differences and
+ * closed forms in the tests.
+ *
  * Layouts (all dense, row-major, float64):
  *   q, k, a : [B, T, H, dk]      v, o : [B, T, H, dv]     b : [B, T, H]
  *   S0, S_T : [N, H, dk, dv]     N = B, or n_seqs when cu_seqlens != NULL
@@ -85,6 +93,20 @@ static void gate_values(const double *a, double b, int n, int signed_gate,
         *beta = 2.0 * sigmoid(b);
     else
         *beta = b;
+}
+
+/*
+ * Derivatives of the activations, same forms as gate_values:
+ * sigma'(x) = sigma(x) sigma(-x) (so 0 at +-inf), twice that for 2 sigma - 1 and
+ * 2 sigma, and 1 for raw values.
+ */
+static double sigmoid_deriv(double x) { return sigmoid(x) * sigmoid(-x); }
+static void gate_derivs(const double *a, double b, int n, int signed_gate,
+                        double *dalpha_da, double *dbeta_db) {
+    const int af = alpha_form(signed_gate), bf = beta_form(signed_gate);
+    for (int i = 0; i < n; ++i)
+        dalpha_da[i] = af == 0 ? sigmoid_deriv(a[i]) : (af == 1 ? 2.0 * sigmoid_deriv(a[i]) : 1.0);
+    *dbeta_db = bf == 0 ? sigmoid_deriv(b) : (bf == 1 ? 2.0 * sigmoid_deriv(b) : 1.0);
 }
 
 /* Elementwise activation of n_a gate logits and n_b strength logits. */
@@ -229,6 +251,227 @@ int oracle_ckda_fwd(const double *q, const double *k, const double *v, const dou
         for (int i = 0; i < n_threads; ++i)
             if (pthread_create(&th[i], NULL, fwd_worker, &J) == 0) ++started;
         if (started == 0) fwd_worker(&J);
+        for (int i = 0; i < started; ++i) pthread_join(th[i], NULL);
+        free(th);
+    }
+    pthread_mutex_destroy(&J.lock);
+    return J.status;
+}
+
+/*
+ * Reverse of token_step for one token.  S_prev = S_{t-1}, S_cur = S_t.  On entry
+ * dS holds dL/dS_t from the later tokens (and dS_T); on return dL/dS_{t-1}.
+ * Forward quantities:  St = Diag(alpha) S_prev,  p = St^T k,  u = beta (v - p),
+ * S_t = St + k u^T,  o = S_t^T q.  Their adjoints, in reverse:
+ *   o:   dS += q dO^T,            dq = S_t dO
+ *   S_t: dSt = dS,  dk = dS u,    du = dS^T k
+ *   u:   dbeta = du . (v - p),    dv = beta du,   dp = -beta du
+ *   p:   dSt += k dp^T,           dk += St dp
+ *   St:  dalpha_i = sum_j dSt_ij S_prev_ij,       dS_{t-1} = Diag(alpha) dSt
+ * and da = dalpha * alpha'(a), db = dbeta * beta'(b).  dO may be NULL (zero).
+ */
+static void token_step_bwd(const double *S_prev, const double *S_cur, const double *q,
+                           const double *k, const double *v, const double *alpha, double beta,
+                           const double *dalpha_da, double dbeta_db, const double *dO,
+                           int dk, int dv, double *dS, double *dq, double *dk_out,
+                           double *dv_out, double *da, double *db, double *St, double *p,
+                           double *du) {
+    for (int i = 0; i < dk; ++i) {
+        double acc = 0.0;
+        if (dO)
+            for (int j = 0; j < dv; ++j) {
+                dS[(size_t)i * dv + j] += q[i] * dO[j];
+                acc += S_cur[(size_t)i * dv + j] * dO[j];
+            }
+        dq[i] = acc;
+    }
+    for (int i = 0; i < dk; ++i)
+        for (int j = 0; j < dv; ++j) St[(size_t)i * dv + j] = alpha[i] * S_prev[(size_t)i * dv + j];
+    for (int j = 0; j < dv; ++j) {
+        double acc = 0.0;
+        for (int i = 0; i < dk; ++i) acc += k[i] * St[(size_t)i * dv + j];
+        p[j] = acc;
+    }
+    for (int i = 0; i < dk; ++i) {
+        double acc = 0.0;
+        for (int j = 0; j < dv; ++j) acc += dS[(size_t)i * dv + j] * beta * (v[j] - p[j]);
+        dk_out[i] = acc;
+    }
+    double dbeta = 0.0;
+    for (int j = 0; j < dv; ++j) {
+        double acc = 0.0;
+        for (int i = 0; i < dk; ++i) acc += dS[(size_t)i * dv + j] * k[i];
+        du[j] = acc;
+        dbeta += acc * (v[j] - p[j]);
+        dv_out[j] = beta * acc;
+    }
+    /* dp = -beta du */
+    for (int i = 0; i < dk; ++i) {
+        double acc = 0.0;
+        for (int j = 0; j < dv; ++j) acc += St[(size_t)i * dv + j] * (-beta * du[j]);
+        dk_out[i] += acc;
+    }
+    for (int i = 0; i < dk; ++i)
+        for (int j = 0; j < dv; ++j) dS[(size_t)i * dv + j] += k[i] * (-beta * du[j]);
+    for (int i = 0; i < dk; ++i) {
+        double acc = 0.0;
+        for (int j = 0; j < dv; ++j) acc += dS[(size_t)i * dv + j] * S_prev[(size_t)i * dv + j];
+        da[i] = acc * dalpha_da[i];
+        for (int j = 0; j < dv; ++j) dS[(size_t)i * dv + j] *= alpha[i];
+    }
+    *db = dbeta * dbeta_db;
+}
+
+typedef struct {
+    const double *q, *k, *v, *a, *b, *S0, *dO, *dS_T;
+    const int32_t *cu;
+    int B, T, H, dk, dv, signed_gate;
+    double *gq, *gk, *gv, *ga, *gb, *gS0; /* outputs: dq, dk, dv, da, db, dS0 */
+    int n_units;
+    int next_unit; /* guarded by lock */
+    pthread_mutex_t lock;
+    int status;
+} bwd_job;
+
+#define BWD_SEG 64 /* tokens between state checkpoints */
+
+static int run_unit_bwd(bwd_job *J, int unit) {
+    const int H = J->H, dk = J->dk, dv = J->dv;
+    const int n = unit / H, h = unit % H;
+    const size_t dd = (size_t)dk * dv;
+    long t0, t1, bofs;
+    if (J->cu) {
+        t0 = J->cu[n];
+        t1 = J->cu[n + 1];
+        bofs = 0;
+    } else {
+        t0 = 0;
+        t1 = J->T;
+        bofs = (long)n * J->T;
+    }
+    const long len = t1 - t0;
+    const long n_seg = (len + BWD_SEG - 1) / BWD_SEG;
+    const size_t sofs = ((size_t)n * H + h) * dd;
+    /* checkpoints: the state before each segment; states: one segment's S_{t-1}, S_t chain */
+    double *ckpt = (double *)malloc(sizeof(double) * dd * (size_t)(n_seg > 0 ? n_seg : 1));
+    double *states = (double *)malloc(sizeof(double) * dd * (BWD_SEG + 1));
+    double *dS = (double *)malloc(sizeof(double) * dd);
+    double *St = (double *)malloc(sizeof(double) * dd);
+    double *alpha = (double *)malloc(sizeof(double) * (size_t)dk);
+    double *dalpha = (double *)malloc(sizeof(double) * (size_t)dk);
+    double *p = (double *)malloc(sizeof(double) * (size_t)dv);
+    double *du = (double *)malloc(sizeof(double) * (size_t)dv);
+    int rc = ORACLE_OK;
+    if (!ckpt || !states || !dS || !St || !alpha || !dalpha || !p || !du) {
+        rc = ORACLE_ERR_NOMEM;
+        goto done;
+    }
+    /* forward, keeping the state at every segment start */
+    if (J->S0) memcpy(St, J->S0 + sofs, sizeof(double) * dd);
+    else memset(St, 0, sizeof(double) * dd);
+    for (long t = t0; t < t1; ++t) {
+        if ((t - t0) % BWD_SEG == 0) memcpy(ckpt + (size_t)((t - t0) / BWD_SEG) * dd, St, sizeof(double) * dd);
+        const size_t row = (size_t)(bofs + t) * H + h;
+        double beta;
+        gate_values(J->a + row * dk, J->b[row], dk, J->signed_gate, alpha, &beta);
+        token_step(St, J->q + row * dk, J->k + row * dk, J->v + row * dv, alpha, beta, dk, dv,
+                   NULL, p);
+    }
+    if (J->dS_T) memcpy(dS, J->dS_T + sofs, sizeof(double) * dd);
+    else memset(dS, 0, sizeof(double) * dd);
+    for (long sg = n_seg - 1; sg >= 0; --sg) {
+        const long s0 = t0 + sg * BWD_SEG;
+        const long s1 = s0 + BWD_SEG < t1 ? s0 + BWD_SEG : t1;
+        memcpy(states, ckpt + (size_t)sg * dd, sizeof(double) * dd);
+        for (long t = s0; t < s1; ++t) {
+            const size_t row = (size_t)(bofs + t) * H + h;
+            double beta;
+            double *S = states + (size_t)(t - s0 + 1) * dd;
+            memcpy(S, S - dd, sizeof(double) * dd);
+            gate_values(J->a + row * dk, J->b[row], dk, J->signed_gate, alpha, &beta);
+            token_step(S, J->q + row * dk, J->k + row * dk, J->v + row * dv, alpha, beta, dk, dv,
+                       NULL, p);
+        }
+        for (long t = s1 - 1; t >= s0; --t) {
+            const size_t row = (size_t)(bofs + t) * H + h;
+            double beta, dbeta_db;
+            gate_values(J->a + row * dk, J->b[row], dk, J->signed_gate, alpha, &beta);
+            gate_derivs(J->a + row * dk, J->b[row], dk, J->signed_gate, dalpha, &dbeta_db);
+            const double *S_cur = states + (size_t)(t - s0 + 1) * dd;
+            token_step_bwd(S_cur - dd, S_cur, J->q + row * dk, J->k + row * dk, J->v + row * dv,
+                           alpha, beta, dalpha, dbeta_db, J->dO ? J->dO + row * dv : NULL, dk, dv,
+                           dS, J->gq + row * dk, J->gk + row * dk, J->gv + row * dv,
+                           J->ga + row * dk, J->gb + row, St, p, du);
+        }
+    }
+    if (J->gS0) memcpy(J->gS0 + sofs, dS, sizeof(double) * dd);
+done:
+    free(ckpt); free(states); free(dS); free(St); free(alpha); free(dalpha); free(p); free(du);
+    return rc;
+}
+
+static void *bwd_worker(void *arg) {
+    bwd_job *J = (bwd_job *)arg;
+    for (;;) {
+        pthread_mutex_lock(&J->lock);
+        int u = J->next_unit++;
+        pthread_mutex_unlock(&J->lock);
+        if (u >= J->n_units) break;
+        if (run_unit_bwd(J, u) != ORACLE_OK) {
+            pthread_mutex_lock(&J->lock);
+            J->status = ORACLE_ERR_NOMEM;
+            pthread_mutex_unlock(&J->lock);
+        }
+    }
+    return NULL;
+}
+
+/*
+ * Gradients of L = sum dO . o + sum dS_T . S_T for the forward of oracle_ckda_fwd
+ * (same arguments, layouts and gate forms).  dO [B,T,H,dv] and dS_T [N,H,dk,dv]
+ * may each be NULL (zero).  Outputs, all written: dq, dk, da [B,T,H,dk],
+ * dv [B,T,H,dv], db [B,T,H], dS0 [N,H,dk,dv] (dS0 may be NULL: not written).
+ * Every token belongs to exactly one sequence (cu_seqlens[N] == T is required),
+ * so every element of dq, dk, dv, da, db is written.
+ */
+int oracle_ckda_bwd(const double *q, const double *k, const double *v, const double *a,
+                    const double *b, const double *S0, const int32_t *cu_seqlens,
+                    int n_seqs, int B, int T, int H, int dk, int dv, int signed_gate,
+                    const double *dO, const double *dS_T, double *dq, double *dk_out,
+                    double *dv_out, double *da, double *db, double *dS0, int n_threads) {
+    if (!q || !k || !v || !a || !b || !dq || !dk_out || !dv_out || !da || !db)
+        return ORACLE_ERR_ARG;
+    if (B < 0 || T < 0 || H <= 0 || dk <= 0 || dv <= 0) return ORACLE_ERR_ARG;
+    if (signed_gate < 0 || signed_gate > 4) return ORACLE_ERR_ARG;
+    int N = B;
+    if (cu_seqlens) {
+        if (B != 1 || n_seqs < 0) return ORACLE_ERR_ARG;
+        if (cu_seqlens[0] != 0 || cu_seqlens[n_seqs] != T) return ORACLE_ERR_SEQLENS;
+        for (int i = 0; i < n_seqs; ++i)
+            if (cu_seqlens[i + 1] < cu_seqlens[i]) return ORACLE_ERR_SEQLENS;
+        N = n_seqs;
+    }
+    bwd_job J;
+    J.q = q; J.k = k; J.v = v; J.a = a; J.b = b; J.S0 = S0; J.dO = dO; J.dS_T = dS_T;
+    J.cu = cu_seqlens; J.B = B; J.T = T; J.H = H; J.dk = dk; J.dv = dv;
+    J.signed_gate = signed_gate;
+    J.gq = dq; J.gk = dk_out; J.gv = dv_out; J.ga = da; J.gb = db; J.gS0 = dS0;
+    J.n_units = N * H; J.next_unit = 0; J.status = ORACLE_OK;
+    pthread_mutex_init(&J.lock, NULL);
+    if (n_threads <= 0) {
+        long nc = sysconf(_SC_NPROCESSORS_ONLN);
+        n_threads = nc > 0 ? (int)nc : 1;
+    }
+    if (n_threads > J.n_units) n_threads = J.n_units > 0 ? J.n_units : 1;
+    if (n_threads <= 1) {
+        bwd_worker(&J);
+    } else {
+        pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)n_threads);
+        if (!th) { pthread_mutex_destroy(&J.lock); return ORACLE_ERR_NOMEM; }
+        int started = 0;
+        for (int i = 0; i < n_threads; ++i)
+            if (pthread_create(&th[i], NULL, bwd_worker, &J) == 0) ++started;
+        if (started == 0) bwd_worker(&J);
         for (int i = 0; i < started; ++i) pthread_join(th[i], NULL);
         free(th);
     }

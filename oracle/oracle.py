@@ -60,6 +60,10 @@ class Oracle:
         lib.oracle_ckda_fwd.restype = _i
         lib.oracle_ckda_fwd.argtypes = [_dp, _dp, _dp, _dp, _dp, _dp, _ip,
                                         _i, _i, _i, _i, _i, _i, _i, _dp, _dp, _i]
+        lib.oracle_ckda_bwd.restype = _i
+        lib.oracle_ckda_bwd.argtypes = [_dp, _dp, _dp, _dp, _dp, _dp, _ip,
+                                        _i, _i, _i, _i, _i, _i, _i,
+                                        _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp, _i]
         lib.oracle_decode_step.restype = _i
         lib.oracle_decode_step.argtypes = [_dp, _dp, _dp, _dp, _dp, _dp, _i, _i, _i, _i, _i, _dp]
         lib.oracle_transition.restype = None
@@ -104,6 +108,34 @@ class Oracle:
         if rc != 0:
             raise ValueError(f"oracle_ckda_fwd failed with code {rc}")
         return o, S_T
+
+    def ckda_bwd(self, q, k, v, a, b, S0=None, dO=None, dS_T=None, cu_seqlens=None,
+                 signed_gate: int = 1, threads: int = 0):
+        """Gradients of L = sum(dO * o) + sum(dS_T * S_T) for ``ckda_fwd`` on the same
+        arguments; dO [B,T,H,dv] and dS_T [N,H,dk,dv] default to zero.
+        Returns (dq, dk, dv, da, db, dS0) with the shapes of q, k, v, a, b and
+        [N,H,dk,dv]."""
+        q, k, v, a, b = (_f64(x) for x in (q, k, v, a, b))
+        B, T, H, dk = q.shape
+        dv = v.shape[-1]
+        cu_p, N = None, B
+        if cu_seqlens is not None:
+            cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+            N = cu.size - 1
+            cu_p = cu.ctypes.data_as(_ip)
+        S0 = None if S0 is None else _f64(S0)
+        dO = None if dO is None else _f64(dO)
+        dS_T = None if dS_T is None else _f64(dS_T)
+        gq, gk, gv, ga = (np.empty_like(x) for x in (q, k, v, a))
+        gb = np.empty_like(b)
+        gS0 = np.empty((N, H, dk, dv))
+        rc = self.lib.oracle_ckda_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(S0), cu_p,
+                                      N, B, T, H, dk, dv, int(signed_gate), _ptr(dO), _ptr(dS_T),
+                                      _ptr(gq), _ptr(gk), _ptr(gv), _ptr(ga), _ptr(gb), _ptr(gS0),
+                                      int(threads))
+        if rc != 0:
+            raise ValueError(f"oracle_ckda_bwd failed with code {rc}")
+        return gq, gk, gv, ga, gb, gS0
 
     def decode_step(self, q, k, v, a, b, S, signed_gate: int = 1):
         """One decode step.  Returns (o [B,H,dv], S_new [B,H,dk,dv]); S is not modified."""
@@ -161,6 +193,10 @@ def gates(*a, **kw):
 
 def ckda_fwd(*a, **kw):
     return default().ckda_fwd(*a, **kw)
+
+
+def ckda_bwd(*a, **kw):
+    return default().ckda_bwd(*a, **kw)
 
 
 def decode_step(*a, **kw):

@@ -16,6 +16,9 @@ on a mismatch, so the same checks run on the real oracle
   [CHUNK] CyFA blog, section 5.5 (chunk = 1 and chunk = 64 must agree)
   [FIG6]  "Complex KDA" review, "Experimental results", Figure 6 (the gate range or the
           strength range widened alone)
+  [FIG5]  same page, Figure 5 (the kernels are measured forward plus backward; the pages give
+          no backward formulas, so the backward oracle is pinned by calculus alone: finite
+          differences, Euler identities of the linear arguments, closed forms)
 """
 from __future__ import annotations
 
@@ -452,6 +455,155 @@ def pin_period_two(orc):
     assert _rel(S, S0) < 1e-13
     _, S1 = _one(orc, np.zeros((T - 1, n)), k[:-1], v[:-1], a[:-1], np.full(T - 1, INF), S0, 1)
     assert _rel(S1, orc.transition(k[0], np.ones(n), 2.0) @ S0 + 2 * np.outer(k[0], v[0])) < 1e-13
+
+
+# ---------------------------------------------------------------- backward ([FIG5])
+
+
+def _bwd_case(rng, B, T, H, dk, dv, n_seqs=None):
+    q = rng.standard_normal((B, T, H, dk))
+    k = _unit(rng, B, T, H, dk)
+    v = rng.standard_normal((B, T, H, dv))
+    a = rng.standard_normal((B, T, H, dk)) * 1.5
+    b = rng.standard_normal((B, T, H))
+    N = B if n_seqs is None else n_seqs
+    S0 = rng.standard_normal((N, H, dk, dv))
+    dO = rng.standard_normal((B, T, H, dv))
+    dS_T = rng.standard_normal((N, H, dk, dv))
+    return [q, k, v, a, b, S0], dO, dS_T
+
+
+def _check_fd(orc, args, dO, dS_T, sg, cu=None, h=1e-5, tol=1e-7):
+    """Central differences of L = sum dO . o + sum dS_T . S_T in every input element."""
+    def loss(xs):
+        o, S = orc.ckda_fwd(*xs, cu_seqlens=cu, signed_gate=sg, threads=1)
+        return float((dO * o).sum() + (dS_T * S).sum())
+
+    grads = orc.ckda_bwd(*args, dO=dO, dS_T=dS_T, cu_seqlens=cu, signed_gate=sg, threads=1)
+    for idx, (x, g) in enumerate(zip(args, grads)):
+        fd = np.empty_like(x)
+        for e in range(x.size):
+            xs = list(args)
+            xp, xm = x.copy(), x.copy()
+            xp.flat[e] += h
+            xm.flat[e] -= h
+            xs[idx] = xp
+            lp = loss(xs)
+            xs[idx] = xm
+            fd.flat[e] = (lp - loss(xs)) / (2 * h)
+        assert _rel(g, fd) < tol, ("q k v a b S0".split()[idx], sg, _rel(g, fd))
+
+
+def pin_bwd_finite_differences(orc):
+    """[FIG5] every gradient of the backward oracle equals central finite differences of the
+    forward, in all five gate forms; and across state checkpoints (sequences longer than 64
+    tokens) with packed sequences, one of them empty."""
+    rng = np.random.default_rng(70)
+    args, dO, dS_T = _bwd_case(rng, 2, 11, 2, 3, 4)
+    for sg in range(5):
+        _check_fd(orc, args, dO, dS_T, sg)
+    cu = np.array([0, 70, 70, 150], dtype=np.int32)
+    args, dO, dS_T = _bwd_case(rng, 1, 150, 1, 2, 3, n_seqs=3)
+    _check_fd(orc, args, dO, dS_T, 1, cu=cu)
+
+
+def pin_bwd_euler_identities(orc):
+    """[FIG5] exact identities of the linear arguments (Euler's theorem for functions of degree
+    one): o is linear in q and S_T does not depend on q, so sum dq . q = sum dO . o; o and S_T
+    are jointly linear in (v, S0), so sum dv . v + sum dS0 . S0 = L."""
+    rng = np.random.default_rng(71)
+    for sg in (0, 1):
+        args, dO, dS_T = _bwd_case(rng, 2, 150, 2, 8, 6)
+        q, k, v, a, b, S0 = args
+        o, S = orc.ckda_fwd(*args, signed_gate=sg, threads=2)
+        L = (dO * o).sum() + (dS_T * S).sum()
+        dq, dk, dv, da, db, dS0 = orc.ckda_bwd(*args, dO=dO, dS_T=dS_T, signed_gate=sg, threads=2)
+        assert abs((dq * q).sum() - (dO * o).sum()) < 1e-12 * np.abs(dO * o).sum()
+        assert abs((dv * v).sum() + (dS0 * S0).sum() - L) < 1e-12 * (np.abs(dO * o).sum()
+                                                                       + np.abs(dS_T * S).sum())
+
+
+def pin_bwd_beta_zero(orc):
+    """[FIG5] with beta = 0 the state is Diag(G_t) S0: closed forms of every gradient, the
+    strength's taken through the write and erase terms it switches on
+    (d S_s / d beta_t = Diag(g(s,t)) k_t (v_t - p_t)^T, p_t = S0^T Diag(G_t) k_t)."""
+    rng = np.random.default_rng(72)
+    T, dk, dv = 9, 4, 3
+    q, k, v = rng.standard_normal((T, dk)), _unit(rng, T, dk), rng.standard_normal((T, dv))
+    alpha = rng.uniform(-1, 1, (T, dk))
+    S0, dO, dS_T = (rng.standard_normal(s) for s in ((dk, dv), (T, dv), (dk, dv)))
+    r = lambda x, *s: x.reshape(*s)
+    dq, dk_, dv_, da, db, dS0 = orc.ckda_bwd(r(q, 1, T, 1, dk), r(k, 1, T, 1, dk), r(v, 1, T, 1, dv),
+                                             r(alpha, 1, T, 1, dk), np.zeros((1, T, 1)),
+                                             r(S0, 1, 1, dk, dv), dO=r(dO, 1, T, 1, dv),
+                                             dS_T=r(dS_T, 1, 1, dk, dv), signed_gate=2, threads=1)
+    dq, dk_, dv_, da, db, dS0 = (x.reshape(-1, x.shape[-1]) if x.ndim == 4 else x
+                                 for x in (dq, dk_, dv_, da, db, dS0))
+    db = db.ravel()
+    dS0 = dS0.reshape(dk, dv)
+
+    def g(s, t):                       # prod_{r=t+1..s} alpha_r (1 when s == t)
+        out = np.ones(dk)
+        for x in range(t + 1, s + 1):
+            out = out * alpha[x]
+        return out
+
+    def g_skip(s, t):                  # prod_{r<=s, r != t} alpha_r
+        out = np.ones(dk)
+        for x in range(s + 1):
+            if x != t:
+                out = out * alpha[x]
+        return out
+
+    G = [g(t, -1) for t in range(T)]
+    assert np.abs(dk_).max() == 0.0 and np.abs(dv_).max() == 0.0
+    for t in range(T):
+        assert _rel(dq[t], (G[t][:, None] * S0) @ dO[t]) < 1e-13
+    want = sum(np.outer(G[t] * q[t], dO[t]) for t in range(T)) + G[T - 1][:, None] * dS_T
+    assert _rel(dS0, want) < 1e-13
+    for t in range(T):
+        want_a = sum(g_skip(s, t) * q[s] * (S0 @ dO[s]) for s in range(t, T))
+        want_a = want_a + g_skip(T - 1, t) * (S0 * dS_T).sum(axis=1)
+        assert _rel(da[t], want_a) < 1e-12
+        dS_t = sum(np.outer(g(s, t) * q[s], dO[s]) for s in range(t, T)) + g(T - 1, t)[:, None] * dS_T
+        p_t = S0.T @ (G[t] * k[t])
+        assert abs(db[t] - (dS_t.T @ k[t]) @ (v[t] - p_t)) < 1e-12 * (1 + abs(db[t]))
+
+
+def pin_bwd_linear_attention(orc):
+    """[FIG5] [LA] alpha = 1, beta = 1, orthonormal keys, S0 = 0 (linear attention): the
+    transitions are commuting projectors, so dv_j = sum_{t>=j} (k_j . q_t) dO_t + dS_T^T k_j,
+    dq_t = sum_{j<=t} k_j (v_j . dO_t), dS0 = sum_t P_t q_t dO_t^T + P_T dS_T with
+    P_t = I - sum_{j<=t} k_j k_j^T, dbeta_t = sum_{s>=t} (q_s . k_t)(v_t . dO_s) + k_t^T dS_T v_t,
+    and dalpha_t,i = sum_{s>=t} (M_ts q_s)_i (S_{t-1} dO_s)_i + sum_j (M_tT dS_T)_ij (S_{t-1})_ij
+    with M_ts = I - sum_{r=t..s} k_r k_r^T."""
+    rng = np.random.default_rng(73)
+    dk, dv, T = 8, 5, 7
+    Qm, _ = np.linalg.qr(rng.standard_normal((dk, dk)))
+    k = Qm.T[:T]
+    q, v, dO = rng.standard_normal((T, dk)), rng.standard_normal((T, dv)), rng.standard_normal((T, dv))
+    dS_T = rng.standard_normal((dk, dv))
+    r = lambda x, *s: x.reshape(*s)
+    dq, _, dv_, da, db, dS0 = orc.ckda_bwd(r(q, 1, T, 1, dk), r(k, 1, T, 1, dk), r(v, 1, T, 1, dv),
+                                           np.ones((1, T, 1, dk)), np.ones((1, T, 1)), None,
+                                           dO=r(dO, 1, T, 1, dv), dS_T=r(dS_T, 1, 1, dk, dv),
+                                           signed_gate=2, threads=1)
+    dq, dv_, da = dq.reshape(T, dk), dv_.reshape(T, dv), da.reshape(T, dk)
+    db, dS0 = db.ravel(), dS0.reshape(dk, dv)
+    I = np.eye(dk)
+    M = lambda t, s: I - sum((np.outer(k[x], k[x]) for x in range(t, s + 1)), np.zeros((dk, dk)))
+    S_prev = lambda t: sum((np.outer(k[j], v[j]) for j in range(t)), np.zeros((dk, dv)))
+    for j in range(T):
+        want = sum((k[j] @ q[t]) * dO[t] for t in range(j, T)) + dS_T.T @ k[j]
+        assert _rel(dv_[j], want) < 1e-12
+        assert _rel(dq[j], sum(k[x] * (v[x] @ dO[j]) for x in range(j + 1))) < 1e-12
+        want_b = sum((q[s] @ k[j]) * (v[j] @ dO[s]) for s in range(j, T)) + k[j] @ dS_T @ v[j]
+        assert abs(db[j] - want_b) < 1e-12 * (1 + abs(want_b))
+        want_a = sum((M(j, s) @ q[s]) * (S_prev(j) @ dO[s]) for s in range(j, T))
+        want_a = want_a + ((M(j, T - 1) @ dS_T) * S_prev(j)).sum(axis=1)
+        assert np.allclose(da[j], want_a, rtol=1e-12, atol=1e-12)
+    want = sum(M(0, t) @ np.outer(q[t], dO[t]) for t in range(T)) + M(0, T - 1) @ dS_T
+    assert _rel(dS0, want) < 1e-12
 
 
 ALL_PINS = [v for n, v in sorted(globals().items()) if n.startswith("pin_")]

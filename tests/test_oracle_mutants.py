@@ -25,6 +25,24 @@ MUTANTS = [
     ("initial_state_ignored", "if (J->S0)\n        memcpy", "if (0)\n        memcpy"),
     ("varlen_start_shifted", "t0 = J->cu[n];", "t0 = J->cu[n] + (n > 0);"),
     ("readout_uses_k", "acc += q[i] * S[(size_t)i * dv + j];\n            o[j]", "acc += k[i] * S[(size_t)i * dv + j];\n            o[j]"),
+    # backward
+    ("bwd_readout_grad_uses_k", "dS[(size_t)i * dv + j] += q[i] * dO[j];",
+     "dS[(size_t)i * dv + j] += k[i] * dO[j];"),
+    ("bwd_dq_from_previous_state", "acc += S_cur[(size_t)i * dv + j] * dO[j];",
+     "acc += S_prev[(size_t)i * dv + j] * dO[j];"),
+    ("bwd_erase_adjoint_dropped", "dS[(size_t)i * dv + j] += k[i] * (-beta * du[j]);",
+     "dS[(size_t)i * dv + j] += 0.0 * k[i] * (-beta * du[j]);"),
+    ("bwd_dp_sign_flipped", "acc += St[(size_t)i * dv + j] * (-beta * du[j]);",
+     "acc += St[(size_t)i * dv + j] * (beta * du[j]);"),
+    ("bwd_dbeta_without_erase", "dbeta += acc * (v[j] - p[j]);", "dbeta += acc * v[j];"),
+    ("bwd_dalpha_from_new_state", "acc += dS[(size_t)i * dv + j] * S_prev[(size_t)i * dv + j];",
+     "acc += dS[(size_t)i * dv + j] * S_cur[(size_t)i * dv + j];"),
+    ("bwd_state_grad_ungated", "for (int j = 0; j < dv; ++j) dS[(size_t)i * dv + j] *= alpha[i];",
+     "for (int j = 0; j < dv; ++j) dS[(size_t)i * dv + j] *= 1.0;"),
+    ("bwd_ckda_derivative_halved", "(af == 1 ? 2.0 * sigmoid_deriv(a[i]) : 1.0)",
+     "(af == 1 ? sigmoid_deriv(a[i]) : 1.0)"),
+    ("bwd_checkpoint_off_by_one", "memcpy(states, ckpt + (size_t)sg * dd",
+     "memcpy(states, ckpt + (size_t)(sg > 0 ? sg - 1 : 0) * dd"),
 ]
 
 
