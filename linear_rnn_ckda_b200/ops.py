@@ -82,6 +82,75 @@ def _ptr(t: Optional[torch.Tensor]):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _need(cond: bool, msg: str):
+    if not cond:
+        raise ValueError(msg)
+
+
+def _same_device(ref: torch.Tensor, **tensors):
+    for name, t in tensors.items():
+        if t is not None and t.device != ref.device:
+            raise ValueError(f"{name} is on {t.device}, q on {ref.device}")
+
+
+def check_prefill_args(q, k, v, a, b, S0=None, cu_seqlens=None, o=None, S_T=None,
+                       o_dtype=None):
+    """Shapes, dtypes and devices that ``ckda_chunk_fwd`` relies on but cannot see (it receives
+    bare pointers, so a short or mistyped buffer would be read or written past its end).
+    Raises ValueError; returns (N, dv).  The offsets inside ``cu_seqlens`` are checked on the
+    device (the workspace status word), not here."""
+    _need(q.dim() == 4, f"q must be [B,T,H,dk], got {tuple(q.shape)}")
+    _need(q.dtype in _DT, f"q must be float32 or bfloat16, got {q.dtype}")
+    B, T, H, dk = q.shape
+    for name, t in (("k", k), ("a", a)):
+        _need(t.shape == q.shape and t.dtype == q.dtype,
+              f"{name} must match q ({tuple(q.shape)}, {q.dtype}), got {tuple(t.shape)}, {t.dtype}")
+    _need(v.dim() == 4 and v.shape[:3] == q.shape[:3] and v.dtype == q.dtype,
+          f"v must be [B,T,H,dv] in q's dtype, got {tuple(v.shape)}, {v.dtype}")
+    dv = v.shape[-1]
+    _need(b.shape == (B, T, H) and b.dtype == torch.float32,
+          f"b must be [B,T,H] float32, got {tuple(b.shape)}, {b.dtype}")
+    N = B
+    if cu_seqlens is not None:
+        _need(cu_seqlens.dim() == 1 and cu_seqlens.numel() >= 1 and cu_seqlens.dtype == torch.int32,
+              "cu_seqlens must be a 1-D int32 tensor of N+1 offsets")
+        _need(B == 1, "packed sequences (cu_seqlens) need B == 1")
+        N = cu_seqlens.numel() - 1
+    for name, t in (("S0", S0), ("S_T", S_T)):
+        _need(t is None or (t.shape == (N, H, dk, dv) and t.dtype == torch.float32),
+              f"{name} must be [N,H,dk,dv] = {(N, H, dk, dv)} float32")
+    od = q.dtype if o_dtype is None else o_dtype
+    _need(od in _DT, f"o_dtype must be float32 or bfloat16, got {od}")
+    _need(o is None or (o.shape == (B, T, H, dv) and o.dtype == od),
+          f"o must be [B,T,H,dv] = {(B, T, H, dv)} in {od}")
+    _same_device(q, k=k, v=v, a=a, b=b, S0=S0, cu_seqlens=cu_seqlens, o=o, S_T=S_T)
+    return N, dv
+
+
+def check_decode_args(q, k, v, a, b, S, o=None, o_dtype=None):
+    """The same checks for ``ckda_decode_step``: q, k, a [B,H,dk]; v [B,H,dv] in q's dtype;
+    b [B,H] float32; S [B,H,dk,dv] float32; o [B,H,dv] in the output dtype."""
+    _need(q.dim() == 3, f"q must be [B,H,dk], got {tuple(q.shape)}")
+    _need(q.dtype in _DT, f"q must be float32 or bfloat16, got {q.dtype}")
+    B, H, dk = q.shape
+    for name, t in (("k", k), ("a", a)):
+        _need(t.shape == q.shape and t.dtype == q.dtype,
+              f"{name} must match q ({tuple(q.shape)}, {q.dtype}), got {tuple(t.shape)}, {t.dtype}")
+    _need(v.dim() == 3 and v.shape[:2] == q.shape[:2] and v.dtype == q.dtype,
+          f"v must be [B,H,dv] in q's dtype, got {tuple(v.shape)}, {v.dtype}")
+    dv = v.shape[-1]
+    _need(b.shape == (B, H) and b.dtype == torch.float32,
+          f"b must be [B,H] float32, got {tuple(b.shape)}, {b.dtype}")
+    _need(S.shape == (B, H, dk, dv) and S.dtype == torch.float32,
+          f"S must be [B,H,dk,dv] = {(B, H, dk, dv)} float32")
+    od = q.dtype if o_dtype is None else o_dtype
+    _need(od in _DT, f"o_dtype must be float32 or bfloat16, got {od}")
+    _need(o is None or (o.shape == (B, H, dv) and o.dtype == od),
+          f"o must be [B,H,dv] = {(B, H, dv)} in {od}")
+    _same_device(q, k=k, v=v, a=a, b=b, S=S, o=o)
+    return dv
+
+
 def _stream(device) -> ctypes.c_void_p:
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
@@ -104,11 +173,10 @@ def chunk_fwd(q, k, v, a, b, S0=None, cu_seqlens=None, chunk: int = 64, signed_g
     S0: [N,H,dk,dv] fp32 or None; cu_seqlens: int32 CUDA tensor [N+1] or None.
     """
     lib = load()
+    N, dv = check_prefill_args(q, k, v, a, b, S0, cu_seqlens, o, S_T, o_dtype)
     B, T, H, dk = q.shape
-    dv = v.shape[-1]
     io = _DT[q.dtype]
     od = io if o_dtype is None else _DT[o_dtype]
-    N = B if cu_seqlens is None else cu_seqlens.numel() - 1
     dev = q.device
     if want_o and o is None:
         o = torch.empty((B, T, H, dv), dtype=_TORCH_DT[od], device=dev)
@@ -116,11 +184,12 @@ def chunk_fwd(q, k, v, a, b, S0=None, cu_seqlens=None, chunk: int = 64, signed_g
         S_T = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
     if workspace is None:
         workspace = new_workspace(B, T, H, dk, dv, chunk, N, dev)
+    _need(workspace.device == dev, f"workspace is on {workspace.device}, q on {dev}")
     rc = lib.ckda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(S0),
                             _ptr(cu_seqlens), N if cu_seqlens is not None else 0, B, T, H, dk, dv,
                             chunk, signed_gate, io, od, _ptr(o if want_o else None),
                             _ptr(S_T if want_state else None), _ptr(workspace),
-                            workspace.numel(), _stream(dev))
+                            workspace.numel() * workspace.element_size(), _stream(dev))
     if rc != 0:
         raise CkdaError("ckda_chunk_fwd", rc)
     return (o if want_o else None), (S_T if want_state else None)
@@ -129,8 +198,8 @@ def chunk_fwd(q, k, v, a, b, S0=None, cu_seqlens=None, chunk: int = 64, signed_g
 def decode_step(q, k, v, a, b, S, signed_gate: int = 1, o_dtype=None, o=None, want_o=True):
     """One decode step; S [B,H,dk,dv] fp32 is updated in place.  Returns o [B,H,dv]."""
     lib = load()
+    dv = check_decode_args(q, k, v, a, b, S, o, o_dtype)
     B, H, dk = q.shape
-    dv = v.shape[-1]
     io = _DT[q.dtype]
     od = io if o_dtype is None else _DT[o_dtype]
     if want_o and o is None:

@@ -121,3 +121,78 @@ def test_binding_has_no_cpu_fallback(lib):
     with pytest.raises(ValueError):
         ops.decode_step(x[:, 0], x[:, 0], x[:, 0], x[:, 0], torch.zeros(1, 1),
                         torch.zeros(1, 1, 16, 16))
+
+
+# ---------------------------------------------------------------- binding argument checks
+# The C ABI receives bare pointers, so the binding checks what it cannot: that every tensor
+# has the shape and dtype its pointer is read or written as.
+
+from linear_rnn_ckda_b200 import synth  # noqa: E402
+
+
+@pytest.mark.parametrize("w", [synth.TINY_CKDA_FP32, synth.KDA_STD.with_(B=2, T=70, H=3),
+                               synth.CKDA_SPREAD.with_(B=2, T=70, H=3, o_dtype="f32"),
+                               synth.CKDA_SPREAD.with_(B=1, H=2, seq_lens=(0, 1, 65), T=66)],
+                         ids=["tiny", "kda", "ckda_s0", "varlen"])
+def test_binding_accepts_the_workloads(w):
+    d = synth.make_prefill(w, seed=0)
+    od = torch.float32 if w.o_dtype == "f32" else torch.bfloat16
+    N, dv = ops.check_prefill_args(d["q"], d["k"], d["v"], d["a"], d["b"], d["S0"],
+                                   d["cu_seqlens"], o_dtype=od)
+    assert (N, dv) == (w.n_seqs, w.dv)
+    B, T, H = d["q"].shape[:3]
+    o = torch.empty(B, T, H, dv, dtype=od)
+    S_T = torch.empty(N, H, w.dk, dv)
+    ops.check_prefill_args(d["q"], d["k"], d["v"], d["a"], d["b"], d["S0"], d["cu_seqlens"],
+                           o=o, S_T=S_T, o_dtype=od)
+    dec = synth.make_decode(synth.DECODE.with_(B=2, H=3), seed=0, steps=2)
+    assert ops.check_decode_args(dec["q"][0], dec["k"][0], dec["v"][0], dec["a"][0],
+                                 dec["b"][0], dec["S"], o_dtype=torch.float32) == 128
+
+
+def _prefill_bad(**over):
+    w = synth.KDA_STD.with_(B=2, T=70, H=3, s0=True)
+    d = synth.make_prefill(w, seed=0)
+    args = dict(q=d["q"], k=d["k"], v=d["v"], a=d["a"], b=d["b"], S0=d["S0"], cu_seqlens=None)
+    args.update(over)
+    return args
+
+
+@pytest.mark.parametrize("name,over", [
+    ("k_shorter", lambda d: dict(k=d["k"][:, :60])),
+    ("a_other_dtype", lambda d: dict(a=d["a"].float())),
+    ("v_other_dtype", lambda d: dict(v=d["v"].float())),
+    ("v_other_heads", lambda d: dict(v=d["v"][:, :, :2])),
+    ("b_bf16", lambda d: dict(b=d["b"].to(torch.bfloat16))),
+    ("b_per_channel", lambda d: dict(b=d["a"].float())),
+    ("q_3d", lambda d: dict(q=d["q"][0])),
+    ("S0_wrong_heads", lambda d: dict(S0=d["S0"][:, :2])),
+    ("S0_bf16", lambda d: dict(S0=d["S0"].to(torch.bfloat16))),
+    ("seqlens_int64", lambda d: dict(cu_seqlens=torch.tensor([0, 70]))),
+    ("seqlens_with_batch", lambda d: dict(cu_seqlens=torch.tensor([0, 70], dtype=torch.int32))),
+    ("o_wrong_dtype", lambda d: dict(o=torch.empty(2, 70, 3, 128))),
+    ("o_short", lambda d: dict(o=torch.empty(2, 69, 3, 128, dtype=torch.bfloat16))),
+    ("S_T_wrong", lambda d: dict(S_T=torch.empty(2, 3, 128, 64))),
+])
+def test_binding_rejects_mismatched_buffers(name, over):
+    base = _prefill_bad()
+    args = _prefill_bad(**over(base))
+    with pytest.raises(ValueError):
+        ops.check_prefill_args(**args)
+
+
+@pytest.mark.parametrize("name,over", [
+    ("k_shorter", lambda d: dict(k=d["k"][:1])),
+    ("b_bf16", lambda d: dict(b=d["b"].to(torch.bfloat16))),
+    ("S_wrong_dv", lambda d: dict(S=d["S"][..., :64])),
+    ("S_bf16", lambda d: dict(S=d["S"].to(torch.bfloat16))),
+    ("v_other_dtype", lambda d: dict(v=d["v"].float())),
+    ("o_wrong_shape", lambda d: dict(o=torch.empty(2, 3, 64))),
+])
+def test_decode_binding_rejects_mismatched_buffers(name, over):
+    dec = synth.make_decode(synth.DECODE.with_(B=2, H=3), seed=0, steps=1)
+    d = {k: (v[0] if k != "S" else v) for k, v in dec.items()}
+    args = dict(q=d["q"], k=d["k"], v=d["v"], a=d["a"], b=d["b"], S=d["S"])
+    args.update(over(d))
+    with pytest.raises(ValueError):
+        ops.check_decode_args(**args)
