@@ -18,6 +18,11 @@ file states them in numpy and checks
   * the integer tf32 rounding ((bits + 0x1000) & ~0x1FFF) against the
     definition of round-to-nearest, ties away from zero, onto the tf32 grid.
 
+Both ways of applying (I + A)^{-1} are checked: the fused kernel's
+block-diagonal product plus three correction rounds, and the full T assembled
+from the same blocks and applied in one product (the form a state pass that
+reads T computed elsewhere would use).
+
 The tensor core's own accumulation order is not specified; the emulation
 forms each product exactly and rounds it to fp32 once, which is the most
 favourable accumulation, so the checks on the plan keep a factor of two of
@@ -173,9 +178,29 @@ def _block_solve(A, plan: _Plan):
     return X, M
 
 
-def chunk_kernel_form(q, k, v, a, b, S0, form: int, plan: _Plan):
+def _full_T(Xi, M, be, dt):
+    """(I + A)^{-1} Diag(beta) assembled from the block solve: diagonal blocks X_i Diag(beta_i),
+    T_ij = -sum_{k=j}^{i-1} M_ik T_kj below them (three dependency levels)."""
+    Tf = np.zeros((C, C), dtype=dt)
+    for i in range(C // NB):
+        sl = slice(i * NB, (i + 1) * NB)
+        Tf[sl, sl] = Xi[i] * be[sl][None, :]
+    for lev in (1, 2, 3):
+        for j in range(C // NB - lev):
+            i = j + lev
+            acc = np.zeros((NB, NB))
+            for kk in range(j, i):
+                acc += M[(i, kk)].astype(np.float64) @ Tf[kk * NB:(kk + 1) * NB,
+                                                           j * NB:(j + 1) * NB].astype(np.float64)
+            Tf[i * NB:(i + 1) * NB, j * NB:(j + 1) * NB] = (-acc).astype(dt)
+    return Tf
+
+
+def chunk_kernel_form(q, k, v, a, b, S0, form: int, plan: _Plan, solve: str = "rounds"):
     """One sequence and head through the kernel's steps.  q, k, a [T,d]; v [T,dv]; b [T]
-    (logits); S0 [d,dv].  Returns (o [T,dv], S_T [d,dv])."""
+    (logits); S0 [d,dv].  Returns (o [T,dv], S_T [d,dv]).  ``solve`` = "rounds": U from the
+    block-diagonal part of T and three correction rounds (the fused kernel); "full": U from
+    the full T in one product (a state pass that reads T precomputed elsewhere)."""
     dt = plan.dt
     T, dk = q.shape
     if plan.tf32:
@@ -218,16 +243,21 @@ def chunk_kernel_form(q, k, v, a, b, S0, form: int, plan: _Plan):
         lo = plan.tmem((Vp - hi).astype(dt))
         # (c) U = Tb V' with Tb = blockdiag(X_i) Diag(beta); rounds U_i -= M_ij U_j
         Xi, M = _block_solve(A, plan)
-        Tb = np.zeros((C, C), dtype=dt)
-        for i in range(C // NB):
-            sl = slice(i * NB, (i + 1) * NB)
-            Tb[sl, sl] = Xi[i] * be[sl][None, :]
-        Tb = plan.smem(Tb)
-        U = plan.mma(Tb, lo, plan.mma(Tb, hi))
-        for j in range(C // NB - 1):
-            Uj = plan.tmem(U[j * NB:(j + 1) * NB])
-            for i in range(j + 1, C // NB):
-                U[i * NB:(i + 1) * NB] = plan.mma(-plan.smem(M[(i, j)]), Uj, U[i * NB:(i + 1) * NB])
+        if solve == "full":
+            Tt = plan.smem(_full_T(Xi, M, be, dt))
+            U = plan.mma(Tt, lo, plan.mma(Tt, hi))
+        else:
+            Tb = np.zeros((C, C), dtype=dt)
+            for i in range(C // NB):
+                sl = slice(i * NB, (i + 1) * NB)
+                Tb[sl, sl] = Xi[i] * be[sl][None, :]
+            Tb = plan.smem(Tb)
+            U = plan.mma(Tb, lo, plan.mma(Tb, hi))
+            for j in range(C // NB - 1):
+                Uj = plan.tmem(U[j * NB:(j + 1) * NB])
+                for i in range(j + 1, C // NB):
+                    U[i * NB:(i + 1) * NB] = plan.mma(-plan.smem(M[(i, j)]), Uj,
+                                                      U[i * NB:(i + 1) * NB])
         # (d) O += P U;  S += Kc^T U, then the columns scaled by G_{C-1}
         Ut = plan.tmem(U)
         o[t0:t0 + n] = plan.mma(P, Ut, Oc)[:n]
@@ -247,16 +277,17 @@ def _units(inp):
             yield n, h, q[n, :, h], k[n, :, h], v[n, :, h], a[n, :, h], b[n, :, h], s0
 
 
+@pytest.mark.parametrize("solve", ["rounds", "full"])
 @pytest.mark.parametrize("form", [0, 1], ids=["kda", "ckda"])
 @pytest.mark.parametrize("T", [64, 3 * 64 + 37])
-def test_kernel_form_is_exact(form, T):
+def test_kernel_form_is_exact(form, T, solve):
     """The regrouped, block-solved chunk form equals the recurrence (fp64, no rounding)."""
     w = synth.CKDA_SPREAD.with_(B=1, T=T, H=2, dk=32, dv=24, signed_gate=form,
                                 io_dtype="f32", o_dtype="f32")
     inp = synth.make_prefill(w, seed=21)
     ro, rS = oracle_prefill(inp, form)
     for n, h, q, k, v, a, b, s0 in _units(inp):
-        o, S = chunk_kernel_form(q, k, v, a, b, s0, form, _Plan(tf32=False))
+        o, S = chunk_kernel_form(q, k, v, a, b, s0, form, _Plan(tf32=False), solve)
         assert rel(o, unit_rows(ro, inp, n, h)) < 1e-11
         assert rel(S, rS[n, h]) < 1e-11
 
@@ -277,10 +308,11 @@ def test_block_solve_inverts_unit_lower_triangle():
     assert np.allclose(Tinv @ (np.eye(C) + A), np.eye(C), atol=1e-10)
 
 
+@pytest.mark.parametrize("solve", ["rounds", "full"])
 @pytest.mark.parametrize("base,form", [(synth.KDA_STD, 0), (synth.CKDA_SPREAD, 1),
                                        (synth.KDA_STD.with_(signed_gate=1, gate="tiny"), 1)],
                          ids=["kda_std", "ckda_spread", "ckda_tiny"])
-def test_tf32_operand_plan_within_tolerance(base, form):
+def test_tf32_operand_plan_within_tolerance(base, form, solve):
     """bf16 inputs at the full head size (d = 128, chunk 64), several chunks and a ragged
     tail: the kernel's operand plan stays at half the bf16 tolerance or below.  In the
     "tiny" CKDA case (gate logits N(0, 1.5)) the first two chunks of each head decay below
@@ -290,7 +322,7 @@ def test_tf32_operand_plan_within_tolerance(base, form):
     ro, rS = oracle_prefill(inp, form)
     os_, ss_, ro_, rs_ = [], [], [], []
     for n, h, q, k, v, a, b, s0 in _units(inp):
-        o, S = chunk_kernel_form(q, k, v, a, b, s0, form, _Plan(tf32=True))
+        o, S = chunk_kernel_form(q, k, v, a, b, s0, form, _Plan(tf32=True), solve)
         os_.append(o)
         ss_.append(S)
         ro_.append(unit_rows(ro, inp, n, h))
