@@ -17,7 +17,7 @@
 //   (1) [A;P]   = [Kr;Qr] Kc^T          M=128 (64 Kr rows + 64 Qr rows), N=64, K=128
 //   (a) [X^T|O^T] = S^T [Kr;Qr]^T       N=128 (X = Kr S, and O's first term), K=128
 //   (b) V' = V - X in fp32 (threads), kept in TMEM as tf32 hi + lo parts
-//   (c) U^T     = V'^T Tm^T              A = V'^T in TMEM (hi and lo), K=64, then three rounds
+//   (c) U^T     = V'^T Tm^T              A = V'^T in TMEM (hi and lo), K=64, then three corrections
 //   (d) [O^T|S^T] += U^T [P;Kc^T]^T     N=192, then S^T columns scaled by G_63 (threads)
 // (1) and (a) need only the chunk's inputs and S, so they are issued together
 // when the chunk starts, and (b) overlaps the solve.  All MMAs are kind::tf32
@@ -75,9 +75,9 @@ constexpr uint32_t COL_U = 0, COL_VT0 = 64, COL_AP = 128, COL_LO = 128, COL_X = 
                    COL_S = 320, COL_VT1 = 448;
 
 constexpr uint32_t IDESC_N64 = idesc_tf32(128, 64, false, false);         // (1), (c), O += U P^T
-constexpr uint32_t IDESC_N48_NEG = idesc_tf32(128, 48, false, false, true);  // (c) round 2
-constexpr uint32_t IDESC_N32_NEG = idesc_tf32(128, 32, false, false, true);  // (c) round 3
-constexpr uint32_t IDESC_N16_NEG = idesc_tf32(128, 16, false, false, true);  // (c) round 4
+constexpr uint32_t IDESC_N48_NEG = idesc_tf32(128, 48, false, false, true);  // (c) correction 1
+constexpr uint32_t IDESC_N32_NEG = idesc_tf32(128, 32, false, false, true);  // (c) correction 2
+constexpr uint32_t IDESC_N16_NEG = idesc_tf32(128, 16, false, false, true);  // (c) correction 3
 constexpr uint32_t IDESC_N128 = idesc_tf32(128, 128, false, false);       // (a)
 constexpr uint32_t IDESC_N192 = idesc_tf32(128, 192, false, false);       // (d)
 
@@ -138,7 +138,7 @@ constexpr int kAS = 68;
 // takes one of them (lane = column, kept in registers, rows finished in order, each row of
 // D_i read as a broadcast; all fp32), two per warp over warps w0..w0+4.  Written as tf32:
 // Tb into the T tile (its zero blocks by solve_T_zeros), [M10; M20; M30] and [M21; M31; M32]
-// into two 48-row tiles (K = 16 of each 32-wide row used).  The MMA rounds then apply the
+// into two 48-row tiles (K = 16 of each 32-wide row used).  MMA corrections then apply the
 // M_ij as each U_j becomes final.
 __device__ __forceinline__ void solve_T(const float *A, uint8_t *sT, uint8_t *sR2, uint8_t *sR34,
                                         const float *beta, int task2, int lane) {
@@ -222,7 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   float *sBeta = reinterpret_cast<float *>(sm + OFF_MISC);     // [64]
   float *sGC = sBeta + 64;                                       // [2][128] G_63, double-buffered
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_MISC + 1280);
-  // completion (TMA or tcgen05.commit): staging, (1), (a), rounds 1/2 of (c), (d), all MMAs
+  // completion (TMA or tcgen05.commit): staging, (1), (a), the steps of (c), (d), all MMAs
   uint64_t *bar_tma = bars, *bar_mma1 = bars + 1, *bar_a = bars + 2, *bar_r = bars + 3,
            *bar_d = bars + 4, *bar_fin = bars + 5;
   // compute warps -> issuer (one arrival per compute warp): a chunk's tiles are ready and
@@ -232,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // issuer -> compute warps: a token-by-token announcement has been consumed (so the next
   // announcement cannot be mistaken for it)
   uint64_t *bar_ack = bars + 10;
-  // the last round of (c) is done: the R tiles in Kc's area have been read
+  // the last correction of (c) is done: the R tiles in Kc's area have been read
   uint64_t *bar_r4 = bars + 11;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_MISC + 1392);
   volatile int *sAbort = reinterpret_cast<volatile int *>(sm + OFF_MISC + 1396);
@@ -336,7 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ts(tmem + COL_X, tmem + COL_S + 8 * s, dadd(dKQ, off), IDESC_N128, s > 0);
         }
         mma_commit(bar_a);
-        // (c) round 1: U^T = V'^T Tb^T, hi and lo parts of V'
+        // (c) first step: U^T = V'^T Tb^T, hi and lo parts of V'
         if (!(ok = mbar_wait_or_abort(rdy3, ph3, kWaitNs, sAbort))) break;
         ph3 ^= 1;
         const uint32_t vt_cur = (((cs - t0) / kC) & 1) ? COL_VT1 : COL_VT0;
@@ -350,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ts(tmem + COL_U, tmem + COL_LO + 8 * s, dadd(dT, (s >> 2) * 8192 + (s & 3) * 32),
                  IDESC_N64, 1);
         mma_commit(bar_r);
-        // rounds 2, 3, 4: U_i -= M_ij U_j for the blocks j = 0, 1, 2 as each becomes final
+        // corrections: U_i -= M_ij U_j for the blocks j = 0, 1, 2 as each becomes final
         // (U_j^T read from TMEM, K = 16)
         if (!(ok = mbar_wait_or_abort(bar_r, phr, kWaitNs, sAbort))) break;
         phr ^= 1;

@@ -4,7 +4,7 @@ checked against the sequential fp64 oracle.
 Test infrastructure (numpy only; shares no code with the CUDA path).  The
 tensor-core prefill does not follow the textbook WY form step by step: it
 regroups U = T (V - (K*G) S), inverts (I + A) in 16-row blocks with the
-off-diagonal blocks applied as three correction rounds, keeps K*G^{-1} with the
+off-diagonal blocks applied as three corrections, keeps K*G^{-1} with the
 final G folded in afterwards, and rounds every tensor-core operand to tf32.
 Each of those choices is an algebraic identity or a precision decision; this
 file states them in numpy and checks
@@ -19,7 +19,7 @@ file states them in numpy and checks
     definition of round-to-nearest, ties away from zero, onto the tf32 grid.
 
 Both ways of applying (I + A)^{-1} are checked: the fused kernel's
-block-diagonal product plus three correction rounds, and the full T assembled
+block-diagonal product plus three corrections, and the full T assembled
 from the same blocks and applied in one product (the form a state pass that
 reads T computed elsewhere would use).
 
@@ -196,10 +196,10 @@ def _full_T(Xi, M, be, dt):
     return Tf
 
 
-def chunk_kernel_form(q, k, v, a, b, S0, form: int, plan: _Plan, solve: str = "rounds"):
+def chunk_kernel_form(q, k, v, a, b, S0, form: int, plan: _Plan, solve: str = "corrections"):
     """One sequence and head through the kernel's steps.  q, k, a [T,d]; v [T,dv]; b [T]
-    (logits); S0 [d,dv].  Returns (o [T,dv], S_T [d,dv]).  ``solve`` = "rounds": U from the
-    block-diagonal part of T and three correction rounds (the fused kernel); "full": U from
+    (logits); S0 [d,dv].  Returns (o [T,dv], S_T [d,dv]).  ``solve`` = "corrections": U from the
+    block-diagonal part of T and three corrections (the fused kernel); "full": U from
     the full T in one product (a state pass that reads T precomputed elsewhere)."""
     dt = plan.dt
     T, dk = q.shape
@@ -241,7 +241,7 @@ def chunk_kernel_form(q, k, v, a, b, S0, form: int, plan: _Plan, solve: str = "r
         Vp = (V - X).astype(dt)
         hi = plan.smem(Vp)
         lo = plan.tmem((Vp - hi).astype(dt))
-        # (c) U = Tb V' with Tb = blockdiag(X_i) Diag(beta); rounds U_i -= M_ij U_j
+        # (c) U = Tb V' with Tb = blockdiag(X_i) Diag(beta); corrections U_i -= M_ij U_j
         Xi, M = _block_solve(A, plan)
         if solve == "full":
             Tt = plan.smem(_full_T(Xi, M, be, dt))
@@ -277,7 +277,7 @@ def _units(inp):
             yield n, h, q[n, :, h], k[n, :, h], v[n, :, h], a[n, :, h], b[n, :, h], s0
 
 
-@pytest.mark.parametrize("solve", ["rounds", "full"])
+@pytest.mark.parametrize("solve", ["corrections", "full"])
 @pytest.mark.parametrize("form", [0, 1], ids=["kda", "ckda"])
 @pytest.mark.parametrize("T", [64, 3 * 64 + 37])
 def test_kernel_form_is_exact(form, T, solve):
@@ -308,7 +308,7 @@ def test_block_solve_inverts_unit_lower_triangle():
     assert np.allclose(Tinv @ (np.eye(C) + A), np.eye(C), atol=1e-10)
 
 
-@pytest.mark.parametrize("solve", ["rounds", "full"])
+@pytest.mark.parametrize("solve", ["corrections", "full"])
 @pytest.mark.parametrize("base,form", [(synth.KDA_STD, 0), (synth.CKDA_SPREAD, 1),
                                        (synth.KDA_STD.with_(signed_gate=1, gate="tiny"), 1)],
                          ids=["kda_std", "ckda_spread", "ckda_tiny"])
