@@ -4,6 +4,7 @@
 // status read-back, which says so).
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 
@@ -18,18 +19,20 @@ bool aligned(const void *p, uintptr_t n) {
 }
 bool aligned16(const void *p) { return aligned(p, 16); }
 
-// sm_100 check for the current device, cached per device.
+// sm_100 check for the current device, cached per device (atomics: host threads may call the
+// library concurrently; the cached value is the same whoever writes it).
 int check_device() {
-  static int cached[64];  // 0 unknown, 1 ok, -1 not sm_100
+  static std::atomic<int> cached[64];  // 0 unknown, 1 ok, -1 not sm_100
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return CKDA_ERR_CUDA;
-  if (dev >= 0 && dev < 64 && cached[dev] != 0) return cached[dev] > 0 ? CKDA_OK : CKDA_ERR_DEVICE;
+  const int known = dev >= 0 && dev < 64 ? cached[dev].load(std::memory_order_relaxed) : 0;
+  if (known != 0) return known > 0 ? CKDA_OK : CKDA_ERR_DEVICE;
   int major = 0, minor = 0;
   if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
     return CKDA_ERR_CUDA;
   const bool ok = (major == 10 && minor == 0);
-  if (dev >= 0 && dev < 64) cached[dev] = ok ? 1 : -1;
+  if (dev >= 0 && dev < 64) cached[dev].store(ok ? 1 : -1, std::memory_order_relaxed);
   return ok ? CKDA_OK : CKDA_ERR_DEVICE;
 }
 
