@@ -1,11 +1,16 @@
 """The chunkwise (UT-form) backward, stated independently in numpy
 (``chunkwise_bwd_ref.py``), equals the sequential oracle's backward in fp64: the algebra a
-chunkwise backward kernel computes, checked before any such kernel exists.  CPU only."""
+chunkwise backward kernel computes, checked before any such kernel exists.  With tf32
+operands in every matrix product it stays within the bf16 tolerance provided the gate
+gradient is formed pairwise (see the reference's docstring).  CPU only."""
 import numpy as np
 import pytest
 
 import oracle
 from chunkwise_bwd_ref import chunk_bwd_one
+from helpers import TOL_BF16, f64
+from linear_rnn_ckda_b200 import synth
+from test_chunk_algebra import tf32_nearest
 
 
 def _case(T, dk, dv, seed, zero_ends=False):
@@ -32,13 +37,51 @@ def _oracle(q, k, v, alpha, beta, S0, dO, dST):
     return [x.reshape(-1) for x in out]
 
 
+@pytest.mark.parametrize("gate_grad", ["factorised", "pairwise"])
 @pytest.mark.parametrize("chunk", [1, 2, 16, 64])
 @pytest.mark.parametrize("T,zero_ends", [(150, False), (64, True), (7, False)])
-def test_chunkwise_backward_equals_sequential(chunk, T, zero_ends):
+def test_chunkwise_backward_equals_sequential(chunk, T, zero_ends, gate_grad):
     args = _case(T, 8, 6, seed=T + chunk, zero_ends=zero_ends)
     ref = _oracle(*args)
-    got = chunk_bwd_one(*args, chunk)
+    got = chunk_bwd_one(*args, chunk, gate_grad)
     for name, g, r in zip(("dq", "dk", "dv", "dalpha", "dbeta", "dS0"), got, ref):
         n = np.linalg.norm(r)
         err = np.linalg.norm(g.reshape(-1) - r) / (n if n > 0 else 1.0)
         assert err < 1e-11, (name, err)
+
+
+# ---------------------------------------------------------------- tf32 operand plan
+def _mm_tf32(a, b):
+    """A matrix product with tf32 operands (round to nearest) and an fp32 result."""
+    a32 = tf32_nearest(np.asarray(a, np.float32)).astype(np.float64)
+    b32 = tf32_nearest(np.asarray(b, np.float32)).astype(np.float64)
+    return (a32 @ b32).astype(np.float32).astype(np.float64)
+
+
+@pytest.mark.parametrize("base,form", [(synth.KDA_STD, 0), (synth.CKDA_SPREAD, 1)],
+                         ids=["kda_std", "ckda_spread"])
+def test_tf32_operand_plan(base, form):
+    """bf16 inputs at the full head size (d = 128, chunk 64, a ragged tail) with every matrix
+    product on tf32 operands: with the pairwise gate gradient every gradient stays at half the
+    bf16 tolerance or below.  The factorised gate gradient sums terms that cancel when the
+    chunk's gate products decay (K/G grows as G shrinks), so on the spread workload its
+    error is several times the pairwise one."""
+    w = base.with_(B=1, T=2 * 64 + 45, H=1, signed_gate=form, o_dtype="f32")
+    inp = synth.make_prefill(w, seed=7)
+    q, k, v, a, b = (f64(inp[x])[0, :, 0] for x in "qkvab")
+    alpha, beta = oracle.gates(a, b, form)
+    T, d = q.shape
+    rng = np.random.default_rng(1)
+    S0 = f64(inp["S0"])[0, 0] if inp["S0"] is not None else np.zeros((d, d))
+    dO = rng.standard_normal((T, d))
+    dST = rng.standard_normal((d, d)) * 0.02
+    ref = _oracle(q, k, v, alpha, beta, S0, dO, dST)
+    errs = {}
+    for gate_grad in ("pairwise", "factorised"):
+        got = chunk_bwd_one(q, k, v, alpha, beta, S0, dO, dST, 64, gate_grad, mm=_mm_tf32)
+        errs[gate_grad] = [np.linalg.norm(g.reshape(-1) - r) / np.linalg.norm(r)
+                           for g, r in zip(got, ref)]
+    assert max(errs["pairwise"]) < TOL_BF16 / 2, errs["pairwise"]
+    if form == 1:
+        assert errs["factorised"][3] > 5 * errs["pairwise"][3], (errs["factorised"][3],
+                                                                 errs["pairwise"][3])
