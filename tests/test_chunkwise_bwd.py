@@ -85,3 +85,26 @@ def test_tf32_operand_plan(base, form):
     if form == 1:
         assert errs["factorised"][3] > 5 * errs["pairwise"][3], (errs["factorised"][3],
                                                                  errs["pairwise"][3])
+
+
+def test_state_gradient_recurrence():
+    """The backward's only sequential dependency, written with the forward's chunk tiles:
+    dS_prev = dZ - Kr^T T^T (Kc dZ) + (Qr^T dO - Kr^T T^T P^T dO), dZ = Diag(g) dS'; equal
+    to the state gradient of the step-by-step reverse (chunkwise_bwd_ref's order)."""
+    rng = np.random.default_rng(2)
+    n, dk, dv = 16, 6, 5
+    Q, K = rng.standard_normal((n, dk)), rng.standard_normal((n, dk))
+    alpha = rng.uniform(0.4, 1, (n, dk)) * rng.choice([-1.0, 1.0], (n, dk))
+    beta = rng.uniform(0, 2, n)
+    dO, dS_out = rng.standard_normal((n, dv)), rng.standard_normal((dk, dv))
+    G = np.cumprod(alpha, axis=0)
+    Kr, Qr, Kc = K * G, Q * G, K / G
+    A = np.tril(beta[:, None] * (Kr @ Kc.T), -1)
+    Tm = np.linalg.inv(np.eye(n) + A) @ np.diag(beta)
+    P = np.tril(Qr @ Kc.T)
+    dZ = G[-1][:, None] * dS_out
+    # step-by-step reverse: dU from the state write and the output, dV' = T^T dU
+    dVp = Tm.T @ (Kc @ dZ + P.T @ dO)
+    step = dZ + Qr.T @ dO - Kr.T @ dVp
+    recurrence = dZ - Kr.T @ (Tm.T @ (Kc @ dZ)) + (Qr.T @ dO - Kr.T @ (Tm.T @ (P.T @ dO)))
+    assert np.allclose(recurrence, step, rtol=1e-12, atol=1e-12 * np.abs(step).max())
