@@ -85,6 +85,8 @@ extern "C" {
  *            Without it N = B and every batch row is one sequence of T tokens.
  *            Offsets are checked on the device: a bad sequence is skipped
  *            and CKDA_ERR_SEQLENS is recorded in the workspace status word.
+ *            B * T must not exceed 2^31 - 1 (token rows are addressed with
+ *            32-bit coordinates); larger calls return CKDA_ERR_DIM.
  *   chunk   : 16, 32 or 64 tokens per chunk (a ragged last chunk is fine;
  *            chunks never span two sequences).
  *   workspace : device scratch of at least ckda_chunk_fwd_workspace_size()
@@ -133,15 +135,16 @@ int ckda_decode_step(const void *q, const void *k, const void *v, const void *a,
  * the process exits).  Sizes whose workspace would exceed 4096 bytes are
  * rejected with CKDA_ERR_WORKSPACE.  Neither this call nor the library calls
  * cudaMalloc or cudaFree.
- *   - The first call on each device looks up the scratch array's device
- *     address (cudaGetSymbolAddress) with that device current; make that
- *     first call before any stream capture.
+ *   - Every call looks up the scratch array's device address
+ *     (cudaGetSymbolAddress) with the caller's device current, so the address
+ *     is never stale.  The first call on a device may load the library's
+ *     device code there; make that first call before any stream capture.
  *   - Every call on a device shares the same scratch, and it keeps what the
  *     last call left there; the status header is cleared on `stream` at the
  *     start of each call.  Calls whose work overlaps on the GPU (different
  *     streams without ordering) race on the scratch: serialise them.
- *   - The device status word (bad cu_seqlens, timeouts) cannot be read back
- *     through ckda_workspace_status, since the caller has no pointer to it.
+ *   - The device status word (bad cu_seqlens, timeouts) of the last call is
+ *     read back with ckda_noalloc_status().
  * Returns CKDA_OK or a negative CKDA_ERR_* code.
  */
 int ckda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const void *a,
@@ -150,12 +153,36 @@ int ckda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const vo
                            int io_dtype, int o_dtype, void *o, float *S_T, void *stream);
 
 /*
+ * The device status word of the last ckda_chunk_fwd_noalloc call on the current
+ * device (CKDA_OK, CKDA_ERR_SEQLENS or CKDA_ERR_TIMEOUT), read from the
+ * library's scratch array into *status.  Like ckda_chunk_fwd_noalloc this has no
+ * counterpart on the pages.  It SYNCHRONISES `stream` (a 4-byte copy to the
+ * host) and allocates nothing.  Returns CKDA_OK or CKDA_ERR_NULL / CKDA_ERR_CUDA.
+ */
+int ckda_noalloc_status(int *status, void *stream);
+
+/*
  * Reads the device status word that ckda_chunk_fwd records in `workspace`
  * (CKDA_OK, CKDA_ERR_SEQLENS or CKDA_ERR_TIMEOUT) into *status.  This call
  * SYNCHRONISES `stream` (it copies 4 bytes to the host).  Returns CKDA_OK or
  * CKDA_ERR_NULL / CKDA_ERR_CUDA.
  */
 int ckda_workspace_status(const void *workspace, int *status, void *stream);
+
+/*
+ * TEST HOOK for the failure path of the bounded device waits; not needed in
+ * normal use.  After ckda_debug_wait_injection(chunk_index, wait_ns) with
+ * chunk_index >= 0, every later ckda_chunk_fwd call that runs on the
+ * tensor-core kernel (bf16 inputs, dk = dv = 128, chunk 64) adds, in every
+ * (sequence, head) unit that reaches chunk number `chunk_index`, one wait at
+ * the start of that chunk on a barrier that nothing ever arrives on, bounded
+ * by `wait_ns` nanoseconds (0 = the normal 2 s bound).  The wait runs out, the
+ * unit abandons its work (outputs of that unit are left unwritten or partial),
+ * lets every copy and product it started finish, releases its tensor memory
+ * and records CKDA_ERR_TIMEOUT in the status word.  chunk_index < 0 switches
+ * the hook off (the default).  Process-wide; takes effect at the next launch.
+ */
+void ckda_debug_wait_injection(int chunk_index, unsigned long long wait_ns);
 
 /* Static, human-readable text for a status code (never NULL). */
 const char *ckda_status_string(int status);

@@ -82,6 +82,9 @@ constexpr uint32_t IDESC_N128 = idesc_tf32(128, 128, false, false);       // (a)
 constexpr uint32_t IDESC_N192 = idesc_tf32(128, 192, false, false);       // (d)
 
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s bound on any single wait
+// bound on the waits that drain in-flight copies and products before a unit gives up (these
+// always finish; the bound only keeps a broken invariant from hanging the GPU)
+constexpr uint64_t kDrainNs = 2000000000ull;
 
 struct TcParams {
   const float *b;
@@ -91,6 +94,8 @@ struct TcParams {
   float *S_T;
   int *status;
   int n_seqs, T, H, signed_gate;
+  int inject_chunk;         // test hook: chunk index of the never-completing wait (-1: off)
+  uint64_t inject_wait_ns;  // its bound
 };
 
 // byte offset of fp32 element (r, c) in a 128-byte-swizzled tile of R rows
@@ -234,8 +239,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *bar_ack = bars + 10;
   // the last correction of (c) is done: the R tiles in Kc's area have been read
   uint64_t *bar_r4 = bars + 11;
+  // test hook: a barrier nothing ever arrives on (ckda_debug_wait_injection)
+  uint64_t *bar_never = bars + 12;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_MISC + 1392);
   volatile int *sAbort = reinterpret_cast<volatile int *>(sm + OFF_MISC + 1396);
+  // staging loads issued so far (by the issuer or compute thread 0); the compute warps count
+  // the ones they consumed, so a unit that gives up knows whether one is still in flight
+  unsigned int *sTmaIssued = reinterpret_cast<unsigned int *>(sm + OFF_MISC + 1400);
   const uint32_t sbase = smem_u32(sm);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -263,7 +273,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int x = 6; x < 10; ++x) mbar_init(bars + x, kCompute / 32);
     mbar_init(bar_ack, 1);
     mbar_init(bar_r4, 1);
+    mbar_init(bar_never, 1);
     *sAbort = 0;
+    *sTmaIssued = 0;
     mbar_fence_init();
   }
   if (warp == 0) tmem_alloc(tmem_slot, 512);
@@ -282,6 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto dadd = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (bytes >> 4); };
 
   auto issue_tma = [&](long cs) {
+    atomicAdd(sTmaIssued, 1u);
     mbar_arrive_expect_tx(bar_tma, 4 * 2 * 8192);
     const int row = (int)(bofs + cs);
     const CUtensorMap *maps[4] = {&tm_q, &tm_k, &tm_v, &tm_a};
@@ -291,6 +304,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int bx = 0; bx < 2; ++bx)
         tma_load_3d(sStg + x * 16384 + bx * 8192, maps[x], bar_tma, bx * 64, h, row);
   };
+
+  // the compute side's staging-load bookkeeping, for the drain at the end
+  uint32_t tma_ph_out = 0;
+  unsigned int tma_consumed_out = 0;
 
   if (warp == kCompute / 32) {
     // ================================================================ issuer (one thread)
@@ -389,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) *sAbort = 1;
       // every MMA issued above has finished before TMEM is released
       mma_commit(bar_fin);
-      mbar_wait(bar_fin, 0, kWaitNs);
+      mbar_wait(bar_fin, 0, kDrainNs);
     }
     __syncwarp();
   } else {
@@ -401,7 +418,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int jrow = 32 * (warp & 3) + lane;
     const int c = jrow;
     const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
-    uint32_t tma_ph = 0, mma1_ph = 0, a_ph = 0, d_ph = 0, ack_ph = 0, r4_ph = 0;
+    uint32_t tma_ph = 0, mma1_ph = 0, a_ph = 0, d_ph = 0, ack_ph = 0, r4_ph = 0, never_ph = 0;
+    unsigned int tma_consumed = 0;   // staging loads whose completion the compute warps saw
     // bf16 O (16 KB per chunk) is staged in T's tile and written by one TMA store;
     // fp32 O is written directly from registers
     constexpr bool kTmaStoreO = sizeof(TOut) == 2;
@@ -409,12 +427,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     auto csync = [&]() { bar_sync(kBarC, kCompute); };
     // warp 0 polls a completion barrier; the compute warps then agree on the outcome
-    auto cwait = [&](uint64_t *bar, uint32_t &ph) -> bool {
+    // (the phase advances only on success, so after a failure it still names the phase that
+    // did not complete)
+    auto cwait_for = [&](uint64_t *bar, uint32_t &ph, uint64_t limit_ns) -> bool {
       bool ok = true;
-      if (warp == 0) ok = mbar_wait_or_abort(bar, ph, kWaitNs, sAbort);
-      ph ^= 1;
-      return bar_and(kBarC, kCompute, ok);
+      if (warp == 0) ok = mbar_wait_or_abort(bar, ph, limit_ns, sAbort);
+      ok = bar_and(kBarC, kCompute, ok);
+      if (ok) {
+        ph ^= 1;
+        if (bar == bar_tma) ++tma_consumed;
+      }
+      return ok;
     };
+    auto cwait = [&](uint64_t *bar, uint32_t &ph) -> bool { return cwait_for(bar, ph, kWaitNs); };
     // one arrival per warp, after the whole warp's writes (each thread fenced its own)
     auto announce = [&](uint64_t *bar) {
       __syncwarp();
@@ -635,6 +660,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       float *gc_cur = sGC + 128 * gsel, *gc_next = sGC + 128 * (gsel ^ 1);
       const uint32_t vt_cur = gsel ? COL_VT1 : COL_VT0, vt_next = gsel ? COL_VT0 : COL_VT1;
 
+      if (p.inject_chunk >= 0 && (cs - t0) / kC == p.inject_chunk) {
+        // test hook: a wait that runs out (nothing arrives on bar_never)
+        if (!cwait_for(bar_never, never_ph, p.inject_wait_ns ? p.inject_wait_ns : kWaitNs)) {
+          failed = true;
+          break;
+        }
+      }
+
       if (slow) {
         // ------------------------------------------------------------ exact token-by-token path
         // state S[i][j] in smem over Kr/Qr, gates over Kc, partial sums over [P;Kc^T]; thread
@@ -854,13 +887,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (tid == 0) bulk_wait_all();
 
+    tma_ph_out = tma_ph;
+    tma_consumed_out = tma_consumed;
     if (failed) {
       if (tid == 0) {
         set_status(p.status, CKDA_ERR_TIMEOUT);
-        *sAbort = 1;
+        *sAbort = 1;   // the issuer leaves its loop at its next wait
       }
-      // a staging load may still be in flight: let it land (bounded) before leaving
-      if (tid == 0) mbar_wait(bar_tma, tma_ph, kWaitNs);
     } else if (p.S_T) {
       tc_fence_after();
       uint32_t r[32];
@@ -873,6 +906,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   tc_fence_before();
+  __syncthreads();
+  // Both sides have left their loops, so no further staging load can be issued.  A load the
+  // compute warps did not consume (a unit that gave up) must land before the CTA's shared
+  // memory is released; at most one is ever in flight, on the phase tma_ph names.  The issuer
+  // has already waited for its last products (bar_fin).
+  if (tid == 0 && *sTmaIssued != tma_consumed_out) mbar_wait(bar_tma, tma_ph_out, kDrainNs);
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
@@ -937,6 +976,8 @@ int launch_typed(const ChunkArgs &g, cudaStream_t stream) {
   TcParams p;
   p.b = g.b; p.S0 = g.S0; p.cu = g.cu_seqlens; p.o = g.o; p.S_T = g.S_T; p.status = g.status;
   p.n_seqs = g.n_seqs; p.T = g.T; p.H = g.H; p.signed_gate = g.signed_gate;
+  p.inject_chunk = g.inject_chunk;
+  p.inject_wait_ns = g.inject_wait_ns;
   auto kern = chunk_tc_kernel<TOut, SG>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) !=
       cudaSuccess)

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <climits>
 #include <cstdint>
 #include <cstring>
 
@@ -36,9 +37,42 @@ int check_device() {
   return ok ? CKDA_OK : CKDA_ERR_DEVICE;
 }
 
+// ckda_debug_wait_injection's settings (process-wide, read at each launch)
+std::atomic<int> g_inject_chunk{-1};
+std::atomic<unsigned long long> g_inject_wait_ns{0};
+
 }  // namespace
 
+namespace ckda {
+
+int check_chunk_args(const void *q, const void *k, const void *v, const void *a, const float *b,
+                     const float *S0, const int32_t *cu_seqlens, int n_seqs, int B, int T, int H,
+                     int dk, int dv, int chunk, int signed_gate, int io_dtype, int o_dtype,
+                     const void *o, const float *S_T) {
+  if (!q || !k || !v || !a || !b) return CKDA_ERR_NULL;
+  if (!valid_dim(dk) || !valid_dim(dv) || B < 0 || T < 0 || H <= 0) return CKDA_ERR_DIM;
+  if (chunk != 16 && chunk != 32 && chunk != 64) return CKDA_ERR_CHUNK;
+  if (signed_gate < 0 || signed_gate > 4 || (io_dtype != CKDA_F32 && io_dtype != CKDA_BF16) ||
+      (o_dtype != CKDA_F32 && o_dtype != CKDA_BF16))
+    return CKDA_ERR_DTYPE;
+  if (cu_seqlens && (B != 1 || n_seqs < 0)) return CKDA_ERR_DIM;
+  // token rows are 32-bit coordinates in the kernels (TMA tile coordinates included)
+  if ((long long)B * T > (long long)INT32_MAX || (long long)B * T * H > (1LL << 40))
+    return CKDA_ERR_DIM;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(a) || !aligned(b, 4) ||
+      !aligned16(S0) || !aligned16(o) || !aligned16(S_T) || !aligned(cu_seqlens, 4))
+    return CKDA_ERR_ALIGN;
+  return CKDA_OK;
+}
+
+}  // namespace ckda
+
 extern "C" {
+
+void ckda_debug_wait_injection(int chunk_index, unsigned long long wait_ns) {
+  g_inject_wait_ns.store(wait_ns, std::memory_order_relaxed);
+  g_inject_chunk.store(chunk_index < 0 ? -1 : chunk_index, std::memory_order_relaxed);
+}
 
 const char *ckda_status_string(int status) {
   switch (status) {
@@ -68,21 +102,10 @@ int ckda_chunk_fwd(const void *q, const void *k, const void *v, const void *a, c
                    const float *S0, const int32_t *cu_seqlens, int n_seqs, int B, int T, int H,
                    int dk, int dv, int chunk, int signed_gate, int io_dtype, int o_dtype,
                    void *o, float *S_T, void *workspace, size_t workspace_bytes, void *stream) {
-  if (!q || !k || !v || !a || !b) return CKDA_ERR_NULL;
-  if (!valid_dim(dk) || !valid_dim(dv) || B < 0 || T < 0 || H <= 0) return CKDA_ERR_DIM;
-  if (chunk != 16 && chunk != 32 && chunk != 64) return CKDA_ERR_CHUNK;
-  if (signed_gate < 0 || signed_gate > 4 || (io_dtype != CKDA_F32 && io_dtype != CKDA_BF16) ||
-      (o_dtype != CKDA_F32 && o_dtype != CKDA_BF16))
-    return CKDA_ERR_DTYPE;
-  int N = B;
-  if (cu_seqlens) {
-    if (B != 1 || n_seqs < 0) return CKDA_ERR_DIM;
-    N = n_seqs;
-  }
-  if ((long long)B * T * H > (1LL << 40)) return CKDA_ERR_DIM;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(a) || !aligned(b, 4) ||
-      !aligned16(S0) || !aligned16(o) || !aligned16(S_T) || !aligned(cu_seqlens, 4))
-    return CKDA_ERR_ALIGN;
+  const int arg_rc = ckda::check_chunk_args(q, k, v, a, b, S0, cu_seqlens, n_seqs, B, T, H, dk, dv,
+                                            chunk, signed_gate, io_dtype, o_dtype, o, S_T);
+  if (arg_rc != CKDA_OK) return arg_rc;
+  const int N = cu_seqlens ? n_seqs : B;
   const size_t need = ckda_chunk_fwd_workspace_size(B, T, H, dk, dv, chunk, n_seqs);
   if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return CKDA_ERR_WORKSPACE;
@@ -98,6 +121,8 @@ int ckda_chunk_fwd(const void *q, const void *k, const void *v, const void *a, c
   g.status = static_cast<int *>(workspace);
   g.workspace = workspace;
   g.workspace_bytes = workspace_bytes;
+  g.inject_chunk = g_inject_chunk.load(std::memory_order_relaxed);
+  g.inject_wait_ns = g_inject_wait_ns.load(std::memory_order_relaxed);
   if (ckda::chunk_tc_supported(g)) return ckda::launch_chunk_tc(g, s);
   return ckda::launch_chunk_simt(g, s);
 }

@@ -10,7 +10,6 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
-#include <mutex>
 
 #include "../../include/ckda.h"
 #include "internal.h"
@@ -24,22 +23,14 @@ static_assert(kNoAllocScratchBytes >= ckda::kWorkspaceHeader, "scratch smaller t
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mutex;
-void *g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of the scratch array on the current device (looked up once
-// per device; the host-side name of the array is not a device address).
+// Device address of the scratch array on the current device.  Looked up on every call: the
+// lookup is cheap once the library's module is loaded on the device, and a cached address
+// would go stale if the module were unloaded and loaded again (after cudaDeviceReset, for
+// example).  The host-side name of the array is only a stand-in, not a device address.
 int scratch_for_current_device(void **out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return CKDA_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_mutex);
-  if (!g_scratch_ptr[dev]) {
-    void *ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return CKDA_ERR_CUDA;
-    g_scratch_ptr[dev] = ptr;
-  }
-  *out = g_scratch_ptr[dev];
+  void *ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return CKDA_ERR_CUDA;
+  *out = ptr;
   return CKDA_OK;
 }
 
@@ -50,6 +41,10 @@ extern "C" int ckda_chunk_fwd_noalloc(const void *q, const void *k, const void *
                                       int n_seqs, int B, int T, int H, int dk, int dv, int chunk,
                                       int signed_gate, int io_dtype, int o_dtype, void *o,
                                       float *S_T, void *stream) {
+  // the arguments are checked before any CUDA call, as ckda_chunk_fwd does
+  const int arg_rc = ckda::check_chunk_args(q, k, v, a, b, S0, cu_seqlens, n_seqs, B, T, H, dk, dv,
+                                            chunk, signed_gate, io_dtype, o_dtype, o, S_T);
+  if (arg_rc != CKDA_OK) return arg_rc;
   const size_t need = ckda_chunk_fwd_workspace_size(B, T, H, dk, dv, chunk, n_seqs);
   if (need > kNoAllocScratchBytes) return CKDA_ERR_WORKSPACE;
   void *scratch = nullptr;
@@ -59,4 +54,17 @@ extern "C" int ckda_chunk_fwd_noalloc(const void *q, const void *k, const void *
   // its kernels run, so nothing a previous call left behind leaks into this one.
   return ckda_chunk_fwd(q, k, v, a, b, S0, cu_seqlens, n_seqs, B, T, H, dk, dv, chunk, signed_gate,
                         io_dtype, o_dtype, o, S_T, scratch, kNoAllocScratchBytes, stream);
+}
+
+extern "C" int ckda_noalloc_status(int *status, void *stream) {
+  if (!status) return CKDA_ERR_NULL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int host = 0;
+  // offset 0 of the scratch is the status word the kernels write (the workspace header)
+  if (cudaMemcpyFromSymbolAsync(&host, g_noalloc_scratch, sizeof(int), 0, cudaMemcpyDeviceToHost,
+                                s) != cudaSuccess)
+    return CKDA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return CKDA_ERR_CUDA;
+  *status = host;
+  return CKDA_OK;
 }

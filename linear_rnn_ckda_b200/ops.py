@@ -35,6 +35,8 @@ SIGNATURES = {
     "ckda_chunk_fwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
                                     _i, _i, _i, _vp, _vp, _vp]),
     "ckda_workspace_status": (_i, [_vp, ctypes.POINTER(_i), _vp]),
+    "ckda_noalloc_status": (_i, [ctypes.POINTER(_i), _vp]),
+    "ckda_debug_wait_injection": (None, [_i, ctypes.c_ulonglong]),
     "ckda_status_string": (ctypes.c_char_p, [_i]),
     "ckda_version": (_i, []),
 }
@@ -209,6 +211,22 @@ def decode_step(q, k, v, a, b, S, signed_gate: int = 1, o_dtype=None, o=None, wa
     if rc != 0:
         raise CkdaError("ckda_decode_step", rc)
     return o if want_o else None
+
+
+def noalloc_status(device=None) -> int:
+    """Device status word of the last ``ckda_chunk_fwd_noalloc`` call on the current device
+    (synchronises the current stream)."""
+    st = ctypes.c_int(0)
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    rc = load().ckda_noalloc_status(ctypes.byref(st), _stream(dev))
+    if rc != 0:
+        raise CkdaError("ckda_noalloc_status", rc)
+    return st.value
+
+
+def debug_wait_injection(chunk_index: int, wait_ns: int = 0) -> None:
+    """Test hook: see ``ckda_debug_wait_injection`` in ``include/ckda.h`` (-1 switches it off)."""
+    load().ckda_debug_wait_injection(int(chunk_index), int(wait_ns))
 
 
 def workspace_status(workspace: torch.Tensor) -> int:

@@ -95,6 +95,8 @@ def _dec(lib, **kw):
     (dict(k=MIS), -5), (dict(o=MIS), -5), (dict(S0=MIS), -5), (dict(S_T=MIS), -5),
     (dict(b=ODD), -5), (dict(cu=ODD), -5),
     (dict(ws=None), -7), (dict(wsb=16), -7), (dict(ws=ctypes.c_void_p((1 << 20) + 16)), -7),
+    # token rows are 32-bit coordinates: B * T above 2^31 - 1 is refused
+    (dict(B=2, T=1 << 30), -2), (dict(B=1 << 16, T=1 << 15), -2),
 ])
 def test_chunk_fwd_rejects(lib, kw, code):
     assert _fwd(lib, **kw) == code
@@ -112,6 +114,26 @@ def test_decode_rejects(lib, kw, code):
 def test_workspace_status_rejects_null(lib):
     st = ctypes.c_int(0)
     assert lib.ckda_workspace_status(None, ctypes.byref(st), None) == -1
+    assert lib.ckda_noalloc_status(None, None) == -1
+
+
+def test_largest_token_count_passes_validation(lib):
+    """B * T = 2^31 - 1 is inside the limit: with a too-small workspace the call gets past the
+    size checks and stops at the workspace check (no CUDA call is made)."""
+    assert _fwd(lib, B=1, T=(1 << 31) - 1, wsb=0) == -7
+
+
+def test_noalloc_rejects_before_any_cuda_call(lib):
+    """The no-allocation entry point validates like ckda_chunk_fwd (a bad chunk size)."""
+    rc = lib.ckda_chunk_fwd_noalloc(P, P, P, P, P, None, None, 0, 1, 8, 1, 16, 16, 8, 1, 0, 0, P, P,
+                                    None)
+    assert rc == -3
+
+
+def test_wait_injection_hook_is_settable(lib):
+    """The test hook takes any value and is switched off again (no device work)."""
+    ops.debug_wait_injection(3, 1000)
+    ops.debug_wait_injection(-1, 0)
 
 
 def test_binding_has_no_cpu_fallback(lib):

@@ -9,7 +9,7 @@ import ctypes
 import pytest
 import torch
 
-from helpers import TOL_BF16, TOL_FP32, f64, rel, to_device
+from helpers import TOL_BF16, TOL_FP32, assert_close, f64, to_device
 from linear_rnn_ckda_b200 import synth
 
 pytestmark = pytest.mark.gpu
@@ -43,8 +43,30 @@ def test_noalloc_matches_workspace_entry_point(cuda_lib, w, tol):
         S_T = torch.full_like(ref_S, float("nan"))
         _noalloc(cuda_lib, d, w, o, S_T)
         torch.cuda.synchronize()
-        assert rel(f64(o), f64(ref_o)) <= tol, call
-        assert rel(f64(S_T), f64(ref_S)) <= tol, call
+        assert cuda_lib.noalloc_status() == 0, call
+        assert_close(f64(o), f64(ref_o), tol, f"o call {call}")
+        assert_close(f64(S_T), f64(ref_S), tol, f"S_T call {call}")
+
+
+def test_noalloc_status_reports_bad_offsets_then_clears(cuda_lib):
+    """Offsets that do not end at T make the kernel skip the bad sequence and record
+    CKDA_ERR_SEQLENS in the scratch's status word, readable with ckda_noalloc_status; the
+    next good call starts from a cleared status and matches ckda_chunk_fwd."""
+    w = synth.CKDA_SPREAD.with_(B=1, H=2, seq_lens=(50, 70), T=120, o_dtype="f32")
+    d = to_device(synth.make_prefill(w, seed=42))
+    bad = dict(d, cu_seqlens=torch.tensor([0, 50, 110], dtype=torch.int32, device="cuda"))
+    o = torch.zeros(1, 120, 2, 128, device="cuda")
+    S_T = torch.zeros(2, 2, 128, 128, device="cuda")
+    _noalloc(cuda_lib, bad, w, o, S_T)
+    assert cuda_lib.noalloc_status() == -6          # CKDA_ERR_SEQLENS
+    ref_o, ref_S = cuda_lib.chunk_fwd(d["q"], d["k"], d["v"], d["a"], d["b"], d["S0"],
+                                      d["cu_seqlens"], signed_gate=1, o_dtype=torch.float32)
+    o = torch.full_like(ref_o, float("nan"))
+    S_T = torch.full_like(ref_S, float("nan"))
+    _noalloc(cuda_lib, d, w, o, S_T)
+    assert cuda_lib.noalloc_status() == 0
+    assert_close(f64(o), f64(ref_o), TOL_BF16, "o after a failed call")
+    assert_close(f64(S_T), f64(ref_S), TOL_BF16, "S_T after a failed call")
 
 
 def test_noalloc_rejects_bad_arguments(cuda_lib):
