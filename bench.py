@@ -2,19 +2,23 @@
 """Benchmark of the KDA / Complex-KDA hot path on B200.
 
 Prints ONE JSON line (rank 0).  The headline is the chunkwise prefill
-(``ckda_chunk_fwd``) on the standard KDA workload B=4, H=16, T=4096,
-dk=dv=128, chunk 64, bf16 q/k/v/a, bf16 o, fp32 state: ``value`` is prefill
-tokens/s for the whole job, one step = one ``ckda_chunk_fwd`` call over the
-whole batch with its inputs resident in HBM.  The same run times the decode
-step (``ckda_decode_step``, B=256, H=32, d=128, fp32 state updated in place,
-bf16 q/k/v/a, fp32 o) and reports its state GB/s against HBM in ``decode``.
+(``ckda_chunk_fwd``) on the largest single-GPU workload, the long-context
+varlen CKDA batch: H=32, dk=dv=128, 16 packed sequences of lengths uniform in
+[512, 8192] plus one of 65,536 tokens (cu_seqlens), per-sequence S0 ~ N(0, 0.02),
+chunk 64, bf16 q/k/v/a, bf16 o, fp32 state.  ``value`` is prefill tokens/s for
+the whole job; one step = one ``ckda_chunk_fwd`` call over the whole packed
+batch with its inputs resident in HBM.  The same run reports, each with its own
+roofline: the KDA workload (B=4, T=4096, H=16), the CKDA spread-init workload
+(B=8, T=8192, H=16, S0), the CKDA/KDA throughput ratio of the same kernel, and
+the decode step (``ckda_decode_step``, B=256, H=32, fp32 state in place) as
+state GB/s against HBM.
 
-Multi-GPU (torchrun, one rank per GPU): every rank runs the same workload on
+Multi-GPU (torchrun, one rank per GPU): every rank runs the same workloads on
 its own seeded data (independent (sequence, head) units, no data-path
 collective); ``value`` = all ranks' tokens / max-over-ranks time ("weak").
 
 ``--impl reference`` times the fp64 CPU oracle (the only other arm; there is
-no installable reference implementation) on a bounded sample of the same
+no installable reference implementation) on a bounded sample of the headline
 workload, on the host cores of rank 0.
 """
 from __future__ import annotations
@@ -35,14 +39,17 @@ import torch  # noqa: E402
 
 from linear_rnn_ckda_b200 import synth  # noqa: E402
 
-PREFILL = synth.KDA_STD
-DECODE = synth.DECODE
+# the metric as the headline's definition states it (both arms print it verbatim)
+METRIC = "chunk-fwd prefill tokens/s + % tensor roofline; decode state GB/s vs HBM peak"
+HEADLINE = synth.varlen_workload(0)
+KDA = synth.KDA_STD
 SPREAD = synth.CKDA_SPREAD
+DECODE = synth.DECODE
 
 # Algorithmic counts per unit (d = dk = dv = 128, chunk C = 64):
 #   prefill FLOP per token-head = 6 d^2 + C (3 dk + 2 dv) + C^2 / 3
 #   prefill bytes per token-head = q + k + v + a (bf16) + b (fp32) + o (bf16)
-#   plus S_T (fp32 d^2) per (sequence, head); S0 is not read (zero state)
+#   plus S_T (fp32 d^2) per (sequence, head), and S0 when the workload has one
 #   decode bytes per head-step = read + write of the fp32 state + q, k, v, a, b, o
 
 
@@ -80,12 +87,13 @@ def source_hash(files):
     return h.hexdigest()
 
 
-def profiled_traffic(kernel):
-    """DRAM bytes per launch from the committed ncu capture of `kernel`, or None
-    when the kernel's sources changed after the capture."""
+def profiled_traffic(key):
+    """DRAM bytes per launch of one kernel on one workload (``key`` = "kernel/workload") from
+    the committed ncu capture, or None when there is none or the kernel's sources changed
+    after the capture."""
     try:
         with open(PROFILED) as f:
-            rec = json.load(f)[kernel]
+            rec = json.load(f)[key]
         if source_hash(rec["sources"]) != rec["source_sha256"]:
             return None
         return float(rec["dram_bytes_per_launch"])
@@ -218,51 +226,127 @@ def time_loop(fn, steps, warmup, world, stream):
     return ev0.elapsed_time(ev1)  # ms
 
 
-def cpu_oracle_sample(w, seed, max_units=None):
-    """Oracle on a bounded sample of (sequence, head) units of workload w: (seconds, token-heads, cores)."""
+def _oracle_run(inp, signed_gate, threads):
+    """The oracle on one host input dict (upcast to fp64); returns its wall time."""
     import numpy as np
 
     import oracle
 
-    cores = os.cpu_count() or 1
-    H = w.H
-    inp = synth.make_prefill(w.with_(B=1), seed)  # one batch row = H units of T tokens
-    units = H if max_units is None else min(H, max_units)
-    f = lambda t: t[:, :, :units].to(torch.float64).numpy()
-    q, k, v, a = (np.ascontiguousarray(f(inp[x])) for x in "qkva")
-    b = np.ascontiguousarray(inp["b"][:, :, :units].to(torch.float64).numpy())
+    f = lambda t: None if t is None else np.ascontiguousarray(t.to(torch.float64).numpy())
+    cu = inp.get("cu_seqlens")
+    args = [f(inp[x]) for x in "qkvab"]
     oracle.build()
     t0 = time.perf_counter()
-    oracle.ckda_fwd(q, k, v, a, b, None, signed_gate=w.signed_gate, threads=cores)
-    dt = time.perf_counter() - t0
-    return dt, units * w.T, min(cores, units)
+    oracle.ckda_fwd(*args, f(inp.get("S0")), cu_seqlens=None if cu is None else cu.numpy(),
+                    signed_gate=signed_gate, threads=threads, want_o=True)
+    return time.perf_counter() - t0
+
+
+def _slice_sequences(inp, lo, hi):
+    """Sequences lo..hi-1 of a packed (cu_seqlens) input dict, repacked."""
+    cu = inp["cu_seqlens"]
+    t0, t1 = int(cu[lo]), int(cu[hi])
+    out = {x: inp[x][:, t0:t1].contiguous() for x in "qkvab"}
+    out["S0"] = None if inp.get("S0") is None else inp["S0"][lo:hi].contiguous()
+    out["cu_seqlens"] = (cu[lo:hi + 1] - cu[lo]).to(torch.int32)
+    return out
+
+
+def cpu_baseline_sample(host, w, seqs):
+    """The oracle, as it stands, on sequences ``seqs`` (a range) of the packed workload ``w``
+    (all heads) with every host core: (tokens/s, cores, description)."""
+    cores = os.cpu_count() or 1
+    sub = _slice_sequences(host, seqs.start, seqs.stop)
+    tokens = int(sub["cu_seqlens"][-1])
+    dt = _oracle_run(sub, w.signed_gate, cores)
+    units = (seqs.stop - seqs.start) * w.H
+    desc = (f"sequences {seqs.start}..{seqs.stop - 1} of {w.name} ({tokens} tokens x {w.H} heads, "
+            f"{units} (sequence, head) units), fp64 sequential per unit, {dt:.2f} s wall")
+    return tokens / dt, min(cores, units), desc
 
 
 def run_reference(args, world, rank):
+    """The reference arm: the oracle on the host cores, on a bounded sample of the headline
+    workload per step (two of its sequences, regenerated from the same recipe), with the
+    headline's metric, unit and config."""
     if rank != 0:
         return
-    w = PREFILL
-    times = []
-    th = 0
-    cores = 1
+    w = HEADLINE
+    lens = w.seq_lens
+    cores = os.cpu_count() or 1
+    times, toks = [], []
     for i in range(args.warmup + args.steps):
-        dt, th, cores = cpu_oracle_sample(w, seed=i)
+        j = (2 * i) % 16
+        sw = w.with_(seq_lens=(lens[j], lens[j + 1]), T=lens[j] + lens[j + 1])
+        inp = synth.make_prefill(sw, seed=1000 + i)
+        dt = _oracle_run(inp, w.signed_gate, cores)
         if i >= args.warmup:
             times.append(dt)
+            toks.append(sw.tokens)
     tot = sum(times)
-    value = (th / w.H) * len(times) / tot  # tokens/s (a token carries H heads)
-    sample = f"one batch row of {w.name}: {w.H} heads x {w.T} tokens per step (fp64, sequential per head)"
+    value = sum(toks) / tot
+    sample = (f"per step two of the 16 short sequences of {w.name} (lengths from its length "
+              f"list, regenerated from the same recipe; {w.H} heads each), fp64 sequential per "
+              f"(sequence, head) unit")
     line = {
-        "impl": "reference", "metric": "chunk-fwd prefill tokens/s", "value": value,
+        "impl": "reference", "metric": METRIC, "value": value,
         "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1000 * tot / len(times), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "sample": sample},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": sample},
+        "config": headline_config(w),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": min(cores, 2 * w.H),
+                         "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def headline_config(w):
+    return {"workload": w.name, "H": w.H, "dk": w.dk, "dv": w.dv, "chunk": w.chunk,
+            "signed_gate": w.signed_gate, "n_seqs": w.n_seqs, "tokens": w.tokens,
+            "seq_lens": "16 x U{512..8192} (seed 0) + 65536", "io_dtype": w.io_dtype,
+            "o_dtype": w.o_dtype, "state_dtype": "f32", "S0": "N(0, 0.02) per sequence",
+            "l2": "inputs larger than L2 (q,k,v,a 4.4 GB + o 1.1 GB per step)"}
+
+
+def to_dev(host, dev):
+    return {k: (None if v is None else v.to(dev)) for k, v in host.items()}
+
+
+class PrefillCase:
+    """One workload's device buffers and its ckda_chunk_fwd call."""
+
+    def __init__(self, ops, w, host, dev, signed_gate=None):
+        self.ops, self.w = ops, w
+        self.sg = w.signed_gate if signed_gate is None else signed_gate
+        self.d = to_dev(host, dev)
+        B, T = host["q"].shape[:2]
+        self.o = torch.empty((B, T, w.H, w.dv), dtype=torch.bfloat16, device=dev)
+        self.S_T = torch.empty((w.n_seqs, w.H, w.dk, w.dv), dtype=torch.float32, device=dev)
+        self.ws = ops.new_workspace(B, T, w.H, w.dk, w.dv, w.chunk, w.n_seqs, dev)
+
+    def __call__(self):
+        d = self.d
+        self.ops.chunk_fwd(d["q"], d["k"], d["v"], d["a"], d["b"], d["S0"], d["cu_seqlens"],
+                           chunk=self.w.chunk, signed_gate=self.sg, o=self.o, S_T=self.S_T,
+                           workspace=self.ws)
+
+    def check(self, what):
+        st = self.ops.workspace_status(self.ws)
+        if st != 0:
+            raise RuntimeError(f"device status {st} after {what}")
+
+
+def prefill_roofline(w, ms_launch, peaks, traffic_key):
+    byts = prefill_bytes(w)
+    flops = prefill_flops_per_token_head(w.dk, w.dv, w.chunk) * w.tokens * w.H
+    gbs = byts / (ms_launch * 1e-3) / 1e9
+    tf = flops / (ms_launch * 1e-3) / 1e12
+    return {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": gbs / peaks["hbm_gbs"], "traffic": profiled_traffic(traffic_key),
+            "peak_source": peaks["source"], "algorithmic_bytes_per_launch": byts,
+            "algorithmic_flop_per_launch": flops, "tensor_tflops": tf,
+            "tensor_frac_of_bf16": tf / peaks["bf16_tflops"]}
 
 
 def main():
@@ -274,9 +358,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--decode-steps", type=int, default=None,
                     help="timed decode steps (default: --steps rounded up to the 128-step cycle)")
-    ap.add_argument("--legs", default="prefill,e2e,ckda,decode",
-                    help="comma list of legs to run (prefill, e2e, ckda, decode); a profiling "
-                         "run can select one, the default runs all")
+    ap.add_argument("--legs", default="varlen,e2e,kda,spread,ratio,decode",
+                    help="comma list of legs to run (varlen = the headline, e2e, kda, spread, "
+                         "ratio, decode); a profiling run can select one, the default runs all")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -295,65 +379,46 @@ def main():
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
     peaks = load_peaks()
-
     legs = set(args.legs.split(","))
-    # ------------------------------------------------------------ prefill leg
-    w = PREFILL
+    extra_steps = max(3, min(args.steps, 10))
+
+    # ------------------------------------------------------------ headline: varlen CKDA
+    w = HEADLINE
     host = synth.make_prefill(w, seed=rank)
-    d = {k: (None if v is None else v.to(dev)) for k, v in host.items()}
-    o = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.bfloat16, device=dev)
-    S_T = torch.empty((w.n_seqs, w.H, w.dk, w.dv), dtype=torch.float32, device=dev)
-    ws = ops.new_workspace(w.B, w.T, w.H, w.dk, w.dv, w.chunk, 0, dev)
-
-    def prefill():
-        ops.chunk_fwd(d["q"], d["k"], d["v"], d["a"], d["b"], None, None, chunk=w.chunk,
-                      signed_gate=w.signed_gate, o=o, S_T=S_T, workspace=ws)
-
+    case = PrefillCase(ops, w, host, dev)
+    run_head = "varlen" in legs
     with ClockSampler(local) as clk:
-        ms = time_loop(prefill, args.steps if "prefill" in legs else 1,
-                       args.warmup if "prefill" in legs else 0, world, stream)
-    if "prefill" not in legs:
-        ms = float("nan")
-    ms = max_over_ranks(ms, world)
+        ms = time_loop(case, args.steps if run_head else 1, args.warmup if run_head else 0, world,
+                       stream)
+    ms = max_over_ranks(ms, world) if run_head else float("nan")
+    case.check("the headline leg")
     ms_step = ms / args.steps
     tokens = w.tokens * world
     value = tokens * args.steps / (ms / 1000.0)
-    status = ops.workspace_status(ws)
-    if status != 0:
-        raise RuntimeError(f"device status {status} after the prefill leg")
+    # dominant kernel: the chunk kernel, one launch per step (the 256-byte status memset
+    # before it is included, < 2 us)
+    roofline = prefill_roofline(w, ms_step, peaks, "chunk_tc_kernel/" + w.name)
 
-    # dominant kernel: the chunk kernel; its launch average from the same events
-    # (the memset of the 256-byte status word is included, < 2 us)
-    byts = prefill_bytes(w)
-    flops = prefill_flops_per_token_head(w.dk, w.dv, w.chunk) * w.tokens * w.H
-    achieved_gbs = byts / (ms_step * 1e-3) / 1e9
-    roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved_gbs / peaks["hbm_gbs"],
-                "traffic": profiled_traffic("chunk_tc_kernel"),
-                "peak_source": peaks["source"],
-                "algorithmic_bytes_per_launch": byts, "algorithmic_flop_per_launch": flops,
-                "tensor_tflops": flops / (ms_step * 1e-3) / 1e12,
-                "tensor_frac_of_bf16": flops / (ms_step * 1e-3) / 1e12 / peaks["bf16_tflops"]}
-
-    # ------------------------------------------------------------ e2e prefill (host buffers)
-    # Each step copies its own q, k, v, a, b from pinned host memory, runs ckda_chunk_fwd and
-    # reads o and S_T back.  Steps are pipelined the way a streaming caller would run them:
-    # input copies, compute and output copies on three streams with two sets of device
-    # buffers, so one step's read-back overlaps the next step's upload (the link carries the
-    # two directions at once).  Timed with CUDA events from the first upload to the last
-    # read-back.
+    # ------------------------------------------------------------ e2e (host buffers)
+    # Each step copies its own q, k, v, a, b, S0 and cu_seqlens from pinned host memory, runs
+    # ckda_chunk_fwd and reads o and S_T back.  Steps are pipelined the way a streaming caller
+    # would run them: input copies, compute and output copies on three streams with two sets
+    # of device buffers, so one step's read-back overlaps the next step's upload.  Timed with
+    # CUDA events from the first upload to the last read-back.
     e2e = None
-    pin = {k: (None if v is None else v.pin_memory()) for k, v in host.items()}
-    h2d = sum(v.numel() * v.element_size() for k, v in pin.items() if v is not None and k in "qkvab")
-    d2h = o.numel() * o.element_size() + S_T.numel() * S_T.element_size()
+    keys = [k for k in ("q", "k", "v", "a", "b", "S0", "cu_seqlens") if host.get(k) is not None]
+    h2d = sum(host[k].numel() * host[k].element_size() for k in keys)
+    d2h = case.o.numel() * case.o.element_size() + case.S_T.numel() * case.S_T.element_size()
     if "e2e" in legs:
+        pin = {k: host[k].pin_memory() for k in keys}
         nbuf = 2
         s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-        dd = [{k: torch.empty_like(host[k], device=dev) for k in "qkvab"} for _ in range(nbuf)]
-        oo = [torch.empty_like(o) for _ in range(nbuf)]
-        SS = [torch.empty_like(S_T) for _ in range(nbuf)]
-        o_host = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for _ in range(nbuf)]
-        S_host = [torch.empty(S_T.shape, dtype=S_T.dtype).pin_memory() for _ in range(nbuf)]
+        dd = [{k: torch.empty_like(host[k], device=dev) for k in keys} for _ in range(nbuf)]
+        oo = [torch.empty_like(case.o) for _ in range(nbuf)]
+        SS = [torch.empty_like(case.S_T) for _ in range(nbuf)]
+        o_host = [torch.empty(case.o.shape, dtype=case.o.dtype).pin_memory() for _ in range(nbuf)]
+        S_host = [torch.empty(case.S_T.shape, dtype=case.S_T.dtype).pin_memory()
+                  for _ in range(nbuf)]
         ev_in = [torch.cuda.Event() for _ in range(nbuf)]
         ev_done = [torch.cuda.Event() for _ in range(nbuf)]
         ev_out = [torch.cuda.Event() for _ in range(nbuf)]
@@ -366,14 +431,15 @@ def main():
             step_no[0] += 1
             with torch.cuda.stream(s_in):
                 s_in.wait_event(ev_done[i])          # the step that last used buffer set i
-                for k in "qkvab":
+                for k in keys:
                     dd[i][k].copy_(pin[k], non_blocking=True)
                 ev_in[i].record(s_in)
             stream.wait_event(ev_in[i])
             stream.wait_event(ev_out[i])             # its outputs have been read back
-            ops.chunk_fwd(dd[i]["q"], dd[i]["k"], dd[i]["v"], dd[i]["a"], dd[i]["b"], None, None,
+            x = dd[i]
+            ops.chunk_fwd(x["q"], x["k"], x["v"], x["a"], x["b"], x.get("S0"), x.get("cu_seqlens"),
                           chunk=w.chunk, signed_gate=w.signed_gate, o=oo[i], S_T=SS[i],
-                          workspace=ws)
+                          workspace=case.ws)
             ev_done[i].record(stream)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev_done[i])
@@ -381,7 +447,6 @@ def main():
                 S_host[i].copy_(SS[i], non_blocking=True)
                 ev_out[i].record(s_out)
 
-        e2e_steps = max(3, min(args.steps, 10))
         for _ in range(2):
             e2e_step()
         torch.cuda.synchronize()
@@ -390,7 +455,7 @@ def main():
         t0e = torch.cuda.Event(enable_timing=True)
         t1e = torch.cuda.Event(enable_timing=True)
         t0e.record(s_in)
-        for _ in range(e2e_steps):
+        for _ in range(extra_steps):
             e2e_step()
         s_in.wait_stream(stream)
         s_in.wait_stream(s_out)
@@ -398,53 +463,48 @@ def main():
         torch.cuda.synchronize()
         barrier(world)
         ms_e2e = max_over_ranks(t0e.elapsed_time(t1e), world)
-        if ops.workspace_status(ws) != 0:
-            raise RuntimeError("device status after the end-to-end leg")
-        e2e = {"value": tokens * e2e_steps / (ms_e2e / 1000.0), "unit": "tokens/s",
+        case.check("the end-to-end leg")
+        e2e = {"value": tokens * extra_steps / (ms_e2e / 1000.0), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": ms_e2e / e2e_steps, "pipelined": "2 buffer sets, 3 streams"}
-        del dd, oo, SS, o_host, S_host
-    del pin
+               "ms_per_step": ms_e2e / extra_steps, "steps": extra_steps,
+               "pipelined": "2 buffer sets, 3 streams"}
+        del dd, oo, SS, o_host, S_host, pin
 
-    # ------------------------------------------------------------ CKDA legs
-    # the same kernel in signed-gate (CKDA) mode: on the KDA shapes and inputs (the throughput
-    # ratio the pages quote as 96-97%), and on the CKDA spread-init workload
-    ckda = None
-    if "ckda" in legs:
-        csteps = max(3, min(args.steps, 10))
+    # ------------------------------------------------------------ CPU baseline (oracle)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v_cpu, cores, desc = cpu_baseline_sample(host, w, range(0, 16))
+        cpu = {"value": v_cpu, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": desc}
+    del case, host
 
-        def prefill_ckda():
-            ops.chunk_fwd(d["q"], d["k"], d["v"], d["a"], d["b"], None, None, chunk=w.chunk,
-                          signed_gate=1, o=o, S_T=S_T, workspace=ws)
+    # ------------------------------------------------------------ the other prefill workloads
+    workloads = {}
+    for leg, wk in (("kda", KDA), ("spread", SPREAD)):
+        if leg not in legs:
+            continue
+        c = PrefillCase(ops, wk, synth.make_prefill(wk, seed=rank), dev)
+        ms_k = max_over_ranks(time_loop(c, extra_steps, args.warmup, world, stream), world)
+        c.check(f"the {leg} leg")
+        ms_l = ms_k / extra_steps
+        workloads[wk.name] = {
+            "ms_per_step": ms_l, "steps": extra_steps,
+            "tokens_per_s": wk.tokens * world / (ms_l / 1000.0),
+            "roofline": prefill_roofline(wk, ms_l, peaks, "chunk_tc_kernel/" + wk.name)}
+        if leg == "kda" and "ratio" in legs:
+            # the same kernel in signed-gate (CKDA) mode on the KDA shapes and inputs: the
+            # throughput ratio the pages quote (96-97 %, forward and backward, on H100)
+            c.sg = 1
+            ms_c = max_over_ranks(time_loop(c, extra_steps, args.warmup, world, stream), world)
+            c.check("the CKDA ratio leg")
+            c.sg = wk.signed_gate
+            ms_k2 = max_over_ranks(time_loop(c, extra_steps, args.warmup, world, stream), world)
+            workloads[wk.name]["ckda_over_kda_throughput"] = (ms_k2 / extra_steps) / (
+                ms_c / extra_steps)
+            workloads[wk.name]["ckda_mode_ms_per_step"] = ms_c / extra_steps
+        del c
 
-        ms_k = max_over_ranks(time_loop(prefill, csteps, args.warmup, world, stream), world)
-        ms_c = max_over_ranks(time_loop(prefill_ckda, csteps, args.warmup, world, stream), world)
-        if ops.workspace_status(ws) != 0:
-            raise RuntimeError("device status after the CKDA leg")
-        ws_ = SPREAD
-        hs = synth.make_prefill(ws_, seed=rank)
-        ds = {k: (None if v is None else v.to(dev)) for k, v in hs.items()}
-        os_ = torch.empty((ws_.B, ws_.T, ws_.H, ws_.dv), dtype=torch.bfloat16, device=dev)
-        Ss = torch.empty((ws_.n_seqs, ws_.H, ws_.dk, ws_.dv), dtype=torch.float32, device=dev)
-        wss = ops.new_workspace(ws_.B, ws_.T, ws_.H, ws_.dk, ws_.dv, ws_.chunk, 0, dev)
-
-        def spread():
-            ops.chunk_fwd(ds["q"], ds["k"], ds["v"], ds["a"], ds["b"], ds["S0"], None,
-                          chunk=ws_.chunk, signed_gate=ws_.signed_gate, o=os_, S_T=Ss,
-                          workspace=wss)
-
-        ms_s = max_over_ranks(time_loop(spread, csteps, args.warmup, world, stream), world)
-        if ops.workspace_status(wss) != 0:
-            raise RuntimeError("device status after the CKDA spread leg")
-        ckda = {"workload": w.name, "steps": csteps,
-                "kda_ms_per_step": ms_k / csteps, "ckda_ms_per_step": ms_c / csteps,
-                "ckda_over_kda_throughput": ms_k / ms_c,
-                "spread": {"workload": ws_.name, "ms_per_step": ms_s / csteps,
-                           "tokens_per_s": ws_.tokens * world * csteps / (ms_s / 1000.0),
-                           "hbm_gbs": prefill_bytes(ws_) * world * csteps / (ms_s / 1000.0) / 1e9}}
-        del ds, os_, Ss, wss
-
-    # ------------------------------------------------------------ decode leg
+    # ------------------------------------------------------------ decode
     wd = DECODE
     dsteps = args.decode_steps or max(args.steps, 128)
     decode_obj = None
@@ -467,30 +527,19 @@ def main():
                       "peak": peaks["hbm_gbs"], "ms_per_step": ms_d / dsteps, "steps": dsteps,
                       "workload": wd.name, "algorithmic_bytes_per_step": dbytes,
                       "state_bytes_per_step": wd.B * wd.H * wd.dk * wd.dv * 8,
-                      "traffic": profiled_traffic("decode_kernel")}
-
-    # ------------------------------------------------------------ CPU baseline (oracle)
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        dt, th, cores = cpu_oracle_sample(w, seed=0)
-        cpu = {"value": (th / w.H) / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-               "sample": f"one batch row of {w.name} ({w.H} heads x {w.T} tokens), "
-                         f"fp64 sequential per head, {dt:.2f} s wall"}
+                      "traffic": profiled_traffic("decode_kernel/" + wd.name)}
 
     clocks = clk.summary()
     if rank == 0:
         line = {
-            "metric": "chunk-fwd prefill tokens/s (+ % roofline); decode state GB/s vs HBM",
+            "metric": METRIC,
             "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded; same shapes and distributions as the pages' workloads)",
-            "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk, "dv": w.dv,
-                       "chunk": w.chunk, "signed_gate": w.signed_gate, "io_dtype": w.io_dtype,
-                       "o_dtype": w.o_dtype, "state_dtype": "f32",
-                       "l2": "inputs larger than L2 (q,k,v,a 268 MB + o 67 MB per step)"},
-            "roofline": roofline, "decode": decode_obj, "ckda": ckda, "cpu_baseline": cpu,
-            "e2e": e2e,
+            "config": headline_config(w),
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "workloads": workloads, "decode": decode_obj,
             "gpu_launches": args.steps, "clocks": clocks, "peaks_source": peaks["source"],
         }
         print(json.dumps(line), flush=True)
