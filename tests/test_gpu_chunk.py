@@ -374,7 +374,7 @@ def test_tc_wait_timeout_recovers(cuda_lib, chunk_index):
     try:
         cuda_lib.debug_wait_injection(chunk_index, 200_000)     # 0.2 ms bound
         cuda_lib.chunk_fwd(d["q"], d["k"], d["v"], d["a"], d["b"], d["S0"], d["cu_seqlens"],
-                           signed_gate=1, o=o, S_T=S, workspace=ws)
+                           signed_gate=1, o_dtype=torch.float32, o=o, S_T=S, workspace=ws)
         assert cuda_lib.workspace_status(ws) == -8      # CKDA_ERR_TIMEOUT
     finally:
         cuda_lib.debug_wait_injection(-1, 0)
