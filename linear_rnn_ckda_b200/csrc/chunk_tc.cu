@@ -214,6 +214,33 @@ __device__ __forceinline__ void solve_T_zeros(uint8_t *sT, int t) {
   }
 }
 
+// Packed batches are processed longest first: the sequence whose rank in descending length
+// order (ties: lower index first) is `rank`.  Every thread of the block calls this; s_cu is
+// shared scratch of n_seqs + 2 ints.  Past kMaxRanked sequences the order is left as given
+// (the ranking is O(n^2) per block).  Offsets are only read here; each block checks its own
+// sequence's offsets afterwards.
+constexpr int kMaxRanked = 1024;
+__device__ __forceinline__ int seq_of_length_rank(const int32_t *cu, int n_seqs, int rank,
+                                                  int *s_cu) {
+  if (n_seqs > kMaxRanked) return rank;
+  for (int x = threadIdx.x; x <= n_seqs; x += blockDim.x) s_cu[x] = cu[x];
+  if (threadIdx.x == 0) s_cu[n_seqs + 1] = rank;   // (the ranks are a permutation: replaced)
+  __syncthreads();
+  for (int sq = threadIdx.x; sq < n_seqs; sq += blockDim.x) {
+    const long len = (long)s_cu[sq + 1] - s_cu[sq];
+    int r = 0;
+    for (int x = 0; x < n_seqs; ++x) {
+      const long lx = (long)s_cu[x + 1] - s_cu[x];
+      r += (lx > len) || (lx == len && x < sq);
+    }
+    if (r == rank) s_cu[n_seqs + 1] = sq;
+  }
+  __syncthreads();
+  const int sel = s_cu[n_seqs + 1];
+  __syncthreads();   // the scratch is reused afterwards
+  return sel;
+}
+
 template <typename TOut, int SG>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -250,7 +277,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = p.H;
-  const int unit = blockIdx.x, n = unit / H, h = unit % H;
+  const int unit = blockIdx.x, h = unit % H;
+  // CTAs start in blockIdx order: in a packed batch the longest sequences go first, so that
+  // the units with the longest serial chunk walk do not start last (ranking in the staging
+  // buffer, which no load has reached yet)
+  const int n = p.cu ? seq_of_length_rank(p.cu, p.n_seqs, unit / H, reinterpret_cast<int *>(sStg))
+                     : unit / H;
   long t0, t1, bofs;
   if (p.cu) {
     t0 = p.cu[n];
