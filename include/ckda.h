@@ -110,6 +110,41 @@ size_t ckda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int ch
                                      int n_seqs);
 
 /*
+ * Chunkwise backward of ckda_chunk_fwd: the gradients of
+ *   L = sum dO . o + sum dS_T . S_T
+ * with respect to q, k, v, the gate logits a, the strength logits b and S0.
+ * The CKDA review measures its kernels forward plus backward ("Experimental
+ * results", Figure 5: CKDA at 96-97 % of KDA's throughput); it gives no
+ * backward formulas, so this is the chain rule of the forward above (the
+ * chunkwise UT form walked in reverse), exact fp32 arithmetic on CUDA cores,
+ * including exact zero gates (an exact zero gate's gradient is the derivative
+ * of L at that gate, which L, affine in each gate, has everywhere).
+ *
+ *   q, k, v, a, b, S0, cu_seqlens, n_seqs, B, T, H, dk, dv, signed_gate,
+ *   io_dtype : as ckda_chunk_fwd (the chunk size is the library's own).
+ *   dO    : [B, T, H, dv] in do_dtype (CKDA_F32 or CKDA_BF16); NULL = zero.
+ *   dS_T  : [N, H, dk, dv] float32; NULL = zero.
+ *   dq, dk_out, da : [B, T, H, dk] float32     dv_out : [B, T, H, dv] float32
+ *   db    : [B, T, H] float32                   (all required, every row written)
+ *   dS0   : [N, H, dk, dv] float32, or NULL (not written)
+ *   workspace : device scratch of ckda_chunk_bwd_workspace_size() bytes (it holds
+ *            the state and the state gradient at every chunk boundary), 256-byte
+ *            aligned, owned by the caller; its status word is read with
+ *            ckda_workspace_status (bad cu_seqlens: the sequence's gradients are
+ *            not written).
+ * Returns CKDA_OK or a negative CKDA_ERR_* code; arguments are checked as by
+ * ckda_chunk_fwd (B * T <= 2^31 - 1, 16-byte alignment of every tensor).
+ */
+int ckda_chunk_bwd(const void *q, const void *k, const void *v, const void *a, const float *b,
+                   const float *S0, const int32_t *cu_seqlens, int n_seqs, int B, int T, int H,
+                   int dk, int dv, int signed_gate, int io_dtype, const void *dO, int do_dtype,
+                   const float *dS_T, float *dq, float *dk_out, float *dv_out, float *da,
+                   float *db, float *dS0, void *workspace, size_t workspace_bytes, void *stream);
+
+/* Bytes of workspace ckda_chunk_bwd needs (host arithmetic, no CUDA call). */
+size_t ckda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int n_seqs);
+
+/*
  * One recurrent decode step for B x H heads: the recurrence above for a
  * single token, applied to the state in place.  The CKDA review notes the
  * extended ranges add no per-token inference cost (section "Research

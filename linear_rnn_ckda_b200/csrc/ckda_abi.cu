@@ -123,8 +123,52 @@ int ckda_chunk_fwd(const void *q, const void *k, const void *v, const void *a, c
   g.workspace_bytes = workspace_bytes;
   g.inject_chunk = g_inject_chunk.load(std::memory_order_relaxed);
   g.inject_wait_ns = g_inject_wait_ns.load(std::memory_order_relaxed);
+  g.S_chunks = nullptr;
   if (ckda::chunk_tc_supported(g)) return ckda::launch_chunk_tc(g, s);
   return ckda::launch_chunk_simt(g, s);
+}
+
+size_t ckda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int n_seqs) {
+  if (B < 0 || T < 0 || H <= 0 || dk <= 0 || dv <= 0 || n_seqs < 0) return ckda::kWorkspaceHeader;
+  const bool packed = n_seqs > 0;
+  const long slots = ckda::chunk_slots(packed, packed ? 1 : B, (long)(packed ? T : T),
+                                       packed ? n_seqs : B, ckda::bwd_chunk_rows());
+  return ckda::kWorkspaceHeader + 2 * (size_t)slots * H * dk * dv * sizeof(float);
+}
+
+int ckda_chunk_bwd(const void *q, const void *k, const void *v, const void *a, const float *b,
+                   const float *S0, const int32_t *cu_seqlens, int n_seqs, int B, int T, int H,
+                   int dk, int dv, int signed_gate, int io_dtype, const void *dO, int do_dtype,
+                   const float *dS_T, float *dq, float *dk_out, float *dv_out, float *da,
+                   float *db, float *dS0, void *workspace, size_t workspace_bytes, void *stream) {
+  const int arg_rc = ckda::check_chunk_args(q, k, v, a, b, S0, cu_seqlens, n_seqs, B, T, H, dk, dv,
+                                            16, signed_gate, io_dtype, CKDA_F32, nullptr, nullptr);
+  if (arg_rc != CKDA_OK) return arg_rc;
+  if (!dq || !dk_out || !dv_out || !da || !db) return CKDA_ERR_NULL;
+  if (do_dtype != CKDA_F32 && do_dtype != CKDA_BF16) return CKDA_ERR_DTYPE;
+  if (!aligned16(dO) || !aligned16(dS_T) || !aligned16(dq) || !aligned16(dk_out) ||
+      !aligned16(dv_out) || !aligned16(da) || !aligned(db, 4) || !aligned16(dS0))
+    return CKDA_ERR_ALIGN;
+  const int N = cu_seqlens ? n_seqs : B;
+  const size_t need = ckda_chunk_bwd_workspace_size(B, T, H, dk, dv, cu_seqlens ? n_seqs : 0);
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return CKDA_ERR_WORKSPACE;
+  const int dev_rc = check_device();
+  if (dev_rc != CKDA_OK) return dev_rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(workspace, 0, ckda::kWorkspaceHeader, s) != cudaSuccess) return CKDA_ERR_CUDA;
+  const long slots = ckda::chunk_slots(cu_seqlens != nullptr, cu_seqlens ? 1 : B, T, N,
+                                       ckda::bwd_chunk_rows());
+  float *base = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + ckda::kWorkspaceHeader);
+  ckda::BwdArgs g;
+  g.q = q; g.k = k; g.v = v; g.a = a; g.b = b; g.S0 = S0; g.dS_T = dS_T; g.cu_seqlens = cu_seqlens;
+  g.dO = dO; g.gq = dq; g.gk = dk_out; g.gv = dv_out; g.ga = da; g.gb = db; g.gS0 = dS0;
+  g.S_chunks = base;
+  g.dS_chunks = base + (size_t)slots * H * dk * dv;
+  g.status = static_cast<int *>(workspace);
+  g.n_seqs = N; g.B = B; g.T = T; g.H = H; g.dk = dk; g.dv = dv; g.signed_gate = signed_gate;
+  g.io_dtype = io_dtype; g.do_dtype = do_dtype; g.n_slots = slots;
+  return ckda::launch_chunk_bwd(g, s);
 }
 
 int ckda_decode_step(const void *q, const void *k, const void *v, const void *a, const float *b,

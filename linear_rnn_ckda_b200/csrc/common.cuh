@@ -83,6 +83,23 @@ __device__ __forceinline__ void gate_log2(float a, int signed_gate, float &log2a
   }
 }
 
+// Derivatives of the activations with respect to their logits (backward):
+// d sigma(x) / dx = sigma(x) sigma(-x) = e^{-|x|} / (1 + e^{-|x|})^2 (0 at +-inf), doubled for
+// 2 sigma - 1 and 2 sigma, 1 for raw values.
+__device__ __forceinline__ float dsigmoid(float x) {
+  const float e = expf(-fabsf(x));
+  const float d = 1.0f + e;
+  return e / (d * d);
+}
+__device__ __forceinline__ float dalpha_da(float a, int signed_gate) {
+  const int f = alpha_form(signed_gate);
+  return f == 2 ? 1.0f : (f == 1 ? 2.0f : 1.0f) * dsigmoid(a);
+}
+__device__ __forceinline__ float dbeta_db(float b, int signed_gate) {
+  const int f = beta_form(signed_gate);
+  return f == 2 ? 1.0f : (f == 1 ? 2.0f : 1.0f) * dsigmoid(b);
+}
+
 // Records the first device-detected error in the workspace status word.
 __device__ __forceinline__ void set_status(int *status, int code) {
   if (status) atomicCAS(status, 0, code);

@@ -23,6 +23,9 @@ struct ChunkArgs {
   // tensor-core kernel waits on a barrier nothing arrives on (-1: off), and that wait's bound
   int inject_chunk;
   unsigned long long inject_wait_ns;
+  // backward only: the exact kernel saves every chunk's incoming state here,
+  // [slot][H][dk][dv] with slot = chunk_slot_base(sequence) + chunk index (NULL: not saved)
+  float *S_chunks;
 };
 
 struct DecodeArgs {
@@ -46,6 +49,32 @@ int launch_chunk_simt(const ChunkArgs &args, cudaStream_t stream);
 // Tensor-core chunkwise forward (tcgen05, dk = dv = 128, chunk 64, bf16 io).
 bool chunk_tc_supported(const ChunkArgs &args);
 int launch_chunk_tc(const ChunkArgs &args, cudaStream_t stream);
+
+// First chunk slot of sequence n when chunks of C tokens of every sequence are numbered in one
+// array (the backward's saved states): cu[n] / C + n for a packed batch (consecutive sequences
+// never overlap: the next base is at least ceil(len / C) further), n * ceil(T / C) otherwise.
+__host__ __device__ __forceinline__ long chunk_slot_base(const int32_t *cu, int n, long T, int C) {
+  return cu ? (long)cu[n] / C + n : (long)n * ((T + C - 1) / C);
+}
+// Number of chunk slots per head: an upper bound of the last base plus its chunks.
+__host__ __device__ __forceinline__ long chunk_slots(bool packed, int B, long T, int N, int C) {
+  return packed ? T / C + N + 1 : (long)B * ((T + C - 1) / C);
+}
+
+// Chunkwise backward (exact fp32, CUDA cores): gradients of sum dO . o + sum dS_T . S_T.
+struct BwdArgs {
+  const void *q, *k, *v, *a;
+  const float *b, *S0, *dS_T;
+  const int32_t *cu_seqlens;
+  const void *dO;             // may be NULL (zero)
+  float *gq, *gk, *gv, *ga, *gb, *gS0;   // gS0 may be NULL
+  float *S_chunks, *dS_chunks;           // workspace: [n_slots][H][dk][dv] each
+  int *status;
+  int n_seqs, B, T, H, dk, dv, signed_gate, io_dtype, do_dtype;
+  long n_slots;
+};
+int launch_chunk_bwd(const BwdArgs &args, cudaStream_t stream);
+int bwd_chunk_rows();   // the backward's chunk size (its saved states are every this many rows)
 
 // One decode step.  Returns a CKDA_* code.
 int launch_decode(const DecodeArgs &args, cudaStream_t stream);

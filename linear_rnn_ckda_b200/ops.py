@@ -32,6 +32,10 @@ SIGNATURES = {
                             _i, _i, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
     "ckda_chunk_fwd_workspace_size": (ctypes.c_size_t, [_i, _i, _i, _i, _i, _i, _i]),
     "ckda_decode_step": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp]),
+    "ckda_chunk_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i,
+                            _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t,
+                            _vp]),
+    "ckda_chunk_bwd_workspace_size": (ctypes.c_size_t, [_i, _i, _i, _i, _i, _i]),
     "ckda_chunk_fwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
                                     _i, _i, _i, _vp, _vp, _vp]),
     "ckda_workspace_status": (_i, [_vp, ctypes.POINTER(_i), _vp]),
@@ -195,6 +199,54 @@ def chunk_fwd(q, k, v, a, b, S0=None, cu_seqlens=None, chunk: int = 64, signed_g
     if rc != 0:
         raise CkdaError("ckda_chunk_fwd", rc)
     return (o if want_o else None), (S_T if want_state else None)
+
+
+def bwd_workspace_size(B, T, H, dk, dv, n_seqs=0) -> int:
+    return int(load().ckda_chunk_bwd_workspace_size(B, T, H, dk, dv, n_seqs))
+
+
+def chunk_bwd(q, k, v, a, b, S0=None, cu_seqlens=None, dO=None, dS_T=None,
+              signed_gate: int = 1, want_dS0: bool = True, workspace=None, grads=None):
+    """Backward of ``chunk_fwd``: gradients of sum(dO * o) + sum(dS_T * S_T).
+
+    Returns (dq, dk, dv, da, db, dS0) as float32 tensors with the shapes of q, k, v, a, b and
+    S0's [N,H,dk,dv] (dS0 None when not wanted).  dO: [B,T,H,dv] float32 or bfloat16, or None
+    (zero); dS_T: [N,H,dk,dv] float32 or None (zero).  ``grads`` may supply the six output
+    tensors."""
+    lib = load()
+    N, dv = check_prefill_args(q, k, v, a, b, S0, cu_seqlens)
+    B, T, H, dk = q.shape
+    dev = q.device
+    _need(dO is None or (dO.shape == (B, T, H, dv) and dO.dtype in _DT),
+          f"dO must be [B,T,H,dv] = {(B, T, H, dv)} float32 or bfloat16")
+    _need(dS_T is None or (dS_T.shape == (N, H, dk, dv) and dS_T.dtype == torch.float32),
+          f"dS_T must be [N,H,dk,dv] = {(N, H, dk, dv)} float32")
+    _same_device(q, dO=dO, dS_T=dS_T)
+    if grads is None:
+        f32 = dict(dtype=torch.float32, device=dev)
+        grads = (torch.empty((B, T, H, dk), **f32), torch.empty((B, T, H, dk), **f32),
+                 torch.empty((B, T, H, dv), **f32), torch.empty((B, T, H, dk), **f32),
+                 torch.empty((B, T, H), **f32),
+                 torch.empty((N, H, dk, dv), **f32) if want_dS0 else None)
+    gq, gk, gv, ga, gb, gS0 = grads
+    for name, t, shape in (("dq", gq, (B, T, H, dk)), ("dk", gk, (B, T, H, dk)),
+                           ("dv", gv, (B, T, H, dv)), ("da", ga, (B, T, H, dk)),
+                           ("db", gb, (B, T, H)), ("dS0", gS0, (N, H, dk, dv))):
+        _need(t is None or (tuple(t.shape) == shape and t.dtype == torch.float32),
+              f"{name} must be {shape} float32")
+    _need(gS0 is not None or not want_dS0, "dS0 buffer missing")
+    n = bwd_workspace_size(B, T, H, dk, dv, N if cu_seqlens is not None else 0)
+    if workspace is None:
+        workspace = torch.empty(max(n, 256), dtype=torch.uint8, device=dev)
+    rc = lib.ckda_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(S0), _ptr(cu_seqlens),
+                            N if cu_seqlens is not None else 0, B, T, H, dk, dv, signed_gate,
+                            _DT[q.dtype], _ptr(dO), _DT[dO.dtype] if dO is not None else CKDA_F32,
+                            _ptr(dS_T), _ptr(gq), _ptr(gk), _ptr(gv), _ptr(ga), _ptr(gb),
+                            _ptr(gS0), _ptr(workspace),
+                            workspace.numel() * workspace.element_size(), _stream(dev))
+    if rc != 0:
+        raise CkdaError("ckda_chunk_bwd", rc)
+    return gq, gk, gv, ga, gb, gS0
 
 
 def decode_step(q, k, v, a, b, S, signed_gate: int = 1, o_dtype=None, o=None, want_o=True):

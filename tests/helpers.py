@@ -155,3 +155,44 @@ def compare_prefill_whole(o, S, inp: dict, signed_gate: int, tol: float, bf16_ou
             es, _ = assert_close(f64(S[n:n + 1, h0:h1]), rS, tol, "S_T " + tag)
             worst[1] = max(worst[1], es)
     return tuple(worst)
+
+
+GRAD_NAMES = ("dq", "dk", "dv", "da", "db", "dS0")
+
+
+def compare_bwd_whole(grads, inp: dict, dO, dS_T, signed_gate: int, tol: float,
+                      block: int = 1 << 18, threads: int = 0):
+    """Whole-tensor parity of the backward's six gradients (host or device tensors) against
+    the oracle's backward on the same inputs, sequence by sequence and in head blocks of at
+    most ``block`` token-heads (host memory stays bounded).  assert_close's bars hold on
+    every block.  Returns the worst block's global error per gradient."""
+    q, k, v, a, b = (inp[x] for x in "qkvab")
+    S0 = inp.get("S0")
+    H = q.shape[2]
+    grads = [None if g is None else g.detach().cpu() for g in grads]
+    dO = None if dO is None else dO.detach().cpu()
+    dS_T = None if dS_T is None else dS_T.detach().cpu()
+    worst = dict.fromkeys(GRAD_NAMES, 0.0)
+    for (n, row, t0, t1) in _segments(inp):
+        L = t1 - t0
+        hb = max(1, min(H, block // max(L, 1)))
+        for h0 in range(0, H, hb):
+            h1 = min(H, h0 + hb)
+            sl = (slice(row, row + 1), slice(t0, t1), slice(h0, h1))
+            ss = (slice(n, n + 1), slice(h0, h1))
+            ref = oracle.ckda_bwd(f64(q[sl]), f64(k[sl]), f64(v[sl]), f64(a[sl]), f64(b[sl]),
+                                  None if S0 is None else f64(S0[ss]),
+                                  dO=None if dO is None else f64(dO[sl]),
+                                  dS_T=None if dS_T is None else f64(dS_T[ss]),
+                                  signed_gate=signed_gate, threads=threads)
+            tag = f"seq {n} heads {h0}..{h1 - 1}"
+            for i, name in enumerate(GRAD_NAMES):
+                g = grads[i]
+                if g is None:
+                    continue
+                got = f64(g[ss]) if name == "dS0" else f64(g[sl])
+                if got.size == 0:
+                    continue
+                e, _ = assert_close(got, ref[i], tol, f"{name} {tag}")
+                worst[name] = max(worst[name], e)
+    return worst

@@ -218,3 +218,30 @@ def test_decode_binding_rejects_mismatched_buffers(name, over):
     args.update(over(d))
     with pytest.raises(ValueError):
         ops.check_decode_args(**args)
+
+
+def _bwd(lib, **kw):
+    args = dict(q=P, k=P, v=P, a=P, b=P, S0=None, cu=None, n_seqs=0, B=1, T=8, H=1, dk=16, dv=16,
+                sg=1, io=0, dO=P, do_dt=0, dS_T=None, dq=P, dk_=P, dv_=P, da=P, db=P, dS0=None,
+                ws=P, wsb=1 << 30, stream=None)
+    args.update(kw)
+    return lib.ckda_chunk_bwd(*args.values())
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), -1), (dict(dq=None), -1), (dict(db=None), -1), (dict(da=None), -1),
+    (dict(dk=24), -2), (dict(H=0), -2), (dict(B=2, T=1 << 30), -2),
+    (dict(sg=7), -4), (dict(do_dt=3), -4), (dict(io=2), -4),
+    (dict(dq=MIS), -5), (dict(dO=MIS), -5), (dict(dS_T=MIS), -5), (dict(db=ODD), -5),
+    (dict(ws=None), -7), (dict(wsb=256), -7),
+])
+def test_chunk_bwd_rejects(lib, kw, code):
+    assert _bwd(lib, **kw) == code
+
+
+def test_bwd_workspace_size(lib):
+    """Two fp32 [slots][H][dk][dv] arrays (the state and its gradient at every 32-row chunk)
+    plus the 256-byte header; a packed batch allows one extra slot per sequence."""
+    per = 128 * 128 * 4 * 16
+    assert lib.ckda_chunk_bwd_workspace_size(4, 4096, 16, 128, 128, 0) == 256 + 2 * 512 * per
+    assert lib.ckda_chunk_bwd_workspace_size(1, 4096, 16, 128, 128, 3) == 256 + 2 * (128 + 4) * per
