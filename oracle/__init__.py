@@ -5,8 +5,8 @@ and the CPU-baseline leg of ``bench.py``; never by the CUDA library or its
 Python binding.  Every function is pinned by ``tests/pins.py`` against closed
 forms and invariants of the method (run by ``tests/test_oracle_pins.py``).
 """
-from .oracle import (SOURCE, Oracle, build, ckda_bwd, ckda_fwd, ckda_fwd_explicit, compile_c,
-                     decode_step, default, gates, transition)
+from .oracle import (SOURCE, Oracle, build, ckda_bwd, ckda_fwd, ckda_fwd_explicit,
+                     ckda_fwd_product, compile_c, decode_step, default, gates, transition)
 
-__all__ = ["SOURCE", "Oracle", "build", "ckda_bwd", "ckda_fwd", "ckda_fwd_explicit", "compile_c",
-           "decode_step", "default", "gates", "transition"]
+__all__ = ["SOURCE", "Oracle", "build", "ckda_bwd", "ckda_fwd", "ckda_fwd_explicit",
+           "ckda_fwd_product", "compile_c", "decode_step", "default", "gates", "transition"]

@@ -555,3 +555,78 @@ int oracle_ckda_fwd_explicit(const double *q, const double *k, const double *v,
     free(A); free(S); free(N); free(alpha);
     return ORACLE_OK;
 }
+
+/*
+ * DeltaProduct form: nh rank-one delta-rule updates per token, the gate applied once.
+ * The CKDA review names DeltaProduct2 (two rank-one updates per token, "one more value
+ * path") as the other route to plane rotations, with throughput comparable to KDA's
+ * (sections "Research motivation" and "Experimental results" (5)); per token t:
+ *
+ *   S <- Diag(alpha_t) S
+ *   for j = 1 .. nh:  S <- S + beta_tj k_tj (v_tj - S^T k_tj)^T
+ *   o_t = S^T q_t
+ *
+ * i.e. S_t = (I - b_t2 k_t2 k_t2^T)(I - b_t1 k_t1 k_t1^T) Diag(alpha_t) S_{t-1} + writes.
+ * Gate and strength forms as oracle_ckda_fwd (signed_gate 0..4).
+ * Layouts: q, a [B,T,H,dk]; k [B,T,nh,H,dk]; v [B,T,nh,H,dv]; b [B,T,nh,H];
+ * o [B,T,H,dv] (or NULL); S0, S_T [N,H,dk,dv].  One thread, unit after unit.
+ */
+int oracle_ckda_fwd_product(const double *q, const double *k, const double *v, const double *a,
+                            const double *b, const double *S0, const int32_t *cu_seqlens,
+                            int n_seqs, int B, int T, int H, int dk, int dv, int nh,
+                            int signed_gate, double *o, double *S_T) {
+    if (!q || !k || !v || !a || !b || !S_T) return ORACLE_ERR_ARG;
+    if (B < 0 || T < 0 || H <= 0 || dk <= 0 || dv <= 0 || nh < 1) return ORACLE_ERR_ARG;
+    if (signed_gate < 0 || signed_gate > 4) return ORACLE_ERR_ARG;
+    int N = B;
+    if (cu_seqlens) {
+        if (B != 1 || n_seqs < 0) return ORACLE_ERR_ARG;
+        if (cu_seqlens[0] != 0 || cu_seqlens[n_seqs] != T) return ORACLE_ERR_SEQLENS;
+        for (int i = 0; i < n_seqs; ++i)
+            if (cu_seqlens[i + 1] < cu_seqlens[i]) return ORACLE_ERR_SEQLENS;
+        N = n_seqs;
+    }
+    double *S = (double *)malloc(sizeof(double) * (size_t)dk * dv);
+    double *alpha = (double *)malloc(sizeof(double) * (size_t)dk);
+    double *pr = (double *)malloc(sizeof(double) * (size_t)dv);
+    if (!S || !alpha || !pr) { free(S); free(alpha); free(pr); return ORACLE_ERR_NOMEM; }
+    for (int n = 0; n < N; ++n) {
+        const long t0 = cu_seqlens ? cu_seqlens[n] : 0, t1 = cu_seqlens ? cu_seqlens[n + 1] : T;
+        const long tok0 = cu_seqlens ? 0 : (long)n * T;  /* token row of t = 0 */
+        for (int h = 0; h < H; ++h) {
+            const size_t sofs = ((size_t)n * H + h) * (size_t)dk * dv;
+            for (size_t e = 0; e < (size_t)dk * dv; ++e) S[e] = S0 ? S0[sofs + e] : 0.0;
+            for (long t = t0; t < t1; ++t) {
+                const size_t row = (size_t)(tok0 + t) * H + h;
+                double unused;
+                gate_values(a + row * dk, 0.0, dk, signed_gate, alpha, &unused);
+                for (int i = 0; i < dk; ++i)
+                    for (int c = 0; c < dv; ++c) S[(size_t)i * dv + c] *= alpha[i];
+                for (int j = 0; j < nh; ++j) {
+                    /* key, value and strength j of token t */
+                    const size_t sub = ((size_t)(tok0 + t) * nh + j) * H + h;
+                    const double *kj = k + sub * dk, *vj = v + sub * dv;
+                    double bj;
+                    gate_values(NULL, b[sub], 0, signed_gate, &unused, &bj);
+                    for (int c = 0; c < dv; ++c) {
+                        double acc = 0.0;
+                        for (int i = 0; i < dk; ++i) acc += kj[i] * S[(size_t)i * dv + c];
+                        pr[c] = acc;
+                    }
+                    for (int i = 0; i < dk; ++i)
+                        for (int c = 0; c < dv; ++c)
+                            S[(size_t)i * dv + c] += bj * kj[i] * (vj[c] - pr[c]);
+                }
+                if (o)
+                    for (int c = 0; c < dv; ++c) {
+                        double acc = 0.0;
+                        for (int i = 0; i < dk; ++i) acc += q[row * dk + i] * S[(size_t)i * dv + c];
+                        o[row * dv + c] = acc;
+                    }
+            }
+            memcpy(S_T + sofs, S, sizeof(double) * (size_t)dk * dv);
+        }
+    }
+    free(S); free(alpha); free(pr);
+    return ORACLE_OK;
+}

@@ -71,6 +71,9 @@ class Oracle:
         lib.oracle_ckda_fwd_explicit.restype = _i
         lib.oracle_ckda_fwd_explicit.argtypes = [_dp, _dp, _dp, _dp, _dp, _dp,
                                                  _i, _i, _i, _i, _dp, _dp]
+        lib.oracle_ckda_fwd_product.restype = _i
+        lib.oracle_ckda_fwd_product.argtypes = [_dp, _dp, _dp, _dp, _dp, _dp, _ip,
+                                                _i, _i, _i, _i, _i, _i, _i, _i, _dp, _dp]
         lib.oracle_gates.restype = None
         lib.oracle_gates.argtypes = [_dp, _dp, _i, _i, _i, _dp, _dp]
         self.lib = lib
@@ -137,6 +140,29 @@ class Oracle:
             raise ValueError(f"oracle_ckda_bwd failed with code {rc}")
         return gq, gk, gv, ga, gb, gS0
 
+    def ckda_fwd_product(self, q, k, v, a, b, S0=None, cu_seqlens=None, signed_gate: int = 1):
+        """DeltaProduct forward (nh rank-one updates per token, the gate once).
+
+        q, a: [B,T,H,dk]; k: [B,T,nh,H,dk]; v: [B,T,nh,H,dv]; b: [B,T,nh,H]; S0: [N,H,dk,dv]
+        or None.  Returns (o [B,T,H,dv], S_T [N,H,dk,dv])."""
+        q, k, v, a, b = (_f64(x) for x in (q, k, v, a, b))
+        B, T, H, dk = q.shape
+        nh, dv = k.shape[2], v.shape[-1]
+        cu_p, N = None, B
+        if cu_seqlens is not None:
+            cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+            N = cu.size - 1
+            cu_p = cu.ctypes.data_as(_ip)
+        S0 = None if S0 is None else _f64(S0)
+        o = np.empty((B, T, H, dv))
+        S_T = np.empty((N, H, dk, dv))
+        rc = self.lib.oracle_ckda_fwd_product(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b),
+                                              _ptr(S0), cu_p, N, B, T, H, dk, dv, nh,
+                                              int(signed_gate), _ptr(o), _ptr(S_T))
+        if rc != 0:
+            raise ValueError(f"oracle_ckda_fwd_product failed with code {rc}")
+        return o, S_T
+
     def decode_step(self, q, k, v, a, b, S, signed_gate: int = 1):
         """One decode step.  Returns (o [B,H,dv], S_new [B,H,dk,dv]); S is not modified."""
         q, k, v, a, b = (_f64(x) for x in (q, k, v, a, b))
@@ -201,6 +227,10 @@ def ckda_bwd(*a, **kw):
 
 def decode_step(*a, **kw):
     return default().decode_step(*a, **kw)
+
+
+def ckda_fwd_product(*a, **kw):
+    return default().ckda_fwd_product(*a, **kw)
 
 
 def transition(*a, **kw):

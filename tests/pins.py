@@ -19,6 +19,9 @@ on a mismatch, so the same checks run on the real oracle
   [FIG5]  same page, Figure 5 (the kernels are measured forward plus backward; the pages give
           no backward formulas, so the backward oracle is pinned by calculus alone: finite
           differences, Euler identities of the linear arguments, closed forms)
+  [DP2]   same page, "Research motivation" and "Experimental results" (5): DeltaProduct2 reaches
+          plane rotations with two rank-one delta-rule updates per token (one more key and
+          value), the composition of two Householder reflections
 """
 from __future__ import annotations
 
@@ -604,6 +607,97 @@ def pin_bwd_linear_attention(orc):
         assert np.allclose(da[j], want_a, rtol=1e-12, atol=1e-12)
     want = sum(M(0, t) @ np.outer(q[t], dO[t]) for t in range(T)) + M(0, T - 1) @ dS_T
     assert _rel(dS0, want) < 1e-12
+
+
+# ---------------------------------------------------------------- DeltaProduct form [DP2]
+
+
+def _product(orc, q, k, v, alpha, beta, S0, signed_gate=2):
+    """oracle.ckda_fwd_product on one sequence and head: q, alpha [T,dk]; k [T,nh,dk];
+    v [T,nh,dv]; beta [T,nh]."""
+    T, dk = q.shape
+    nh, dv = k.shape[1], v.shape[2]
+    o, S = orc.ckda_fwd_product(q.reshape(1, T, 1, dk), k.reshape(1, T, nh, 1, dk),
+                                v.reshape(1, T, nh, 1, dv), alpha.reshape(1, T, 1, dk),
+                                np.asarray(beta, float).reshape(1, T, nh, 1),
+                                None if S0 is None else S0.reshape(1, 1, dk, dv),
+                                signed_gate=signed_gate)
+    return o.reshape(T, dv), S.reshape(dk, dv)
+
+
+def pin_product_one_update(orc):
+    """[DP2] One update per token is the gated delta rule itself, in every gate form."""
+    rng = np.random.default_rng(40)
+    T, dk, dv = 23, 5, 4
+    q, k, v = rng.standard_normal((T, dk)), _unit(rng, T, dk), rng.standard_normal((T, dv))
+    S0 = rng.standard_normal((dk, dv))
+    for sg in range(5):
+        a = rng.standard_normal((T, dk)) if sg != 2 else rng.uniform(-1, 1, (T, dk))
+        b = rng.standard_normal(T) if sg != 2 else rng.uniform(0, 2, T)
+        o1, S1 = _one(orc, q, k, v, a, b, S0, signed_gate=sg)
+        o2, S2 = _product(orc, q, k[:, None], v[:, None], a, b[:, None], S0, signed_gate=sg)
+        assert np.allclose(o1, o2, atol=1e-13) and np.allclose(S1, S2, atol=1e-13)
+
+
+def pin_product_zero_second_strength(orc):
+    """[DP2] With the second strength 0 the second update is the identity: the result is the
+    one-update recurrence on the first key, value and strength."""
+    rng = np.random.default_rng(41)
+    T, dk, dv = 19, 6, 3
+    q, k, v = rng.standard_normal((T, dk)), _unit(rng, T, 2, dk), rng.standard_normal((T, 2, dv))
+    alpha, beta = rng.uniform(-1, 1, (T, dk)), rng.uniform(0, 2, (T, 2))
+    beta[:, 1] = 0.0
+    S0 = rng.standard_normal((dk, dv))
+    o1, S1 = _one(orc, q, k[:, 0], v[:, 0], alpha, beta[:, 0], S0)
+    o2, S2 = _product(orc, q, k, v, alpha, beta, S0)
+    assert np.allclose(o1, o2, atol=1e-13) and np.allclose(S1, S2, atol=1e-13)
+
+
+def pin_product_idempotent_projection(orc):
+    """[DP2][HH] beta = 1 with a unit key is a projection: repeating the same key and value
+    changes nothing (P (P S + k v^T) + k v^T = P S + k v^T, since P k = 0)."""
+    rng = np.random.default_rng(42)
+    T, dk, dv = 15, 5, 4
+    q, k1, v1 = rng.standard_normal((T, dk)), _unit(rng, T, dk), rng.standard_normal((T, dv))
+    alpha = rng.uniform(-1, 1, (T, dk))
+    S0 = rng.standard_normal((dk, dv))
+    o1, S1 = _one(orc, q, k1, v1, alpha, np.ones(T), S0)
+    o2, S2 = _product(orc, q, np.stack([k1, k1], 1), np.stack([v1, v1], 1), alpha,
+                      np.ones((T, 2)), S0)
+    assert np.allclose(o1, o2, atol=1e-12) and np.allclose(S1, S2, atol=1e-12)
+
+
+def pin_product_rotation(orc):
+    """[DP2][HH] Two reflections (beta = 2) with unit keys at angles t1, t2 and no decay make
+    the rotation R(2 (t2 - t1)); over tokens the angles add."""
+    rng = np.random.default_rng(43)
+    T = 9
+    t1, t2 = rng.uniform(0, 2 * np.pi, T), rng.uniform(0, 2 * np.pi, T)
+    k = np.stack([np.stack([np.cos(t1), np.sin(t1)], 1), np.stack([np.cos(t2), np.sin(t2)], 1)], 1)
+    _, S = _product(orc, rng.standard_normal((T, 2)), k, np.zeros((T, 2, 2)), np.ones((T, 2)),
+                    np.full((T, 2), 2.0), np.eye(2))
+    assert np.allclose(S, _rot(2 * (t2 - t1).sum()), atol=1e-12)
+    _, S1 = _product(orc, np.zeros((1, 2)), k[:1], np.zeros((1, 2, 2)), np.ones((1, 2)),
+                     np.full((1, 2), 2.0), np.eye(2))
+    assert np.allclose(S1, _rot(2 * (t2[0] - t1[0])), atol=1e-14)
+
+
+def pin_product_explicit_matrices(orc):
+    """[DP2] The product form against explicit dk x dk transitions (oracle.transition, pinned
+    by its own closed forms): S <- T2 (T1 S + b1 k1 v1^T) + b2 k2 v2^T with
+    T1 = (I - b1 k1 k1^T) Diag(alpha), T2 = I - b2 k2 k2^T; o = S^T q."""
+    rng = np.random.default_rng(44)
+    T, dk, dv = 12, 5, 3
+    q, k, v = rng.standard_normal((T, dk)), rng.standard_normal((T, 2, dk)), rng.standard_normal((T, 2, dv))
+    alpha, beta = rng.uniform(-1, 1, (T, dk)), rng.uniform(0, 2, (T, 2))
+    S = rng.standard_normal((dk, dv))
+    o, S_T = _product(orc, q, k, v, alpha, beta, S)
+    for t in range(T):
+        T1 = orc.transition(k[t, 0], alpha[t], beta[t, 0])
+        T2 = orc.transition(k[t, 1], np.ones(dk), beta[t, 1])
+        S = T2 @ (T1 @ S + beta[t, 0] * np.outer(k[t, 0], v[t, 0])) + beta[t, 1] * np.outer(k[t, 1], v[t, 1])
+        assert np.allclose(o[t], S.T @ q[t], atol=1e-12)
+    assert np.allclose(S_T, S, atol=1e-12)
 
 
 ALL_PINS = [v for n, v in sorted(globals().items()) if n.startswith("pin_")]

@@ -43,6 +43,14 @@ MUTANTS = [
      "(af == 1 ? sigmoid_deriv(a[i]) : 1.0)"),
     ("bwd_checkpoint_off_by_one", "memcpy(states, ckpt + (size_t)sg * dd",
      "memcpy(states, ckpt + (size_t)(sg > 0 ? sg - 1 : 0) * dd"),
+    # DeltaProduct form
+    ("product_second_update_skipped", "for (int j = 0; j < nh; ++j) {",
+     "for (int j = 0; j < 1; ++j) {"),
+    ("product_gate_twice", "for (int c = 0; c < dv; ++c) S[(size_t)i * dv + c] *= alpha[i];",
+     "for (int c = 0; c < dv; ++c) S[(size_t)i * dv + c] *= alpha[i] * alpha[i];"),
+    ("product_readout_sign", "o[row * dv + c] = acc;", "o[row * dv + c] = -acc;"),
+    ("product_strength_of_first_update", "gate_values(NULL, b[sub], 0,",
+     "gate_values(NULL, b[((size_t)(tok0 + t) * nh) * H + h], 0,"),
 ]
 
 
