@@ -358,9 +358,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--decode-steps", type=int, default=None,
                     help="timed decode steps (default: --steps rounded up to the 128-step cycle)")
-    ap.add_argument("--legs", default="varlen,e2e,kda,spread,ratio,decode",
+    ap.add_argument("--legs", default="varlen,e2e,kda,spread,ratio,bwd,decode",
                     help="comma list of legs to run (varlen = the headline, e2e, kda, spread, "
-                         "ratio, decode); a profiling run can select one, the default runs all")
+                         "ratio, bwd, decode); a profiling run can select one, the default runs "
+                         "all")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -504,6 +505,42 @@ def main():
             workloads[wk.name]["ckda_mode_ms_per_step"] = ms_c / extra_steps
         del c
 
+    # ------------------------------------------------------------ forward + backward
+    # The pages' kernel measurement is forward plus backward (CKDA at 96-97 % of KDA on H100):
+    # one ckda_chunk_fwd and one ckda_chunk_bwd per step on the KDA workload's shapes and
+    # inputs, in KDA mode and in CKDA mode (the same kernels, signed gates).
+    fwd_bwd = None
+    if "bwd" in legs:
+        wk = KDA
+        c = PrefillCase(ops, wk, synth.make_prefill(wk, seed=rank), dev)
+        g = torch.Generator(device="cpu").manual_seed(1234 + rank)
+        dO = torch.randn(c.o.shape, generator=g).to(device=dev, dtype=torch.bfloat16)
+        bws = torch.empty(ops.bwd_workspace_size(wk.B, wk.T, wk.H, wk.dk, wk.dv, 0),
+                          dtype=torch.uint8, device=dev)
+        f32 = dict(dtype=torch.float32, device=dev)
+        grads = (torch.empty(c.d["q"].shape, **f32), torch.empty(c.d["k"].shape, **f32),
+                 torch.empty(c.d["v"].shape, **f32), torch.empty(c.d["a"].shape, **f32),
+                 torch.empty(c.d["b"].shape, **f32), None)
+        res = {}
+        for mode, sg in (("kda", 0), ("ckda", 1)):
+            def fb():
+                c.sg = sg
+                c()
+                ops.chunk_bwd(c.d["q"], c.d["k"], c.d["v"], c.d["a"], c.d["b"], None, None, dO=dO,
+                              signed_gate=sg, want_dS0=False, workspace=bws, grads=grads)
+
+            ms_fb = max_over_ranks(time_loop(fb, extra_steps, args.warmup, world, stream), world)
+            if ops.workspace_status(bws) != 0:
+                raise RuntimeError("device status after the backward leg")
+            res[mode] = ms_fb / extra_steps
+        c.sg = wk.signed_gate
+        fwd_bwd = {"workload": wk.name, "steps": extra_steps,
+                   "kda_ms_per_step": res["kda"], "ckda_ms_per_step": res["ckda"],
+                   "kda_tokens_per_s": wk.tokens * world / (res["kda"] / 1000.0),
+                   "ckda_over_kda_throughput": res["kda"] / res["ckda"],
+                   "path": "forward: tcgen05 kernel; backward: exact fp32 CUDA-core kernels"}
+        del c, grads, bws, dO
+
     # ------------------------------------------------------------ decode
     wd = DECODE
     dsteps = args.decode_steps or max(args.steps, 128)
@@ -539,7 +576,7 @@ def main():
             "data": "synthetic (seeded; same shapes and distributions as the pages' workloads)",
             "config": headline_config(w),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "workloads": workloads, "decode": decode_obj,
+            "workloads": workloads, "fwd_bwd": fwd_bwd, "decode": decode_obj,
             "gpu_launches": args.steps, "clocks": clocks, "peaks_source": peaks["source"],
         }
         print(json.dumps(line), flush=True)

@@ -23,6 +23,22 @@
  *            (3 and 4: the single-range variants of the CKDA review, "Experimental
  *            results", Figure 6)
  * Logits of +-inf are legal and exact: alpha = 0, +-1 and beta = 0, 1, 2.
+ * Flags, OR-ed into signed_gate:
+ *   CKDA_GATE_PER_HEAD  one gate logit per token and head: a is [B, T, H] ([B, H] for
+ *            decode) and the gate alpha_t = alpha_t * 1 is shared by all key channels, the
+ *            scalar (GDN-style) gate the CKDA review sets against KDA's channel-wise one
+ *            (section "Scalar vs channel-wise gating").
+ *   CKDA_QK_L2NORM      q and k arrive as raw projections and are divided by their L2 norm
+ *            over the key channels inside the kernel (a zero vector stays zero), the fused
+ *            normalisation of the review's Triton path (section "Reproducibility").
+ *   CKDA_DELTA_PRODUCT2 DeltaProduct2, the review's other route to plane rotations (sections
+ *            "Research motivation", "Experimental results" (5)): each token carries two keys,
+ *            values and strengths, k [B, T, 2, H, dk], v [B, T, 2, H, dv], b [B, T, 2, H]
+ *            (decode: [B, 2, H, .]); the gate is applied once, then the two delta-rule updates
+ *            in order, then the read-out:
+ *              S <- Diag(alpha_t) S;  S <- S + beta_tj k_tj (v_tj - S^T k_tj)^T, j = 1, 2;
+ *              o_t = S^T q_t.
+ *            Runs on the exact CUDA-core kernel; not available to ckda_chunk_bwd.
  *
  * Conventions for every entry point:
  *   - All tensor pointers are DEVICE pointers, dense and row-major.  Alignment
@@ -67,6 +83,10 @@ extern "C" {
 #define CKDA_F32 0
 #define CKDA_BF16 1
 
+#define CKDA_GATE_PER_HEAD 16  /* flag: one gate per token and head (a is [B, T, H])  */
+#define CKDA_QK_L2NORM 32      /* flag: q and k are L2-normalised inside the kernel   */
+#define CKDA_DELTA_PRODUCT2 64 /* flag: two rank-one delta updates per token          */
+
 /*
  * Chunkwise (WY / UT-transform) parallel forward, "prefill".
  *
@@ -76,6 +96,7 @@ extern "C" {
  * chunks, and the result equals the token-by-token recurrence.
  *
  *   q, k, a : [B, T, H, dk]  io_dtype       v : [B, T, H, dv]  io_dtype
+ *            (a : [B, T, H] with CKDA_GATE_PER_HEAD)
  *   b       : [B, T, H]      float32        o : [B, T, H, dv]  o_dtype (NULL: not written)
  *   S0      : [N, H, dk, dv] float32, NULL = zero initial state
  *   S_T     : [N, H, dk, dv] float32, NULL = not written; may alias S0
@@ -125,6 +146,8 @@ size_t ckda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int ch
  *   dO    : [B, T, H, dv] in do_dtype (CKDA_F32 or CKDA_BF16); NULL = zero.
  *   dS_T  : [N, H, dk, dv] float32; NULL = zero.
  *   dq, dk_out, da : [B, T, H, dk] float32     dv_out : [B, T, H, dv] float32
+ *            (da : [B, T, H] with CKDA_GATE_PER_HEAD; with CKDA_QK_L2NORM dq and dk_out
+ *            are the gradients with respect to the raw, un-normalised q and k)
  *   db    : [B, T, H] float32                   (all required, every row written)
  *   dS0   : [N, H, dk, dv] float32, or NULL (not written)
  *   workspace : device scratch of ckda_chunk_bwd_workspace_size() bytes (it holds
@@ -151,6 +174,7 @@ size_t ckda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int n_
  * motivation"); the step reads and writes each head's fp32 state once.
  *
  *   q, k, a : [B, H, dk] io_dtype     v : [B, H, dv] io_dtype     b : [B, H] float32
+ *            (a : [B, H] with CKDA_GATE_PER_HEAD)
  *   S       : [B, H, dk, dv] float32, updated in place (S_{t-1} -> S_t)
  *   o       : [B, H, dv] o_dtype, o = S_t^T q (NULL: not written)
  * Returns CKDA_OK or a negative CKDA_ERR_* code.

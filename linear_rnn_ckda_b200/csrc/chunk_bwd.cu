@@ -81,9 +81,12 @@ __device__ __forceinline__ bool seq_range(const BwdParams &p, int n, long &t0, l
 //   sL     [kBC][ldk]: L_r = sum of log2|alpha| over the non-zero gates of rows 0..r
 //   sZ     [kBC][ldz]: (zero count << 1) | sign parity of rows 0..r
 //   sBeta  [kBC], sGC [dk] = g (exact), sLC [dk], sZC [dk]
+//   (CKDA_QK_L2NORM: q and k divided by their norms; the factors go to sInvQ / sInvK)
 template <typename TIn>
 __device__ void load_chunk(const BwdParams &p, long row0, int nrows, int h, float *sQ, float *sK,
-                           float *sL, uint8_t *sZ, float *sBeta, float *sGC, float *sLC, int *sZC) {
+                           float *sL, uint8_t *sZ, float *sBeta, float *sGC, float *sLC, int *sZC,
+                           float *sInvQ, float *sInvK) {
+  const bool per_head = per_head_gate(p.signed_gate);
   const int dk = p.dk, ldk = dk + 1, ldz = dk + 4, H = p.H, tid = threadIdx.x;
   const TIn *q = static_cast<const TIn *>(p.q);
   const TIn *k = static_cast<const TIn *>(p.k);
@@ -95,7 +98,7 @@ __device__ void load_chunk(const BwdParams &p, long row0, int nrows, int h, floa
       const size_t row = (size_t)(row0 + r) * H + h;
       qv = to_f32(q[row * dk + c]);
       kv = to_f32(k[row * dk + c]);
-      av = to_f32(a[row * dk + c]);
+      av = to_f32(a[per_head ? row : row * dk + c]);
     }
     sQ[r * ldk + c] = qv;
     sK[r * ldk + c] = kv;
@@ -127,6 +130,10 @@ __device__ void load_chunk(const BwdParams &p, long row0, int nrows, int h, floa
     sGC[c] = zc ? 0.f : (par ? -exp2f(L) : exp2f(L));
   }
   __syncthreads();
+  if (qk_l2norm(p.signed_gate)) {
+    l2norm_rows2(sQ, sK, ldk, nrows, dk, sInvQ, sInvK);
+    __syncthreads();
+  }
 }
 
 // g(t, j)_c from the prefixes (exact: 0 when a zero gate lies in (j, t])
@@ -221,7 +228,8 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_reverse_kernel(BwdParams p) 
   float *sBeta = sdV + kBC * dv;
   float *sGC = sBeta + kBC;
   float *sLC = sGC + dk;
-  int *sZC = reinterpret_cast<int *>(sLC + dk);
+  float *sInv = sLC + dk;                             // [2][kBC] 1 / row norms of q and k
+  int *sZC = reinterpret_cast<int *>(sInv + 2 * kBC);
 
   const int unit = blockIdx.x, n = unit / H, h = unit % H;
   long t0, t1, bofs;
@@ -236,7 +244,8 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_reverse_kernel(BwdParams p) 
     const long cs = t0 + ci * kBC;
     const int nrows = (int)(t1 - cs < kBC ? t1 - cs : kBC);
     __syncthreads();
-    load_chunk<TIn>(p, bofs + cs, nrows, h, sQ, sK, sL, sZ, sBeta, sGC, sLC, sZC);
+    load_chunk<TIn>(p, bofs + cs, nrows, h, sQ, sK, sL, sZ, sBeta, sGC, sLC, sZC, sInv,
+                    sInv + kBC);
     for (int e = tid; e < kBC * dv; e += kBThreads) {
       const int r = e / dv, j = e % dv;
       sdO[e] = (r < nrows && dO) ? to_f32(dO[((size_t)(bofs + cs + r) * H + h) * dv + j]) : 0.f;
@@ -323,7 +332,10 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_grad_kernel(BwdParams p) {
   float *sGC = sdBeta + kBC;
   float *sLC = sGC + dk;
   float *sCarry = sLC + dk;                            // sum_j dS'_cj S_cj
-  int *sZC = reinterpret_cast<int *>(sCarry + dk);
+  float *sInvQ = sCarry + dk;                          // [kBC] 1 / ||q_r|| (CKDA_QK_L2NORM)
+  float *sInvK = sInvQ + kBC;                          // [kBC] 1 / ||k_r||
+  float *sDaRow = sInvK + kBC;                         // [kBC] per-head gate gradient
+  int *sZC = reinterpret_cast<int *>(sDaRow + kBC);
 
   // slot -> (sequence, chunk)
   const long slot = blockIdx.x;
@@ -353,7 +365,9 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_grad_kernel(BwdParams p) {
   const float *S_in = p.S_in + ((size_t)slot * H + h) * dk * dv;
   const float *dSo = p.dS_out + ((size_t)slot * H + h) * dk * dv;
 
-  load_chunk<TIn>(p, row0, nrows, h, sQ, sK, sL, sZ, sBeta, sGC, sLC, sZC);
+  const bool per_head = per_head_gate(p.signed_gate), l2 = qk_l2norm(p.signed_gate);
+  load_chunk<TIn>(p, row0, nrows, h, sQ, sK, sL, sZ, sBeta, sGC, sLC, sZC, sInvQ, sInvK);
+  for (int r = tid; r < kBC; r += kBThreads) sDaRow[r] = 0.f;
   pair_products(dk, sQ, sK, sL, sZ, sM, sP);
   unit_lower_inverse(sM, sBeta, sLi);
   for (int e = tid; e < kBC * dk; e += kBThreads) {
@@ -506,9 +520,36 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_grad_kernel(BwdParams p) {
       if (t > r) w = fmaf(sdM[t * kBC + r], sK[t * ldk + c], w);
       dkv = fmaf(w, f, dkv);
     }
-    const size_t idx = ((size_t)(row0 + r) * H + h) * dk + c;
-    p.gq[idx] = dqv;
-    p.gk[idx] = dkv;
+    if (l2) {   // gradients of the normalised q, k: the chain through the norm follows
+      sKr[r * ldk + c] = dqv;
+      sKd[r * ldk + c] = dkv;
+    } else {
+      const size_t idx = ((size_t)(row0 + r) * H + h) * dk + c;
+      p.gq[idx] = dqv;
+      p.gk[idx] = dkv;
+    }
+  }
+  if (l2) {
+    // x = y / ||y||:  dy = (dx - x (x . dx)) / ||y||   (one warp per row)
+    __syncthreads();
+    const int warp = tid >> 5, lane = tid & 31;
+    for (int r = warp; r < nrows; r += kBThreads / 32) {
+      float dq_dot = 0.f, dk_dot = 0.f;
+      for (int c = lane; c < dk; c += 32) {
+        dq_dot = fmaf(sQ[r * ldk + c], sKr[r * ldk + c], dq_dot);
+        dk_dot = fmaf(sK[r * ldk + c], sKd[r * ldk + c], dk_dot);
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        dq_dot += __shfl_xor_sync(0xffffffffu, dq_dot, off);
+        dk_dot += __shfl_xor_sync(0xffffffffu, dk_dot, off);
+      }
+      for (int c = lane; c < dk; c += 32) {
+        const size_t idx = ((size_t)(row0 + r) * H + h) * dk + c;
+        p.gq[idx] = sInvQ[r] * fmaf(-sQ[r * ldk + c], dq_dot, sKr[r * ldk + c]);
+        p.gk[idx] = sInvK[r] * fmaf(-sK[r * ldk + c], dk_dot, sKd[r * ldk + c]);
+      }
+    }
   }
 
   // ---- gate gradient, one thread per channel.  dL/dalpha_s is the derivative of the gate
@@ -549,8 +590,12 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_grad_kernel(BwdParams p) {
           pairs = fmaf(f, inner[t], pairs);
         }
         const float dalpha = fmaf(Gp, RS[s], fmaf(gd, WS, fmaf(Gp * gd, carry, pairs)));
-        const size_t idx = ((size_t)(row0 + s) * H + h) * dk + c;
-        p.ga[idx] = dalpha * dalpha_da(to_f32(a[idx]), p.signed_gate);
+        if (per_head) {
+          atomicAdd(&sDaRow[s], dalpha);   // one gate shared by every key channel
+        } else {
+          const size_t idx = ((size_t)(row0 + s) * H + h) * dk + c;
+          p.ga[idx] = dalpha * dalpha_da(to_f32(a[idx]), p.signed_gate);
+        }
       }
       // advance WS and inner_t past row s
       const float al = s > 0 ? pair_gate(sL, sZ, ldk, ldz, s, s - 1, c) : prefix_gate(sL, sZ, ldk, ldz, 0, c);
@@ -568,19 +613,20 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_grad_kernel(BwdParams p) {
   for (int r = tid; r < nrows; r += kBThreads) {
     const size_t row = (size_t)(row0 + r) * H + h;
     p.gb[row] = sdBeta[r] * dbeta_db(p.b[row], p.signed_gate);
+    if (per_head) p.ga[row] = sDaRow[r] * dalpha_da(to_f32(a[row]), p.signed_gate);
   }
 }
 
 size_t reverse_smem(int dk, int dv) {
   const int ldk = dk + 1, ldz = dk + 4;
   return sizeof(float) * ((size_t)dk * dv + 3 * kBC * ldk + 3 * kBC * kBC + 3 * kBC * dv + kBC +
-                          2 * dk) +
+                          2 * dk + 2 * kBC) +
          (size_t)kBC * ldz + sizeof(int) * dk + 64;
 }
 size_t grad_smem(int dk) {
   const int ldk = dk + 1, ldz = dk + 4;
   return sizeof(float) * ((size_t)8 * kBC * ldk + 6 * kBC * kBC + 2 * dk * kJS + 5 * kBC * kJS +
-                          2 * kBC + 3 * dk) +
+                          2 * kBC + 3 * dk + 3 * kBC) +
          (size_t)kBC * ldz + sizeof(int) * dk + 64;
 }
 

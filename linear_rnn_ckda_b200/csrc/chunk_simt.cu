@@ -73,6 +73,11 @@ __global__ void __launch_bounds__(kSimtThreads, 1) chunk_simt_kernel(SimtParams 
   const TIn *a = static_cast<const TIn *>(p.a);
   TOut *o = static_cast<TOut *>(p.o);
 
+  const bool per_head = per_head_gate(p.signed_gate), l2 = qk_l2norm(p.signed_gate);
+  // DeltaProduct2: the kernel walks two rows per token (k, v, b are [rows of tokens x 2]);
+  // row 2t carries the gate of token t, row 2t + 1 a gate of 1 and the read-out
+  const int rpt = delta_product2(p.signed_gate) ? 2 : 1;
+  const float unit_logit = alpha_form(p.signed_gate) == 2 ? 1.f : INFINITY;
   const int unit = blockIdx.x;
   const int n = unit / H, h = unit % H;
   const int j0 = blockIdx.y * dvs;
@@ -90,6 +95,10 @@ __global__ void __launch_bounds__(kSimtThreads, 1) chunk_simt_kernel(SimtParams 
     t1 = p.T;
     bofs = (long)n * p.T;
   }
+  // from here on t0, t1, bofs count kernel rows (two per token for DeltaProduct2)
+  t0 *= rpt;
+  t1 *= rpt;
+  bofs *= rpt;
   const size_t sbase = ((size_t)n * H + h) * dk * dv;
 
   for (int e = tid; e < dk * dvs; e += kSimtThreads) {
@@ -113,10 +122,13 @@ __global__ void __launch_bounds__(kSimtThreads, 1) chunk_simt_kernel(SimtParams 
       const int r = e / dk, c = e % dk;
       float qv = 0.f, kv = 0.f, av = 0.f;
       if (r < nrows) {
-        const size_t row = (size_t)(bofs + cs + r) * H + h;
-        qv = to_f32(q[row * dk + c]);
+        const long kr = bofs + cs + r;                    // kernel row
+        const size_t row = (size_t)kr * H + h;            // its k, v, b row
+        const size_t trow = (size_t)(kr / rpt) * H + h;   // its token's q, a, o row
+        const bool first = kr % rpt == 0, last = kr % rpt == rpt - 1;
+        qv = last ? to_f32(q[trow * dk + c]) : 0.f;
         kv = to_f32(k[row * dk + c]);
-        av = to_f32(a[row * dk + c]);
+        av = first ? to_f32(a[per_head ? trow : trow * dk + c]) : unit_logit;
       }
       sQ[r * ldk + c] = qv;
       sK[r * ldk + c] = kv;
@@ -129,6 +141,10 @@ __global__ void __launch_bounds__(kSimtThreads, 1) chunk_simt_kernel(SimtParams 
     for (int r = tid; r < C; r += kSimtThreads)
       sBeta[r] = r < nrows ? gate_beta(p.b[(size_t)(bofs + cs + r) * H + h], p.signed_gate) : 0.f;
     __syncthreads();
+    if (l2) {   // q, k divided by their norms over the key channels
+      l2norm_rows2(sQ, sK, ldk, nrows, dk, nullptr, nullptr);
+      __syncthreads();
+    }
     // ---- gate prefix per channel: L_r, zero count, parity (in place over raw a)
     for (int c = tid; c < dk; c += kSimtThreads) {
       float L = 0.f;
@@ -233,10 +249,12 @@ __global__ void __launch_bounds__(kSimtThreads, 1) chunk_simt_kernel(SimtParams 
     if (o) {
       for (int e = tid; e < nrows * dvs; e += kSimtThreads) {
         const int r = e / dvs, j = e % dvs;
+        const long kr = bofs + cs + r;
+        if (kr % rpt != rpt - 1) continue;   // DeltaProduct2: read out after a token's last update
         float acc = 0.f;
         for (int c = 0; c < dk; ++c) acc = fmaf(sQ[r * ldk + c], sS[c * dvs + j], acc);
         for (int m = 0; m <= r; ++m) acc = fmaf(sP[r * C + m], sU[m * dvs + j], acc);
-        o[((size_t)(bofs + cs + r) * H + h) * dv + j0 + j] = from_f32<TOut>(acc);
+        o[((size_t)(kr / rpt) * H + h) * dv + j0 + j] = from_f32<TOut>(acc);
       }
     }
     __syncthreads();

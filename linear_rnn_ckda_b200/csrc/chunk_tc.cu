@@ -96,6 +96,7 @@ struct TcParams {
   int n_seqs, T, H, signed_gate;
   int inject_chunk;         // test hook: chunk index of the never-completing wait (-1: off)
   uint64_t inject_wait_ns;  // its bound
+  const __nv_bfloat16 *a_head;  // per-head gate logits [rows, H] (CKDA_GATE_PER_HEAD), else NULL
 };
 
 // byte offset of fp32 element (r, c) in a 128-byte-swizzled tile of R rows
@@ -241,7 +242,8 @@ __device__ __forceinline__ int seq_of_length_rank(const int32_t *cu, int n_seqs,
   return sel;
 }
 
-template <typename TOut, int SG>
+// FL: bit 0 per-head gates (CKDA_GATE_PER_HEAD), bit 1 in-kernel q/k normalisation
+template <typename TOut, int SG, int FL>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_a,
@@ -273,6 +275,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   // staging loads issued so far (by the issuer or compute thread 0); the compute warps count
   // the ones they consumed, so a unit that gives up knows whether one is still in flight
   unsigned int *sTmaIssued = reinterpret_cast<unsigned int *>(sm + OFF_MISC + 1400);
+  // per-head gate logits of the chunk in the gate pass (bf16, CKDA_GATE_PER_HEAD), and
+  // 1 / ||q_r||, 1 / ||k_r|| of its rows (CKDA_QK_L2NORM)
+  __nv_bfloat16 *sAh = reinterpret_cast<__nv_bfloat16 *>(sm + OFF_MISC + 1408);
+  float *sInvQ = reinterpret_cast<float *>(sm + OFF_MISC + 1536);
+  float *sInvK = sInvQ + kC;
+  constexpr bool per_head = (FL & 1) != 0;
+  constexpr bool l2 = (FL & 2) != 0;
   const uint32_t sbase = smem_u32(sm);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -325,16 +334,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint64_t dR34 = smem_desc_sw128(sbase + OFF_R34, 16, 1024);
   auto dadd = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (bytes >> 4); };
 
-  auto issue_tma = [&](long cs) {
+  auto issue_tma = [&](long cs) {   // q, k, v and (per-channel gates) a of one chunk
     atomicAdd(sTmaIssued, 1u);
-    mbar_arrive_expect_tx(bar_tma, 4 * 2 * 8192);
+    const int ntens = per_head ? 3 : 4;
+    mbar_arrive_expect_tx(bar_tma, ntens * 2 * 8192);
     const int row = (int)(bofs + cs);
     const CUtensorMap *maps[4] = {&tm_q, &tm_k, &tm_v, &tm_a};
 #pragma unroll
     for (int x = 0; x < 4; ++x)
+      if (x < ntens) {
 #pragma unroll
-      for (int bx = 0; bx < 2; ++bx)
-        tma_load_3d(sStg + x * 16384 + bx * 8192, maps[x], bar_tma, bx * 64, h, row);
+        for (int bx = 0; bx < 2; ++bx)
+          tma_load_3d(sStg + x * 16384 + bx * 8192, maps[x], bar_tma, bx * 64, h, row);
+      }
   };
 
   // the compute side's staging-load bookkeeping, for the drain at the end
@@ -488,6 +500,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // to it); raw gates are checked at every row.
     float b_next = 0.f;
     if (tid < kC && t0 + tid < t1) b_next = p.b[(size_t)(bofs + t0 + tid) * H + h];
+    __nv_bfloat16 a_next = __float2bfloat16_rn(0.f);   // per-head gate logit, a chunk ahead
+    if (per_head && tid < kC && t0 + tid < t1) a_next = p.a_head[(size_t)(bofs + t0 + tid) * H + h];
     float kc[16];
     // The gate pass proper works on channel pairs: thread (pair pc = tid % 64, row group
     // rg = tid / 64) takes channels 2pc, 2pc + 1 of rows 8rg .. 8rg + 7, reading bf16 pairs
@@ -536,7 +550,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int rr = 0; rr < 8; ++rr) {
         float a0, a1, al0, al1, ial0, ial1;
-        ldbf2(sta, 8 * rg + rr, a0, a1);
+        if (per_head) {
+          a0 = a1 = __bfloat162float(sAh[8 * rg + rr]);
+        } else {
+          ldbf2(sta, 8 * rg + rr, a0, a1);
+        }
         if (SG == 1) {
           // the pair's CKDA ratios in packed fp32 pairs (same arithmetic as gate2)
           const uint64_t one = f2pk(1.f, 1.f);
@@ -591,6 +609,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         float q0, q1, k0, k1;
         ldbf2(stq, r, q0, q1);
         ldbf2(stk, r, k0, k1);
+        if (l2) {
+          const float iq = sInvQ[r], ik = sInvK[r];
+          q0 *= iq;
+          q1 *= iq;
+          k0 *= ik;
+          k1 *= ik;
+        }
         *reinterpret_cast<uint2 *>(sKQ + sw32(128, r, ch0)) =
             make_uint2(to_tf32(k0 * gam0), to_tf32(k1 * gam1));
         *reinterpret_cast<uint2 *>(sKQ + sw32(128, 64 + r, ch0)) =
@@ -606,6 +631,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float b_cur = b_next;
       if (tid < kC && cs + kC + tid < t1) b_next = p.b[(size_t)(bofs + cs + kC + tid) * H + h];
       if (tid < kC) sBeta[tid] = tid < nrows ? fast_beta(b_cur, beta_form(p.signed_gate)) : 0.f;
+      if (per_head) {
+        // the chunk's per-head gate logits (rows past the end: a gate of exactly 1)
+        const __nv_bfloat16 a_cur = a_next;
+        if (tid < kC && cs + kC + tid < t1)
+          a_next = p.a_head[(size_t)(bofs + cs + kC + tid) * H + h];
+        if (tid < kC) sAh[tid] = tid < nrows ? a_cur : __float2bfloat16_rn(SG == 2 ? 1.f : 100.f);
+      }
       if (nrows < kC) {
         // Rows past the sequence end hold another sequence's tokens or TMA fill.  They are
         // overwritten in the staging copy with q = k = v = 0 and a gate of exactly 1
@@ -621,6 +653,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                                      (piece & 7) * 16) = make_uint4(f, f, f, f);
         }
         csync();
+      } else if (per_head || l2) {
+        csync();
+      }
+      if (l2) {
+        // 1 / ||q_r|| and 1 / ||k_r|| over the key channels: warp w takes rows w, w + 16, ...
+        // of q and of k, four channels per lane (8 bytes inside one 16-byte chunk); they are
+        // read after the gate pass's exchange barrier
+        for (int it = warp; it < 2 * kC; it += kCompute / 32) {
+          const int r = it % kC;
+          const uint8_t *tile = it < kC ? stq : stk;
+          const uint2 u = *reinterpret_cast<const uint2 *>(tile + swbf(r, 4 * lane));
+          const float x0 = __uint_as_float(u.x << 16), x1 = __uint_as_float(u.x & 0xFFFF0000u);
+          const float x2 = __uint_as_float(u.y << 16), x3 = __uint_as_float(u.y & 0xFFFF0000u);
+          float ss = fmaf(x0, x0, fmaf(x1, x1, fmaf(x2, x2, x3 * x3)));
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+          if (lane == 0) (it < kC ? sInvQ : sInvK)[r] = inv_norm(ss);
+        }
       }
       return gate_core(gc_out, vcol);
     };
@@ -712,7 +762,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 4
         for (int rr = 0; rr < 16; ++rr) {
           const int r = 16 * qg + rr;
-          sAl[r * kD + c] = r < nrows ? gate_alpha(ldbf(sta, r, c), SG) : 1.f;
+          sAl[r * kD + c] =
+              r < nrows ? gate_alpha(per_head ? __bfloat162float(sAh[r]) : ldbf(sta, r, c), SG)
+                        : 1.f;
         }
         tc_fence_after();
         {
@@ -725,12 +777,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         csync();
         for (int t = 0; t < nrows; ++t) {
+          const float iqt = l2 ? sInvQ[t] : 1.f, ikt = l2 ? sInvK[t] : 1.f;
           float pk = 0.f;
           for (int x = 0; x < 32; ++x) {
             const int i = 32 * qg + x;
             const float sv = sS[i * kD + jrow] * sAl[t * kD + i];
             sS[i * kD + jrow] = sv;
-            pk = fmaf(ldbf(stk, t, i), sv, pk);
+            pk = fmaf(ldbf(stk, t, i) * ikt, sv, pk);
           }
           sRed[qg * 128 + jrow] = pk;
           csync();
@@ -740,9 +793,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           float acc = 0.f;
           for (int x = 0; x < 32; ++x) {
             const int i = 32 * qg + x;
-            const float sv = fmaf(ldbf(stk, t, i), u, sS[i * kD + jrow]);
+            const float sv = fmaf(ldbf(stk, t, i) * ikt, u, sS[i * kD + jrow]);
             sS[i * kD + jrow] = sv;
-            acc = fmaf(ldbf(stq, t, i), sv, acc);
+            acc = fmaf(ldbf(stq, t, i) * iqt, sv, acc);
           }
           sRed[512 + qg * 128 + jrow] = acc;
           csync();
@@ -992,7 +1045,7 @@ bool make_out_map(CUtensorMap *map, void *base, int H, long rows, bool bf16) {
              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <typename TOut, int SG>
+template <typename TOut, int SG, int FL>
 int launch_typed(const ChunkArgs &g, cudaStream_t stream) {
   const long rows = (long)g.B * g.T;
   if (rows == 0) {
@@ -1000,8 +1053,10 @@ int launch_typed(const ChunkArgs &g, cudaStream_t stream) {
   }
   CUtensorMap mq, mk, mv, ma, mo;
   const long map_rows = rows > 0 ? rows : 1;
+  const bool per_head = per_head_gate(g.signed_gate);   // a is [rows, H]: no tile map
+  memset(&ma, 0, sizeof(ma));
   if (!make_map(&mq, g.q, g.H, map_rows) || !make_map(&mk, g.k, g.H, map_rows) ||
-      !make_map(&mv, g.v, g.H, map_rows) || !make_map(&ma, g.a, g.H, map_rows))
+      !make_map(&mv, g.v, g.H, map_rows) || (!per_head && !make_map(&ma, g.a, g.H, map_rows)))
     return CKDA_ERR_CUDA;
   memset(&mo, 0, sizeof(mo));
   if (g.o && !make_out_map(&mo, g.o, g.H, map_rows, g.o_dtype == CKDA_BF16)) return CKDA_ERR_CUDA;
@@ -1010,7 +1065,8 @@ int launch_typed(const ChunkArgs &g, cudaStream_t stream) {
   p.n_seqs = g.n_seqs; p.T = g.T; p.H = g.H; p.signed_gate = g.signed_gate;
   p.inject_chunk = g.inject_chunk;
   p.inject_wait_ns = g.inject_wait_ns;
-  auto kern = chunk_tc_kernel<TOut, SG>;
+  p.a_head = per_head ? static_cast<const __nv_bfloat16 *>(g.a) : nullptr;
+  auto kern = chunk_tc_kernel<TOut, SG, FL>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) !=
       cudaSuccess)
     return CKDA_ERR_CUDA;
@@ -1021,18 +1077,26 @@ int launch_typed(const ChunkArgs &g, cudaStream_t stream) {
 }  // namespace
 
 bool chunk_tc_supported(const ChunkArgs &g) {
-  return g.dk == kD && g.dv == kD && g.chunk == kC && g.io_dtype == CKDA_BF16 && g.B * (long)g.T > 0;
+  return g.dk == kD && g.dv == kD && g.chunk == kC && g.io_dtype == CKDA_BF16 &&
+         g.B * (long)g.T > 0 && !delta_product2(g.signed_gate);
 }
 
 int launch_chunk_tc(const ChunkArgs &g, cudaStream_t s) {
   if (g.n_seqs * g.H == 0) return CKDA_OK;
   const bool bf = g.o_dtype == CKDA_BF16;
-  // the kernel is specialised on the gate's form; the strength's form is read at run time
-  switch (alpha_form(g.signed_gate)) {
-    case 0: return bf ? launch_typed<__nv_bfloat16, 0>(g, s) : launch_typed<float, 0>(g, s);
-    case 1: return bf ? launch_typed<__nv_bfloat16, 1>(g, s) : launch_typed<float, 1>(g, s);
-    default: return bf ? launch_typed<__nv_bfloat16, 2>(g, s) : launch_typed<float, 2>(g, s);
+  // the kernel is specialised on the gate's form and the flags; the strength's form is read
+  // at run time
+  const int fl = (per_head_gate(g.signed_gate) ? 1 : 0) | (qk_l2norm(g.signed_gate) ? 2 : 0);
+  switch (alpha_form(g.signed_gate) * 4 + fl) {
+#define CKDA_TC_CASE(SGV, FLV)                                                     \
+  case SGV * 4 + FLV:                                                             \
+    return bf ? launch_typed<__nv_bfloat16, SGV, FLV>(g, s) : launch_typed<float, SGV, FLV>(g, s);
+    CKDA_TC_CASE(0, 0) CKDA_TC_CASE(0, 1) CKDA_TC_CASE(0, 2) CKDA_TC_CASE(0, 3)
+    CKDA_TC_CASE(1, 0) CKDA_TC_CASE(1, 1) CKDA_TC_CASE(1, 2) CKDA_TC_CASE(1, 3)
+    CKDA_TC_CASE(2, 0) CKDA_TC_CASE(2, 1) CKDA_TC_CASE(2, 2) CKDA_TC_CASE(2, 3)
+#undef CKDA_TC_CASE
   }
+  return CKDA_ERR_DTYPE;
 }
 
 }  // namespace ckda

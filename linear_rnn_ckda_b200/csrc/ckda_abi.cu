@@ -19,6 +19,11 @@ bool aligned(const void *p, uintptr_t n) {
   return p == nullptr || (reinterpret_cast<uintptr_t>(p) & (n - 1)) == 0;
 }
 bool aligned16(const void *p) { return aligned(p, 16); }
+// a gate form 0..4, optionally with CKDA_GATE_PER_HEAD, CKDA_QK_L2NORM, CKDA_DELTA_PRODUCT2
+bool valid_gate(int sg) {
+  return sg >= 0 && (sg & 15) <= 4 &&
+         (sg & ~(15 | CKDA_GATE_PER_HEAD | CKDA_QK_L2NORM | CKDA_DELTA_PRODUCT2)) == 0;
+}
 
 // sm_100 check for the current device, cached per device (atomics: host threads may call the
 // library concurrently; the cached value is the same whoever writes it).
@@ -52,13 +57,14 @@ int check_chunk_args(const void *q, const void *k, const void *v, const void *a,
   if (!q || !k || !v || !a || !b) return CKDA_ERR_NULL;
   if (!valid_dim(dk) || !valid_dim(dv) || B < 0 || T < 0 || H <= 0) return CKDA_ERR_DIM;
   if (chunk != 16 && chunk != 32 && chunk != 64) return CKDA_ERR_CHUNK;
-  if (signed_gate < 0 || signed_gate > 4 || (io_dtype != CKDA_F32 && io_dtype != CKDA_BF16) ||
+  if (!valid_gate(signed_gate) || (io_dtype != CKDA_F32 && io_dtype != CKDA_BF16) ||
       (o_dtype != CKDA_F32 && o_dtype != CKDA_BF16))
     return CKDA_ERR_DTYPE;
   if (cu_seqlens && (B != 1 || n_seqs < 0)) return CKDA_ERR_DIM;
-  // token rows are 32-bit coordinates in the kernels (TMA tile coordinates included)
-  if ((long long)B * T > (long long)INT32_MAX || (long long)B * T * H > (1LL << 40))
-    return CKDA_ERR_DIM;
+  // token rows are 32-bit coordinates in the kernels (TMA tile coordinates included); a
+  // DeltaProduct2 token is two rows
+  const long long rows = (long long)B * T * ((signed_gate & CKDA_DELTA_PRODUCT2) ? 2 : 1);
+  if (rows > (long long)INT32_MAX || rows * H > (1LL << 41)) return CKDA_ERR_DIM;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(a) || !aligned(b, 4) ||
       !aligned16(S0) || !aligned16(o) || !aligned16(S_T) || !aligned(cu_seqlens, 4))
     return CKDA_ERR_ALIGN;
@@ -146,6 +152,7 @@ int ckda_chunk_bwd(const void *q, const void *k, const void *v, const void *a, c
   if (arg_rc != CKDA_OK) return arg_rc;
   if (!dq || !dk_out || !dv_out || !da || !db) return CKDA_ERR_NULL;
   if (do_dtype != CKDA_F32 && do_dtype != CKDA_BF16) return CKDA_ERR_DTYPE;
+  if (signed_gate & CKDA_DELTA_PRODUCT2) return CKDA_ERR_DTYPE;   // forward only
   if (!aligned16(dO) || !aligned16(dS_T) || !aligned16(dq) || !aligned16(dk_out) ||
       !aligned16(dv_out) || !aligned16(da) || !aligned(db, 4) || !aligned16(dS0))
     return CKDA_ERR_ALIGN;
@@ -177,7 +184,7 @@ int ckda_decode_step(const void *q, const void *k, const void *v, const void *a,
   if (!q || !k || !v || !a || !b || !S) return CKDA_ERR_NULL;
   if (!valid_dim(dk) || !valid_dim(dv) || B < 0 || H <= 0) return CKDA_ERR_DIM;
   if ((long long)B * H > (1LL << 31) - 1) return CKDA_ERR_DIM;
-  if (signed_gate < 0 || signed_gate > 4 || (io_dtype != CKDA_F32 && io_dtype != CKDA_BF16) ||
+  if (!valid_gate(signed_gate) || (io_dtype != CKDA_F32 && io_dtype != CKDA_BF16) ||
       (o_dtype != CKDA_F32 && o_dtype != CKDA_BF16))
     return CKDA_ERR_DTYPE;
   const uintptr_t in_sz = io_dtype == CKDA_BF16 ? 2 : 4, out_sz = o_dtype == CKDA_BF16 ? 2 : 4;

@@ -31,16 +31,36 @@ __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
   return __float2bfloat16_rn(x);
 }
 
-// Gate forms: signed_gate 0 (KDA) widens no range and 1 (CKDA) both; 3 widens the gate range
-// alone and 4 the strength range alone (the single-range variants of the CKDA review's
-// Figure 6); 2 passes raw values.  The gate is sigma / 2 sigma - 1 / raw for alpha_form
-// 0 / 1 / 2, the strength sigma / 2 sigma / raw for beta_form 0 / 1 / 2.
+// Gate forms (signed_gate & kGateFormMask): 0 (KDA) widens no range and 1 (CKDA) both; 3 widens
+// the gate range alone and 4 the strength range alone (the single-range variants of the CKDA
+// review's Figure 6); 2 passes raw values.  The gate is sigma / 2 sigma - 1 / raw for alpha_form
+// 0 / 1 / 2, the strength sigma / 2 sigma / raw for beta_form 0 / 1 / 2.  Two flag bits ride
+// above the form: kFlagPerHeadGate (one gate per token and head, GDN-style: a is [B,T,H] and
+// the gate is broadcast over the key channels) and kFlagQkL2Norm (q and k are divided by
+// their L2 norm over the key channels inside the kernel).
+constexpr int kGateFormMask = 15;
+constexpr int kFlagPerHeadGate = CKDA_GATE_PER_HEAD;
+constexpr int kFlagQkL2Norm = CKDA_QK_L2NORM;
+constexpr int kFlagProduct2 = CKDA_DELTA_PRODUCT2;
 __host__ __device__ __forceinline__ constexpr int alpha_form(int signed_gate) {
-  return signed_gate == 3 ? 1 : (signed_gate == 4 ? 0 : signed_gate);
+  return (signed_gate & kGateFormMask) == 3 ? 1
+         : (signed_gate & kGateFormMask) == 4 ? 0 : (signed_gate & kGateFormMask);
 }
 __host__ __device__ __forceinline__ constexpr int beta_form(int signed_gate) {
-  return signed_gate == 3 ? 0 : (signed_gate == 4 ? 1 : signed_gate);
+  return (signed_gate & kGateFormMask) == 3 ? 0
+         : (signed_gate & kGateFormMask) == 4 ? 1 : (signed_gate & kGateFormMask);
 }
+__host__ __device__ __forceinline__ constexpr bool per_head_gate(int signed_gate) {
+  return (signed_gate & kFlagPerHeadGate) != 0;
+}
+__host__ __device__ __forceinline__ constexpr bool qk_l2norm(int signed_gate) {
+  return (signed_gate & kFlagQkL2Norm) != 0;
+}
+__host__ __device__ __forceinline__ constexpr bool delta_product2(int signed_gate) {
+  return (signed_gate & kFlagProduct2) != 0;
+}
+// 1 / ||x|| from the sum of squares, 0 for a zero vector (which then stays zero)
+__device__ __forceinline__ float inv_norm(float sumsq) { return sumsq > 0.f ? rsqrtf(sumsq) : 0.f; }
 
 // Linear gate value alpha (decode path).  Exact at +-inf: sigma 1/0, 2 sigma - 1 +-1.
 __device__ __forceinline__ float gate_alpha(float a, int signed_gate) {
@@ -98,6 +118,36 @@ __device__ __forceinline__ float dalpha_da(float a, int signed_gate) {
 __device__ __forceinline__ float dbeta_db(float b, int signed_gate) {
   const int f = beta_form(signed_gate);
   return f == 2 ? 1.0f : (f == 1 ? 2.0f : 1.0f) * dsigmoid(b);
+}
+
+// Divides rows 0..rows-1 of the fp32 tiles X and Y (row stride ld, n columns) by their L2
+// norms (a zero row stays zero); the factors go to inv_x / inv_y when given.  One warp per
+// row, the whole block takes part; the caller synchronises before and after.
+__device__ __forceinline__ void l2norm_rows2(float *X, float *Y, int ld, int rows, int n,
+                                             float *inv_x, float *inv_y) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  for (int r = warp; r < rows; r += nw) {
+    float sx = 0.f, sy = 0.f;
+    for (int c = lane; c < n; c += 32) {
+      const float x = X[r * ld + c], y = Y[r * ld + c];
+      sx = fmaf(x, x, sx);
+      sy = fmaf(y, y, sy);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      sx += __shfl_xor_sync(0xffffffffu, sx, off);
+      sy += __shfl_xor_sync(0xffffffffu, sy, off);
+    }
+    const float ix = inv_norm(sx), iy = inv_norm(sy);
+    for (int c = lane; c < n; c += 32) {
+      X[r * ld + c] *= ix;
+      Y[r * ld + c] *= iy;
+    }
+    if (lane == 0 && inv_x) {
+      inv_x[r] = ix;
+      inv_y[r] = iy;
+    }
+  }
 }
 
 // Records the first device-detected error in the workspace status word.

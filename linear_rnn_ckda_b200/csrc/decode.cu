@@ -24,14 +24,15 @@ template <int DK, int DV, typename TIn, typename TOut>
 __global__ void __launch_bounds__(kDecodeThreads)
     decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
                   const TIn *__restrict__ a, const float *__restrict__ b, float *__restrict__ S,
-                  TOut *__restrict__ o, int n_heads, int signed_gate) {
+                  TOut *__restrict__ o, int n_heads, int H, int signed_gate) {
   constexpr int kWarpsPerHead = DV / 16;
   constexpr int kHeadsPerBlock = (kDecodeThreads / 32) / kWarpsPerHead;
   constexpr int kRows = DK / 8;  // state rows per thread
   __shared__ float s_q[kHeadsPerBlock][DK];
   __shared__ float s_k[kHeadsPerBlock][DK];
   __shared__ float s_al[kHeadsPerBlock][DK];
-  __shared__ float s_beta[kHeadsPerBlock];
+  __shared__ float s_k2[kHeadsPerBlock][DK];     // DeltaProduct2: the token's second key
+  __shared__ float s_beta[kHeadsPerBlock][2];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int hl = warp / kWarpsPerHead;
@@ -50,17 +51,51 @@ __global__ void __launch_bounds__(kDecodeThreads)
       st[m] = *reinterpret_cast<const float4 *>(Sh + (size_t)(r0 + 8 * m) * DV + col);
   }
 
-  // Stage q, k and the activated gate for this head group.
+  // Stage q, k and the activated gate for this head group (one gate per head with
+  // CKDA_GATE_PER_HEAD: a is [B, H]).
+  // (DeltaProduct2: k, v, b hold two rows per token, [B, 2, H, .]; key j of this head is
+  // row (head / H * 2 + j) * H + head % H)
+  const bool per_head = per_head_gate(signed_gate), prod2 = delta_product2(signed_gate);
+  const size_t krow1 = prod2 ? ((size_t)(head / H) * 2) * H + head % H : (size_t)head;
+  const size_t krow2 = krow1 + H;
   if (head < n_heads) {
     for (int i = gtid; i < DK; i += kWarpsPerHead * 32) {
       const size_t e = (size_t)head * DK + i;
       s_q[hl][i] = to_f32(q[e]);
-      s_k[hl][i] = to_f32(k[e]);
-      s_al[hl][i] = gate_alpha(to_f32(a[e]), signed_gate);
+      s_k[hl][i] = to_f32(k[krow1 * DK + i]);
+      if (prod2) s_k2[hl][i] = to_f32(k[krow2 * DK + i]);
+      s_al[hl][i] = gate_alpha(to_f32(a[per_head ? (size_t)head : e]), signed_gate);
     }
-    if (gtid == 0) s_beta[hl] = gate_beta(b[head], signed_gate);
+    if (gtid == 0) {
+      s_beta[hl][0] = gate_beta(b[krow1], signed_gate);
+      if (prod2) s_beta[hl][1] = gate_beta(b[krow2], signed_gate);
+    }
   }
   __syncthreads();
+  if (qk_l2norm(signed_gate)) {
+    // q and k divided by their norms over the key channels (the head group's first warp)
+    if (head < n_heads && gtid < 32) {
+      float sq = 0.f, sk = 0.f, sk2 = 0.f;
+      for (int i = gtid; i < DK; i += 32) {
+        sq = fmaf(s_q[hl][i], s_q[hl][i], sq);
+        sk = fmaf(s_k[hl][i], s_k[hl][i], sk);
+        if (prod2) sk2 = fmaf(s_k2[hl][i], s_k2[hl][i], sk2);
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        sq += __shfl_xor_sync(0xffffffffu, sq, off);
+        sk += __shfl_xor_sync(0xffffffffu, sk, off);
+        sk2 += __shfl_xor_sync(0xffffffffu, sk2, off);
+      }
+      const float iq = inv_norm(sq), ik = inv_norm(sk), ik2 = inv_norm(sk2);
+      for (int i = gtid; i < DK; i += 32) {
+        s_q[hl][i] *= iq;
+        s_k[hl][i] *= ik;
+        if (prod2) s_k2[hl][i] *= ik2;
+      }
+    }
+    __syncthreads();
+  }
   if (head >= n_heads) return;
 
   // S' = Diag(alpha) S and p = S'^T k (partial over this thread's rows)
@@ -82,17 +117,42 @@ __global__ void __launch_bounds__(kDecodeThreads)
   }
 
   // u = beta (v - p)
-  const float beta = s_beta[hl];
-  const TIn *vh = v + (size_t)head * DV + col;
-  const float u0 = beta * (to_f32(vh[0]) - p0), u1 = beta * (to_f32(vh[1]) - p1);
-  const float u2 = beta * (to_f32(vh[2]) - p2), u3 = beta * (to_f32(vh[3]) - p3);
+  const float beta = s_beta[hl][0];
+  const TIn *vh = v + krow1 * DV + col;
+  float u0 = beta * (to_f32(vh[0]) - p0), u1 = beta * (to_f32(vh[1]) - p1);
+  float u2 = beta * (to_f32(vh[2]) - p2), u3 = beta * (to_f32(vh[3]) - p3);
+  if (prod2) {
+    // DeltaProduct2: the first update, then the second key's read p' = S''^T k2 and its update
+    float q0 = 0.f, q1 = 0.f, q2 = 0.f, q3 = 0.f;
+#pragma unroll
+    for (int m = 0; m < kRows; ++m) {
+      const int i = r0 + 8 * m;
+      const float ki = s_k[hl][i], k2i = s_k2[hl][i];
+      st[m].x = fmaf(ki, u0, st[m].x); st[m].y = fmaf(ki, u1, st[m].y);
+      st[m].z = fmaf(ki, u2, st[m].z); st[m].w = fmaf(ki, u3, st[m].w);
+      q0 = fmaf(k2i, st[m].x, q0); q1 = fmaf(k2i, st[m].y, q1);
+      q2 = fmaf(k2i, st[m].z, q2); q3 = fmaf(k2i, st[m].w, q3);
+    }
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      q0 += __shfl_xor_sync(0xffffffffu, q0, off);
+      q1 += __shfl_xor_sync(0xffffffffu, q1, off);
+      q2 += __shfl_xor_sync(0xffffffffu, q2, off);
+      q3 += __shfl_xor_sync(0xffffffffu, q3, off);
+    }
+    const float beta2 = s_beta[hl][1];
+    const TIn *vh2 = v + krow2 * DV + col;
+    u0 = beta2 * (to_f32(vh2[0]) - q0); u1 = beta2 * (to_f32(vh2[1]) - q1);
+    u2 = beta2 * (to_f32(vh2[2]) - q2); u3 = beta2 * (to_f32(vh2[3]) - q3);
+  }
+  const float(*kw)[DK] = prod2 ? s_k2 : s_k;   // the key of the last update
 
   // S = S' + k u^T, written back; o = S^T q
   float r0s = 0.f, r1s = 0.f, r2s = 0.f, r3s = 0.f;
 #pragma unroll
   for (int m = 0; m < kRows; ++m) {
     const int i = r0 + 8 * m;
-    const float ki = s_k[hl][i], qi = s_q[hl][i];
+    const float ki = kw[hl][i], qi = s_q[hl][i];
     st[m].x = fmaf(ki, u0, st[m].x); st[m].y = fmaf(ki, u1, st[m].y);
     st[m].z = fmaf(ki, u2, st[m].z); st[m].w = fmaf(ki, u3, st[m].w);
     *reinterpret_cast<float4 *>(Sh + (size_t)i * DV + col) = st[m];
@@ -121,7 +181,8 @@ int launch_typed(const DecodeArgs &g, cudaStream_t stream) {
   const int blocks = (n_heads + kHeadsPerBlock - 1) / kHeadsPerBlock;
   decode_kernel<DK, DV, TIn, TOut><<<blocks, kDecodeThreads, 0, stream>>>(
       static_cast<const TIn *>(g.q), static_cast<const TIn *>(g.k), static_cast<const TIn *>(g.v),
-      static_cast<const TIn *>(g.a), g.b, g.S, static_cast<TOut *>(g.o), n_heads, g.signed_gate);
+      static_cast<const TIn *>(g.a), g.b, g.S, static_cast<TOut *>(g.o), n_heads, g.H,
+      g.signed_gate);
   return cudaGetLastError() == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
 }
 

@@ -20,6 +20,10 @@ _lib = None
 
 CKDA_F32 = 0
 CKDA_BF16 = 1
+# flags OR-ed into signed_gate (include/ckda.h)
+GATE_PER_HEAD = 16   # one gate logit per token and head: a is [B,T,H] ([B,H] for decode)
+QK_L2NORM = 32       # q and k are L2-normalised inside the kernels
+DELTA_PRODUCT2 = 64  # two keys, values, strengths per token: k [B,T,2,H,dk], v [B,T,2,H,dv], b [B,T,2,H]
 _DT = {torch.float32: CKDA_F32, torch.bfloat16: CKDA_BF16}
 _TORCH_DT = {CKDA_F32: torch.float32, CKDA_BF16: torch.bfloat16}
 
@@ -100,7 +104,7 @@ def _same_device(ref: torch.Tensor, **tensors):
 
 
 def check_prefill_args(q, k, v, a, b, S0=None, cu_seqlens=None, o=None, S_T=None,
-                       o_dtype=None):
+                       o_dtype=None, signed_gate: int = 0):
     """Shapes, dtypes and devices that ``ckda_chunk_fwd`` relies on but cannot see (it receives
     bare pointers, so a short or mistyped buffer would be read or written past its end).
     Raises ValueError; returns (N, dv).  The offsets inside ``cu_seqlens`` are checked on the
@@ -108,14 +112,18 @@ def check_prefill_args(q, k, v, a, b, S0=None, cu_seqlens=None, o=None, S_T=None
     _need(q.dim() == 4, f"q must be [B,T,H,dk], got {tuple(q.shape)}")
     _need(q.dtype in _DT, f"q must be float32 or bfloat16, got {q.dtype}")
     B, T, H, dk = q.shape
-    for name, t in (("k", k), ("a", a)):
-        _need(t.shape == q.shape and t.dtype == q.dtype,
-              f"{name} must match q ({tuple(q.shape)}, {q.dtype}), got {tuple(t.shape)}, {t.dtype}")
-    _need(v.dim() == 4 and v.shape[:3] == q.shape[:3] and v.dtype == q.dtype,
-          f"v must be [B,T,H,dv] in q's dtype, got {tuple(v.shape)}, {v.dtype}")
+    p2 = bool(signed_gate & DELTA_PRODUCT2)
+    lead = (B, T, 2, H) if p2 else (B, T, H)   # rows of k, v, b (two per token for DeltaProduct2)
+    _need(tuple(k.shape) == lead + (dk,) and k.dtype == q.dtype,
+          f"k must be {lead + (dk,)} in q's dtype, got {tuple(k.shape)}, {k.dtype}")
+    a_shape = (B, T, H) if signed_gate & GATE_PER_HEAD else tuple(q.shape)
+    _need(tuple(a.shape) == a_shape and a.dtype == q.dtype,
+          f"a must be {a_shape} in q's dtype, got {tuple(a.shape)}, {a.dtype}")
+    _need(v.dim() == len(lead) + 1 and tuple(v.shape[:-1]) == lead and v.dtype == q.dtype,
+          f"v must be {lead + ('dv',)} in q's dtype, got {tuple(v.shape)}, {v.dtype}")
     dv = v.shape[-1]
-    _need(b.shape == (B, T, H) and b.dtype == torch.float32,
-          f"b must be [B,T,H] float32, got {tuple(b.shape)}, {b.dtype}")
+    _need(tuple(b.shape) == lead and b.dtype == torch.float32,
+          f"b must be {lead} float32, got {tuple(b.shape)}, {b.dtype}")
     N = B
     if cu_seqlens is not None:
         _need(cu_seqlens.dim() == 1 and cu_seqlens.numel() >= 1 and cu_seqlens.dtype == torch.int32,
@@ -133,20 +141,23 @@ def check_prefill_args(q, k, v, a, b, S0=None, cu_seqlens=None, o=None, S_T=None
     return N, dv
 
 
-def check_decode_args(q, k, v, a, b, S, o=None, o_dtype=None):
+def check_decode_args(q, k, v, a, b, S, o=None, o_dtype=None, signed_gate: int = 0):
     """The same checks for ``ckda_decode_step``: q, k, a [B,H,dk]; v [B,H,dv] in q's dtype;
     b [B,H] float32; S [B,H,dk,dv] float32; o [B,H,dv] in the output dtype."""
     _need(q.dim() == 3, f"q must be [B,H,dk], got {tuple(q.shape)}")
     _need(q.dtype in _DT, f"q must be float32 or bfloat16, got {q.dtype}")
     B, H, dk = q.shape
-    for name, t in (("k", k), ("a", a)):
-        _need(t.shape == q.shape and t.dtype == q.dtype,
-              f"{name} must match q ({tuple(q.shape)}, {q.dtype}), got {tuple(t.shape)}, {t.dtype}")
-    _need(v.dim() == 3 and v.shape[:2] == q.shape[:2] and v.dtype == q.dtype,
-          f"v must be [B,H,dv] in q's dtype, got {tuple(v.shape)}, {v.dtype}")
+    lead = (B, 2, H) if signed_gate & DELTA_PRODUCT2 else (B, H)
+    _need(tuple(k.shape) == lead + (dk,) and k.dtype == q.dtype,
+          f"k must be {lead + (dk,)} in q's dtype, got {tuple(k.shape)}, {k.dtype}")
+    a_shape = (B, H) if signed_gate & GATE_PER_HEAD else tuple(q.shape)
+    _need(tuple(a.shape) == a_shape and a.dtype == q.dtype,
+          f"a must be {a_shape} in q's dtype, got {tuple(a.shape)}, {a.dtype}")
+    _need(v.dim() == len(lead) + 1 and tuple(v.shape[:-1]) == lead and v.dtype == q.dtype,
+          f"v must be {lead + ('dv',)} in q's dtype, got {tuple(v.shape)}, {v.dtype}")
     dv = v.shape[-1]
-    _need(b.shape == (B, H) and b.dtype == torch.float32,
-          f"b must be [B,H] float32, got {tuple(b.shape)}, {b.dtype}")
+    _need(tuple(b.shape) == lead and b.dtype == torch.float32,
+          f"b must be {lead} float32, got {tuple(b.shape)}, {b.dtype}")
     _need(S.shape == (B, H, dk, dv) and S.dtype == torch.float32,
           f"S must be [B,H,dk,dv] = {(B, H, dk, dv)} float32")
     od = q.dtype if o_dtype is None else o_dtype
@@ -179,7 +190,7 @@ def chunk_fwd(q, k, v, a, b, S0=None, cu_seqlens=None, chunk: int = 64, signed_g
     S0: [N,H,dk,dv] fp32 or None; cu_seqlens: int32 CUDA tensor [N+1] or None.
     """
     lib = load()
-    N, dv = check_prefill_args(q, k, v, a, b, S0, cu_seqlens, o, S_T, o_dtype)
+    N, dv = check_prefill_args(q, k, v, a, b, S0, cu_seqlens, o, S_T, o_dtype, signed_gate)
     B, T, H, dk = q.shape
     io = _DT[q.dtype]
     od = io if o_dtype is None else _DT[o_dtype]
@@ -214,7 +225,7 @@ def chunk_bwd(q, k, v, a, b, S0=None, cu_seqlens=None, dO=None, dS_T=None,
     (zero); dS_T: [N,H,dk,dv] float32 or None (zero).  ``grads`` may supply the six output
     tensors."""
     lib = load()
-    N, dv = check_prefill_args(q, k, v, a, b, S0, cu_seqlens)
+    N, dv = check_prefill_args(q, k, v, a, b, S0, cu_seqlens, signed_gate=signed_gate)
     B, T, H, dk = q.shape
     dev = q.device
     _need(dO is None or (dO.shape == (B, T, H, dv) and dO.dtype in _DT),
@@ -225,12 +236,12 @@ def chunk_bwd(q, k, v, a, b, S0=None, cu_seqlens=None, dO=None, dS_T=None,
     if grads is None:
         f32 = dict(dtype=torch.float32, device=dev)
         grads = (torch.empty((B, T, H, dk), **f32), torch.empty((B, T, H, dk), **f32),
-                 torch.empty((B, T, H, dv), **f32), torch.empty((B, T, H, dk), **f32),
+                 torch.empty((B, T, H, dv), **f32), torch.empty(tuple(a.shape), **f32),
                  torch.empty((B, T, H), **f32),
                  torch.empty((N, H, dk, dv), **f32) if want_dS0 else None)
     gq, gk, gv, ga, gb, gS0 = grads
     for name, t, shape in (("dq", gq, (B, T, H, dk)), ("dk", gk, (B, T, H, dk)),
-                           ("dv", gv, (B, T, H, dv)), ("da", ga, (B, T, H, dk)),
+                           ("dv", gv, (B, T, H, dv)), ("da", ga, tuple(a.shape)),
                            ("db", gb, (B, T, H)), ("dS0", gS0, (N, H, dk, dv))):
         _need(t is None or (tuple(t.shape) == shape and t.dtype == torch.float32),
               f"{name} must be {shape} float32")
@@ -252,7 +263,7 @@ def chunk_bwd(q, k, v, a, b, S0=None, cu_seqlens=None, dO=None, dS_T=None,
 def decode_step(q, k, v, a, b, S, signed_gate: int = 1, o_dtype=None, o=None, want_o=True):
     """One decode step; S [B,H,dk,dv] fp32 is updated in place.  Returns o [B,H,dv]."""
     lib = load()
-    dv = check_decode_args(q, k, v, a, b, S, o, o_dtype)
+    dv = check_decode_args(q, k, v, a, b, S, o, o_dtype, signed_gate)
     B, H, dk = q.shape
     io = _DT[q.dtype]
     od = io if o_dtype is None else _DT[o_dtype]
