@@ -358,10 +358,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--decode-steps", type=int, default=None,
                     help="timed decode steps (default: --steps rounded up to the 128-step cycle)")
-    ap.add_argument("--legs", default="varlen,e2e,kda,spread,ratio,bwd,decode",
+    ap.add_argument("--legs", default="varlen,e2e,kda,spread,fast,ratio,bwd,decode",
                     help="comma list of legs to run (varlen = the headline, e2e, kda, spread, "
-                         "ratio, bwd, decode); a profiling run can select one, the default runs "
-                         "all")
+                         "fast = KDA with fast-forgetting channels, ratio, bwd, decode); a "
+                         "profiling run can select one, the default runs all")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -384,21 +384,26 @@ def main():
     extra_steps = max(3, min(args.steps, 10))
 
     # ------------------------------------------------------------ headline: varlen CKDA
+    # (a profiling run that leaves the headline out of --legs skips it and its e2e leg)
     w = HEADLINE
-    host = synth.make_prefill(w, seed=rank)
-    case = PrefillCase(ops, w, host, dev)
     run_head = "varlen" in legs
-    with ClockSampler(local) as clk:
-        ms = time_loop(case, args.steps if run_head else 1, args.warmup if run_head else 0, world,
-                       stream)
-    ms = max_over_ranks(ms, world) if run_head else float("nan")
-    case.check("the headline leg")
-    ms_step = ms / args.steps
     tokens = w.tokens * world
-    value = tokens * args.steps / (ms / 1000.0)
-    # dominant kernel: the chunk kernel, one launch per step (the 256-byte status memset
-    # before it is included, < 2 us)
-    roofline = prefill_roofline(w, ms_step, peaks, "chunk_tc_kernel/" + w.name)
+    ms = ms_step = value = float("nan")
+    roofline = None
+    host = case = None
+    clk = ClockSampler(local)
+    if run_head:
+        host = synth.make_prefill(w, seed=rank)
+        case = PrefillCase(ops, w, host, dev)
+        with clk:
+            ms = time_loop(case, args.steps, args.warmup, world, stream)
+        ms = max_over_ranks(ms, world)
+        case.check("the headline leg")
+        ms_step = ms / args.steps
+        value = tokens * args.steps / (ms / 1000.0)
+        # dominant kernel: the chunk kernel, one launch per step (the 256-byte status memset
+        # before it is included, < 2 us)
+        roofline = prefill_roofline(w, ms_step, peaks, "chunk_tc_kernel/" + w.name)
 
     # ------------------------------------------------------------ e2e (host buffers)
     # Each step copies its own q, k, v, a, b, S0 and cu_seqlens from pinned host memory, runs
@@ -407,10 +412,10 @@ def main():
     # of device buffers, so one step's read-back overlaps the next step's upload.  Timed with
     # CUDA events from the first upload to the last read-back.
     e2e = None
-    keys = [k for k in ("q", "k", "v", "a", "b", "S0", "cu_seqlens") if host.get(k) is not None]
-    h2d = sum(host[k].numel() * host[k].element_size() for k in keys)
-    d2h = case.o.numel() * case.o.element_size() + case.S_T.numel() * case.S_T.element_size()
-    if "e2e" in legs:
+    if run_head and "e2e" in legs:
+        keys = [k for k in ("q", "k", "v", "a", "b", "S0", "cu_seqlens") if host.get(k) is not None]
+        h2d = sum(host[k].numel() * host[k].element_size() for k in keys)
+        d2h = case.o.numel() * case.o.element_size() + case.S_T.numel() * case.S_T.element_size()
         pin = {k: host[k].pin_memory() for k in keys}
         nbuf = 2
         s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
@@ -473,7 +478,7 @@ def main():
 
     # ------------------------------------------------------------ CPU baseline (oracle)
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if run_head and rank == 0 and world == 1 and not args.no_cpu_baseline:
         v_cpu, cores, desc = cpu_baseline_sample(host, w, range(0, 16))
         cpu = {"value": v_cpu, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                "sample": desc}
@@ -481,7 +486,7 @@ def main():
 
     # ------------------------------------------------------------ the other prefill workloads
     workloads = {}
-    for leg, wk in (("kda", KDA), ("spread", SPREAD)):
+    for leg, wk in (("kda", KDA), ("spread", SPREAD), ("fast", synth.KDA_FAST)):
         if leg not in legs:
             continue
         c = PrefillCase(ops, wk, synth.make_prefill(wk, seed=rank), dev)

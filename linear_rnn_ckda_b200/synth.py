@@ -13,6 +13,8 @@ Distributions (N(mu, s): s is the standard deviation):
       "std"     N(4, 1)                    (KDA, gates near 1)
       "tiny"    N(0, 1.5)                  (about half of CKDA gates negative)
       "spread"  0.5 N(3,1) + 0.5 N(-3,1)   (spread initialisation, fair coin)
+      "fast"    N(-2, 1) on every fourth key channel (c % 4 == 0), N(4, 1) on the others
+                (fast-forgetting channels beside slow ones)
   * strength logits b, per (token, head):
       "std"     N(0, 1)
       "spread"  0.5 N(-2,0.5) + 0.5 N(2,0.5)
@@ -83,6 +85,10 @@ CKDA_SPREAD = Workload("ckda_spread_b8_t8192_h16_d128_c64", 8, 8192, 16, 128, 12
                        "spread", "spread", True)
 CKDA_VARLEN = Workload("ckda_varlen_h32_16x[512,8192]+65536_d128_c64", 1, 0, 32, 128, 128, 64, 1,
                        "spread", "spread", True, seq_lens=None)
+# KDA with a quarter of the key channels forgetting fast (a robustness workload, not one of the
+# pages' configurations)
+KDA_FAST = Workload("kda_fastforget_b4_t4096_h16_d128_c64", 4, 4096, 16, 128, 128, 64, 0,
+                    "fast", "std", False)
 DECODE = Workload("ckda_decode_b256_h32_d128_128steps", 256, 1, 32, 128, 128, 64, 1,
                   "spread", "spread", True, io_dtype="bf16", o_dtype="f32", decode_steps=128)
 
@@ -138,6 +144,11 @@ def _gate_logits(w: Workload, shape, seed: int, sub: int = 0):
     if w.gate == "spread":
         return _mixture_slabs(_rng(seed, _S_A, sub), _rng(seed, _S_ACOIN, sub), shape,
                               ((3.0, 1.0), (-3.0, 1.0)), w.io_dtype)
+    if w.gate == "fast":
+        out = _normal_slabs(_rng(seed, _S_A, sub), shape, 0.0, 1.0, "f32")   # z ~ N(0, 1)
+        mu = torch.full((shape[-1],), 4.0)
+        mu[0::4] = -2.0
+        return (out + mu).to(_DTYPES[w.io_dtype])
     raise ValueError(w.gate)
 
 

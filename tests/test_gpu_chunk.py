@@ -340,6 +340,14 @@ def test_tc_small_gate_logits(cuda_lib, sg):
     close(S, rS, TOL_BF16, "S_T")
 
 
+def test_tc_fast_forgetting_channels(cuda_lib):
+    """KDA gates with every fourth key channel forgetting fast (logits N(-2, 1)): most chunks
+    decay past the factorised path's range and run token by token on the tensor-core kernel's
+    state; the result matches the oracle whatever path each chunk took."""
+    w = synth.KDA_FAST.with_(B=2, T=400, H=2, o_dtype="f32")
+    check(cuda_lib, w, seed=16)
+
+
 @pytest.mark.parametrize("signed_gate", [3, 4], ids=["gate_range", "strength_range"])
 def test_single_range_variants(cuda_lib, signed_gate):
     """The gate range or the strength range widened alone (CKDA review, Figure 6) on both

@@ -93,3 +93,12 @@ def test_decode_inputs():
     assert d["q"].shape == (5, 4, 3, 128) and d["b"].shape == (5, 4, 3)
     assert d["S"].shape == (4, 3, 128, 128) and d["S"].dtype == torch.float32
     assert abs(f(d["S"]).std() - 0.02) < 1e-3
+
+
+def test_fast_forgetting_recipe():
+    """Every fourth key channel has logits N(-2, 1), the others N(4, 1)."""
+    w = synth.KDA_FAST.with_(B=1, T=2048, H=4, io_dtype="f32")
+    a = synth.make_prefill(w, seed=3)["a"].double()
+    fast, slow = a[..., 0::4], a[..., 1::4]
+    assert abs(fast.mean().item() + 2.0) < 0.02 and abs(fast.std().item() - 1.0) < 0.02
+    assert abs(slow.mean().item() - 4.0) < 0.02 and abs(slow.std().item() - 1.0) < 0.02
