@@ -110,10 +110,14 @@ extern "C" {
  *            32-bit coordinates); larger calls return CKDA_ERR_DIM.
  *   chunk   : 16, 32 or 64 tokens per chunk (a ragged last chunk is fine;
  *            chunks never span two sequences).
- *   workspace : device scratch of at least ckda_chunk_fwd_workspace_size()
- *            bytes, 256-byte aligned; owned by the caller, reused freely
- *            between calls on the same stream, never shared by two calls in
- *            flight at once.
+ *   workspace : device scratch, 256-byte aligned, of at least 256 bytes (the
+ *            status header); owned by the caller, reused freely between calls
+ *            on the same stream, never shared by two calls in flight at once.
+ *            With ckda_chunk_fwd_workspace_size() bytes, the tensor-core path
+ *            hands a (sequence, head) whose gates decay faster than its range
+ *            (a chunk product below 2^-100 in some channel) to a second launch
+ *            that carries per-channel references and stays on the tensor
+ *            cores; with less, such chunks run token by token (exact, slower).
  *   stream  : cudaStream_t.
  * Returns CKDA_OK or a negative CKDA_ERR_* code.
  */
@@ -123,9 +127,11 @@ int ckda_chunk_fwd(const void *q, const void *k, const void *v, const void *a, c
                    void *o, float *S_T, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
- * Bytes of workspace ckda_chunk_fwd needs for these sizes (same meaning as
- * there; n_seqs is ignored when the batch is not packed).  Pure host
- * arithmetic, no CUDA call.
+ * Bytes of workspace ckda_chunk_fwd uses in full for these sizes (same
+ * meaning as there; n_seqs is ignored when the batch is not packed): 256 for
+ * the exact path; for dk = dv = 128 and chunk 64 also a 16-byte queue entry
+ * and a 64 KB saved state per (sequence, head) for the hand-off above.  Pure
+ * host arithmetic, no CUDA call.
  */
 size_t ckda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int chunk,
                                      int n_seqs);
@@ -151,7 +157,8 @@ size_t ckda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int ch
  *   db    : [B, T, H] float32                   (all required, every row written)
  *   dS0   : [N, H, dk, dv] float32, or NULL (not written)
  *   workspace : device scratch of ckda_chunk_bwd_workspace_size() bytes (it holds
- *            the state and the state gradient at every chunk boundary), 256-byte
+ *            the state and the state gradient at every chunk boundary and each chunk's
+ *            state-independent factors), 256-byte
  *            aligned, owned by the caller; its status word is read with
  *            ckda_workspace_status (bad cu_seqlens: the sequence's gradients are
  *            not written).
@@ -191,9 +198,10 @@ int ckda_decode_step(const void *q, const void *k, const void *v, const void *a,
  * and has no device allocator.  Arguments, layouts and results are those of
  * ckda_chunk_fwd; the workspace is replaced by a fixed 4096-byte scratch array
  * compiled into the library (every GPU that loads the library holds it until
- * the process exits).  Sizes whose workspace would exceed 4096 bytes are
- * rejected with CKDA_ERR_WORKSPACE.  Neither this call nor the library calls
- * cudaMalloc or cudaFree.
+ * the process exits).  The scratch holds the status header only, so chunks
+ * whose gates decay past the tensor-core kernel's range run token by token
+ * (no hand-off).  Neither this call nor the library calls cudaMalloc or
+ * cudaFree.
  *   - Every call looks up the scratch array's device address
  *     (cudaGetSymbolAddress) with the caller's device current, so the address
  *     is never stale.  The first call on a device may load the library's

@@ -37,7 +37,6 @@ struct SimtParams {
   void *o;
   float *S_T;
   int *status;
-  float *S_chunks;   // optional: each chunk's incoming state (the backward's first pass)
   int n_seqs, T, H, dk, dv, C, dvs, signed_gate;
 };
 
@@ -106,17 +105,9 @@ __global__ void __launch_bounds__(kSimtThreads, 1) chunk_simt_kernel(SimtParams 
     sS[e] = p.S0 ? p.S0[sbase + (size_t)c * dv + j0 + j] : 0.f;
   }
 
-  const long slot0 = chunk_slot_base(p.cu, n, p.T, C);
   for (long cs = t0; cs < t1; cs += C) {
     const int nrows = (int)(t1 - cs < C ? t1 - cs : C);
     __syncthreads();
-    if (p.S_chunks) {
-      float *dst = p.S_chunks + ((size_t)(slot0 + (cs - t0) / C) * H + h) * dk * dv;
-      for (int e = tid; e < dk * dvs; e += kSimtThreads) {
-        const int c = e / dvs, j = e % dvs;
-        dst[(size_t)c * dv + j0 + j] = sS[e];
-      }
-    }
     // ---- load q, k, raw a (rows past the sequence end: q = k = 0, alpha = 1)
     for (int e = tid; e < C * dk; e += kSimtThreads) {
       const int r = e / dk, c = e % dk;
@@ -279,7 +270,7 @@ template <typename TIn, typename TOut>
 int launch_typed(const ChunkArgs &g, cudaStream_t stream) {
   SimtParams p;
   p.q = g.q; p.k = g.k; p.v = g.v; p.a = g.a; p.b = g.b; p.S0 = g.S0; p.cu = g.cu_seqlens;
-  p.o = g.o; p.S_T = g.S_T; p.status = g.status; p.S_chunks = g.S_chunks;
+  p.o = g.o; p.S_T = g.S_T; p.status = g.status;
   p.n_seqs = g.n_seqs; p.T = g.T; p.H = g.H; p.dk = g.dk; p.dv = g.dv; p.C = g.chunk;
   p.dvs = std::min(g.dv, 64);
   p.signed_gate = g.signed_gate;

@@ -25,10 +25,25 @@
 // tf32 (round-to-nearest) when written.  TMEM operands (S, U) are read as tf32
 // directly (the low mantissa bits ignored); V' is split so that none of it is
 // lost.  The gate products are the signed cumulative products in fp32
-// (the sign bit carries the gate-sign parity).  A chunk whose product falls
-// outside [2^-100, 2^100] in some channel (an exact zero gate, or extreme
-// decay) cannot use the factorisation Kr Kc^T; it is run token by token,
-// exactly, on the same TMEM-resident state (slow path).
+// (the sign bit carries the gate-sign parity).
+//
+// Range of the factorisation.  Kr Kc^T needs G_t and 1/G_t in fp32 for every row.
+// A channel whose chunk product stays above 2^-100 uses them as they are.  A
+// faster-decaying channel i carries a power-of-two reference R_i = 2^e_i, with e_i
+// half the channel's exponent sum over the chunk (exponents summed exactly, so no
+// product underflows on the way): Kr, Qr use G / R and Kc uses R / G, which leaves
+// A and P unchanged and keeps both factors within 2^+-110 for a chunk decay down
+// to 2^-220.  The state is then kept scaled, S^ = Diag(R) S, so that (a) and (d)
+// stay the same products:
+//   X = (Kr/R) S^,  O = (Qr/R) S^ + P U,  S^' = Diag(R') Diag(G_63 / R) (S^ + (Kc R)^T U)
+// with R' the next chunk's reference, applied after G_63 / R (their product can fall below
+// fp32's range while S' itself does not).  A
+// chunk that decays further in some channel is cut after its last row group of 8
+// that fits (the next chunk starts there); a chunk whose first 8 rows already do
+// not fit (an exact zero gate, a NaN, decay beyond 2^-126 in 8 rows) runs those
+// rows token by token, exactly, on the same TMEM-resident state (slow path).
+// Raw gates (which may exceed 1) keep the reference 1 and send a chunk outside
+// [2^-100, 2^100] to the slow path whole.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -97,6 +112,13 @@ struct TcParams {
   int inject_chunk;         // test hook: chunk index of the never-completing wait (-1: off)
   uint64_t inject_wait_ns;  // its bound
   const __nv_bfloat16 *a_head;  // per-head gate logits [rows, H] (CKDA_GATE_PER_HEAD), else NULL
+  // Hand-off of units whose gates decay past the plain kernel's range to the kernel with
+  // per-channel references (NULL: none, such chunks run token by token).  The plain kernel
+  // appends (sequence, head, first row, 0) to queue and the state at that row to saved_S
+  // ([entry][dk][dv]); the kernel with references takes entry blockIdx.x.
+  int *queue_count;
+  int4 *queue;
+  float *saved_S;
 };
 
 // byte offset of fp32 element (r, c) in a 128-byte-swizzled tile of R rows
@@ -128,6 +150,264 @@ __device__ __forceinline__ float fast_beta(float b, int form) {
   if (form == 1) return __fdividef(2.f, 1.f + __expf(-b));
   return b;
 }
+
+// 2^n as an fp32 number, built from its exponent field (n clamped to the normal range)
+__device__ __forceinline__ float exp2i(int n) {
+  n = n < -126 ? -126 : (n > 127 ? 127 : n);
+  return __uint_as_float((uint32_t)(n + 127) << 23);
+}
+
+// Bound on |log2| of the scaled gate factors G/R and R/G of a chunk (the reference R sits
+// halfway): a channel may decay by up to 2^-2kRefRange over one chunk.  The margin to fp32's
+// 2^-126 keeps a key component down to 2^-16 times a factor a normal number.
+constexpr int kRefRange = 110;
+
+// The gate products of one chunk are exchanged between the gate-pass threads as
+// xp[(x * 128 + ch) * 2 + {0, 1}]: the product of the gates of row group x (rows 8x .. 8x + 7) in
+// channel ch, and the product of their inverses.
+//
+// The reference exponent of a channel whose product over a chunk has the exponent sum etot
+// (summed exactly from its group products): none while the product stays above 2^-100, else
+// half the sum (toward zero), which centres G / R and R / G.
+__device__ __forceinline__ int ref_exponent(int etot) { return etot >= -100 ? 0 : -((-etot) >> 1); }
+
+// The references (e0, e1) of channels ch0, ch0 + 1 from the products of row groups 0 .. ng-1;
+// false if one of them, or its inverse, is not a normal number or a channel decays below
+// 2^-2kRefRange over those groups (no reference brings its factors within 2^+-kRefRange).
+__device__ __forceinline__ bool chunk_refs(const float *xp, int ch0, int ng, int &e0, int &e1) {
+  int es0 = 0, es1 = 0;
+  bool ok = true;
+#pragma unroll 1
+  for (int x = 0; x < ng; ++x) {
+    const float4 v = *reinterpret_cast<const float4 *>(xp + (x * 128 + ch0) * 2);
+    const int f0 = (int)((__float_as_uint(v.x) >> 23) & 255u);
+    const int i0 = (int)((__float_as_uint(v.y) >> 23) & 255u);
+    const int f1 = (int)((__float_as_uint(v.z) >> 23) & 255u);
+    const int i1 = (int)((__float_as_uint(v.w) >> 23) & 255u);
+    ok &= f0 >= 1 && f0 <= 254 && i0 >= 1 && i0 <= 254 && f1 >= 1 && f1 <= 254 && i1 >= 1 &&
+          i1 <= 254;
+    es0 += f0 - 127;
+    es1 += f1 - 127;
+  }
+  e0 = ref_exponent(es0);
+  e1 = ref_exponent(es1);
+  return ok && es0 >= -2 * kRefRange && es1 >= -2 * kRefRange;
+}
+
+// The first row group (8 if none) of channels ch0, ch0 + 1 whose product, or its inverse, is not
+// a normal number, or past which the chunk's exponent sum drops below -2kRefRange.
+__device__ __forceinline__ int first_failing_group(const float *xp, int ch0) {
+  int es0 = 0, es1 = 0;
+#pragma unroll 1
+  for (int x = 0; x < 8; ++x) {
+    const float4 v = *reinterpret_cast<const float4 *>(xp + (x * 128 + ch0) * 2);
+    const int e0 = (int)((__float_as_uint(v.x) >> 23) & 255u);
+    const int i0 = (int)((__float_as_uint(v.y) >> 23) & 255u);
+    const int e1 = (int)((__float_as_uint(v.z) >> 23) & 255u);
+    const int i1 = (int)((__float_as_uint(v.w) >> 23) & 255u);
+    es0 += e0 - 127;
+    es1 += e1 - 127;
+    const bool normal = e0 >= 1 && e0 <= 254 && i0 >= 1 && i0 <= 254 && e1 >= 1 && e1 <= 254 &&
+                        i1 >= 1 && i1 <= 254;
+    if (!normal || es0 < -2 * kRefRange || es1 < -2 * kRefRange) return x;
+  }
+  return 8;
+}
+
+// ---------------------------------------------------------------- the gate pass proper
+// Run by the 512 compute threads of a CTA on the chunk in the staging tiles: V^T into TMEM
+// (columns vcol..vcol+63), the Kr, Qr tile, Kc (returned in kc, stored later by the caller)
+// and G_63 / R (gc_out).  Thread (pair pc = tid % 64, row group rg = tid / 64) takes channels
+// 2pc, 2pc + 1 of rows 8rg .. 8rg + 7, reading bf16 pairs and writing 8-byte pairs; V^T keeps
+// the one-channel-per-lane mapping TMEM needs.  Returns whether a channel of this thread leaves
+// the range with the references e0, e1 it was given (R = 2^e for channels 2pc, 2pc + 1; 0: none).
+// (Everything is inline: an out-of-line call anywhere in the kernel costs the common path about
+// 15 %.)
+// the gate and (KDA, CKDA) its inverse, so that the second part needs no reciprocal:
+//   KDA   sigma(a) = 1 / (1 + e^{-a}), inverse 1 + e^{-a}
+//   CKDA  2 sigma(a) - 1 = tanh(a/2) = sign(a) (1 - e^{-|a|}) / (1 + e^{-|a|}), inverse the
+//         ratio upside down; both from one reciprocal r = 1 / (num den) (num r = 1 / den,
+//         den r = 1 / num).  Small |a|: 1 - e^{-|a|} cancels, an error at fp32 rounding level
+//         in absolute terms.  a = 0 gives 0 or NaN (0 inf): either fails the range check.
+template <int SG>
+__device__ __forceinline__ void gate_pair(float a, float &al, float &ial) {
+  if (SG == 0) {
+    const float e = __expf(-a);
+    ial = 1.f + e;
+    al = __fdividef(1.f, ial);
+  } else if (SG == 1) {
+    const float e = __expf(-fabsf(a));
+    const float num = 1.f - e, den = 1.f + e;
+    const float r = __fdividef(1.f, num * den);
+    al = copysignf(num * (num * r), a);
+    ial = copysignf(den * (den * r), a);
+  } else {
+    ial = 1.f;
+    al = a;
+  }
+}
+
+template <int SG, int FL>
+__device__ __forceinline__ bool gate_pass_body(uint8_t *sm, uint32_t tmem, int signed_gate,
+                                               int nrows, float b_this, __nv_bfloat16 a_this,
+                                               float *gc_out, uint32_t vcol, float (&kc)[16],
+                                               int e0, int e1) {
+  constexpr bool per_head = (FL & 1) != 0;
+  constexpr bool l2 = (FL & 2) != 0;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int qg = warp >> 2, c = 32 * (warp & 3) + lane;
+  const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+  const int pc = tid & 63, rg = tid >> 6, ch0 = 2 * pc;
+  uint8_t *sStg = sm + OFF_STG;
+  const uint8_t *stq = sStg, *stk = stq + 16384, *stv = stq + 32768, *sta = stq + 49152;
+  uint8_t *sKQ = sm + OFF_KQ;
+  float *sXp = reinterpret_cast<float *>(sm + OFF_KC);
+  float *sBeta = reinterpret_cast<float *>(sm + OFF_MISC);
+  __nv_bfloat16 *sAh = reinterpret_cast<__nv_bfloat16 *>(sm + OFF_MISC + 1408);
+  float *sInvQ = reinterpret_cast<float *>(sm + OFF_MISC + 1536), *sInvK = sInvQ + kC;
+  if (tid < kC) sBeta[tid] = tid < nrows ? fast_beta(b_this, beta_form(signed_gate)) : 0.f;
+  if (per_head && tid < kC) {
+    // the chunk's per-head gate logits (rows past the end: a gate of exactly 1)
+    sAh[tid] = tid < nrows ? a_this : __float2bfloat16_rn(SG == 2 ? 1.f : 100.f);
+  }
+  if (nrows < kC) {
+    // Rows past the sequence end (or a cut) hold other tokens or TMA fill.  They are
+    // overwritten in the staging copy with q = k = v = 0 and a gate of exactly 1
+    // (a = 100 gives sigma(a) = 2 sigma(a) - 1 = 1 in fp32; raw gates take a = 1), so
+    // the pass needs no per-row masking.
+    const uint32_t afill = SG == 2 ? 0x3F803F80u : 0x42C842C8u;   // bf16 pairs 1.0, 100.0
+    const int nt = (kC - nrows) * 16;   // 16-byte pieces of one array: 8 per row and box
+    for (int e = tid; e < 4 * nt; e += kCompute) {
+      const int x = e / nt, rem = e - x * nt;
+      const int row = nrows + (rem >> 4), piece = rem & 15;
+      const uint32_t f = x == 3 ? afill : 0u;
+      *reinterpret_cast<uint4 *>(sStg + x * 16384 + (piece >> 3) * 8192 + row * 128 +
+                                 (piece & 7) * 16) = make_uint4(f, f, f, f);
+    }
+    bar_sync(kBarC, kCompute);
+  } else if (per_head || l2) {
+    bar_sync(kBarC, kCompute);
+  }
+  if (l2) {
+    // 1 / ||q_r|| and 1 / ||k_r|| over the key channels: warp w takes rows w, w + 16, ...
+    // of q and of k, four channels per lane (8 bytes inside one 16-byte chunk); they are
+    // read after the exchange barrier below
+    for (int it = warp; it < 2 * kC; it += kCompute / 32) {
+      const int r = it % kC;
+      const uint8_t *tile = it < kC ? stq : stk;
+      const uint2 u = *reinterpret_cast<const uint2 *>(tile + swbf(r, 4 * lane));
+      const float x0 = __uint_as_float(u.x << 16), x1 = __uint_as_float(u.x & 0xFFFF0000u);
+      const float x2 = __uint_as_float(u.y << 16), x3 = __uint_as_float(u.y & 0xFFFF0000u);
+      float ss = fmaf(x0, x0, fmaf(x1, x1, fmaf(x2, x2, x3 * x3)));
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+      if (lane == 0) (it < kC ? sInvQ : sInvK)[r] = inv_norm(ss);
+    }
+  }
+  auto ldbf2 = [&](const uint8_t *tile, int r, float &x0, float &x1) {
+    const uint32_t u = *reinterpret_cast<const uint32_t *>(tile + swbf(r, ch0));
+    x0 = __uint_as_float(u << 16);
+    x1 = __uint_as_float(u & 0xFFFF0000u);
+  };
+  {
+    // lane c of TMEM holds V^T[c][.] (V' = V - X is formed in place before (c))
+    uint32_t vt[16];
+#pragma unroll
+    for (int rr = 0; rr < 16; ++rr) vt[rr] = __float_as_uint(ldbf(stv, 16 * qg + rr, c));
+    tmem_st16(lane_addr + vcol + 16 * qg, vt);
+  }
+  float g[16];   // [row][channel of the pair]; the inverse factors are formed from them
+  float run0 = 1.f, run1 = 1.f, irun0 = 1.f, irun1 = 1.f;
+#pragma unroll
+  for (int rr = 0; rr < 8; ++rr) {
+    float a0, a1, al0, al1, ial0, ial1;
+    if (per_head) {
+      a0 = a1 = __bfloat162float(sAh[8 * rg + rr]);
+    } else {
+      ldbf2(sta, 8 * rg + rr, a0, a1);
+    }
+    if (SG == 1) {
+      // the pair's CKDA ratios in packed fp32 pairs (same arithmetic as gate_pair)
+      const uint64_t one = f2pk(1.f, 1.f);
+      const uint64_t e = f2pk(__expf(-fabsf(a0)), __expf(-fabsf(a1)));
+      const uint64_t num = f2sub(one, e), den = f2add(one, e);
+      float p0, p1;
+      f2up(f2mul(num, den), p0, p1);
+      // the gate's sign rides on the shared reciprocal: num^2 r and den^2 r take it
+      const uint64_t rr2 = f2pk(copysignf(__fdividef(1.f, p0), a0),
+                                copysignf(__fdividef(1.f, p1), a1));
+      f2up(f2mul(num, f2mul(num, rr2)), al0, al1);
+      f2up(f2mul(den, f2mul(den, rr2)), ial0, ial1);
+    } else {
+      gate_pair<SG>(a0, al0, ial0);
+      gate_pair<SG>(a1, al1, ial1);
+    }
+    run0 *= al0;
+    run1 *= al1;
+    g[2 * rr] = run0;
+    g[2 * rr + 1] = run1;
+    if (SG != 2) {
+      irun0 *= ial0;
+      irun1 *= ial1;
+    }
+  }
+  *reinterpret_cast<float4 *>(sXp + (rg * 128 + ch0) * 2) = make_float4(run0, irun0, run1, irun1);
+  bar_sync(kBarC, kCompute);
+  // the row group's prefix factors G/R and R/G: products of the earlier row groups (of the
+  // gates and of their inverses), started at 1/R and R so that no partial product leaves fp32's
+  // range (G_t / R lies between 2^-e and G_63 / R)
+  float mult0 = exp2i(-e0), mult1 = exp2i(-e1), imult0 = exp2i(e0), imult1 = exp2i(e1);
+#pragma unroll
+  for (int x = 0; x < 7; ++x)
+    if (x < rg) {
+      const float4 v = *reinterpret_cast<const float4 *>(sXp + (x * 128 + ch0) * 2);
+      mult0 *= v.x;
+      imult0 *= v.y;
+      mult1 *= v.z;
+      imult1 *= v.w;
+    }
+  // each group's own product a normal number (below 2^-126 the running products lose bits)
+  bool bad = SG != 2 && !(fabsf(run0) >= 0x1p-126f && fabsf(run1) >= 0x1p-126f);
+#pragma unroll
+  for (int rr = 0; rr < 8; ++rr) {
+    const int r = 8 * rg + rr;
+    const float gam0 = g[2 * rr] * mult0, gam1 = g[2 * rr + 1] * mult1;
+    if (SG == 2) {
+      const float ag0 = fabsf(gam0), ag1 = fabsf(gam1);
+      bad |= !(ag0 >= 0x1p-100f && ag0 <= 0x1p100f && ag1 >= 0x1p-100f && ag1 <= 0x1p100f);
+    }
+    // R / G_t: the earlier groups' inverse product over this group's running product (a
+    // normal number, checked) -- one reciprocal, accurate to a few ulp like the product itself
+    const float inv0 = SG != 2 ? __fdividef(imult0, g[2 * rr]) : __fdividef(1.f, gam0);
+    const float inv1 = SG != 2 ? __fdividef(imult1, g[2 * rr + 1]) : __fdividef(1.f, gam1);
+    if (SG != 2 && rr == 7 && rg == 7) {
+      // |alpha| <= 1: G/R falls and R/G grows along the chunk, so the last row decides (a NaN
+      // gate reaches it too)
+      const float ag0 = fabsf(gam0), ag1 = fabsf(gam1), ai0 = fabsf(inv0), ai1 = fabsf(inv1);
+      bad |= !(ag0 >= 0x1p-110f && ag1 >= 0x1p-110f && ai0 <= 0x1p110f && ai1 <= 0x1p110f);
+    }
+    float q0, q1, k0, k1;
+    ldbf2(stq, r, q0, q1);
+    ldbf2(stk, r, k0, k1);
+    if (l2) {
+      const float iq = sInvQ[r], ik = sInvK[r];
+      q0 *= iq;
+      q1 *= iq;
+      k0 *= ik;
+      k1 *= ik;
+    }
+    *reinterpret_cast<uint2 *>(sKQ + sw32(128, r, ch0)) =
+        make_uint2(to_tf32(k0 * gam0), to_tf32(k1 * gam1));
+    *reinterpret_cast<uint2 *>(sKQ + sw32(128, 64 + r, ch0)) =
+        make_uint2(to_tf32(q0 * gam0), to_tf32(q1 * gam1));
+    kc[2 * rr] = __uint_as_float(to_tf32(k0 * inv0));
+    kc[2 * rr + 1] = __uint_as_float(to_tf32(k1 * inv1));
+    if (rr == 7 && rg == 7) *reinterpret_cast<float2 *>(gc_out + ch0) = make_float2(gam0, gam1);
+  }
+  tmem_wait_st();
+  return bad;
+}
+
 
 // Row stride (floats) of the plain A array: consecutive rows start 16 bytes
 // apart modulo 128, so 32 threads writing 16 bytes of 32 different rows hit
@@ -242,8 +522,10 @@ __device__ __forceinline__ int seq_of_length_rank(const int32_t *cu, int n_seqs,
   return sel;
 }
 
-// FL: bit 0 per-head gates (CKDA_GATE_PER_HEAD), bit 1 in-kernel q/k normalisation
-template <typename TOut, int SG, int FL>
+// FL: bit 0 per-head gates (CKDA_GATE_PER_HEAD), bit 1 in-kernel q/k normalisation.
+// REFS: the kernel that carries per-channel references (launched on the units the plain one
+// hands off); the plain kernel keeps every factor relative to the chunk start.
+template <typename TOut, int SG, int FL, bool REFS>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_a,
@@ -275,6 +557,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   // staging loads issued so far (by the issuer or compute thread 0); the compute warps count
   // the ones they consumed, so a unit that gives up knows whether one is still in flight
   unsigned int *sTmaIssued = reinterpret_cast<unsigned int *>(sm + OFF_MISC + 1400);
+  // length of the chunk being announced (compute warps -> issuer; chunks are cut short where
+  // a channel's gate product leaves the factorisation's range)
+  volatile int *sLen = reinterpret_cast<volatile int *>(sm + OFF_MISC + 1404);
   // per-head gate logits of the chunk in the gate pass (bf16, CKDA_GATE_PER_HEAD), and
   // 1 / ||q_r||, 1 / ||k_r|| of its rows (CKDA_QK_L2NORM)
   __nv_bfloat16 *sAh = reinterpret_cast<__nv_bfloat16 *>(sm + OFF_MISC + 1408);
@@ -286,27 +571,48 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = p.H;
-  const int unit = blockIdx.x, h = unit % H;
-  // CTAs start in blockIdx order: in a packed batch the longest sequences go first, so that
-  // the units with the longest serial chunk walk do not start last (ranking in the staging
-  // buffer, which no load has reached yet)
-  const int n = p.cu ? seq_of_length_rank(p.cu, p.n_seqs, unit / H, reinterpret_cast<int *>(sStg))
-                     : unit / H;
+  const int unit = blockIdx.x;
+  int n, h;
   long t0, t1, bofs;
-  if (p.cu) {
-    t0 = p.cu[n];
-    t1 = p.cu[n + 1];
-    bofs = 0;
-    if (t0 < 0 || t1 < t0 || t1 > p.T || (n == 0 && t0 != 0) || (n == p.n_seqs - 1 && t1 != p.T)) {
-      if (tid == 0) set_status(p.status, CKDA_ERR_SEQLENS);
-      return;
-    }
+  const float *s_init = p.S0;   // the state the unit starts from ([dk][dv] at s_init + s_init_ofs)
+  size_t sofs;
+  if constexpr (REFS) {
+    // a unit the plain kernel handed off: from its first row on, from the state it saved (this
+    // grid may start before the plain one has finished: wait for it, and for its writes)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (unit >= *p.queue_count) return;
+    const int4 e = p.queue[unit];
+    n = e.x;
+    h = e.y;
+    t0 = e.z;
+    t1 = p.cu ? p.cu[n + 1] : p.T;
+    bofs = p.cu ? 0 : (long)n * p.T;
+    s_init = p.saved_S + (size_t)unit * kD * kD;
+    sofs = ((size_t)n * H + h) * kD * kD;
   } else {
-    t0 = 0;
-    t1 = p.T;
-    bofs = (long)n * p.T;
+    h = unit % H;
+    // CTAs start in blockIdx order: in a packed batch the longest sequences go first, so that
+    // the units with the longest serial chunk walk do not start last (ranking in the staging
+    // buffer, which no load has reached yet)
+    n = p.cu ? seq_of_length_rank(p.cu, p.n_seqs, unit / H, reinterpret_cast<int *>(sStg))
+             : unit / H;
+    if (p.cu) {
+      t0 = p.cu[n];
+      t1 = p.cu[n + 1];
+      bofs = 0;
+      if (t0 < 0 || t1 < t0 || t1 > p.T || (n == 0 && t0 != 0) ||
+          (n == p.n_seqs - 1 && t1 != p.T)) {
+        if (tid == 0) set_status(p.status, CKDA_ERR_SEQLENS);
+        return;
+      }
+    } else {
+      t0 = 0;
+      t1 = p.T;
+      bofs = (long)n * p.T;
+    }
+    sofs = ((size_t)n * H + h) * kD * kD;
   }
-  const size_t sofs = ((size_t)n * H + h) * kD * kD;
+  const size_t s_init_ofs = REFS ? 0 : sofs;
   TOut *o = static_cast<TOut *>(p.o);
 
   if (tid == 0) {
@@ -360,25 +666,35 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t ph1 = 0, phs = 0, ph2 = 0, ph3 = 0, phr = 0;
       bool ok = true;
-      for (long cs = t0; cs < t1 && ok; cs += kC) {
-        // which path does this chunk take?
+      long cs = t0;
+      for (int ci = 0; cs < t1 && ok; ++ci) {
+        // which path does this chunk take, and how long is it?
         bool fast = false;
+        int len = 0;
         {
           const uint64_t w0 = globaltimer();
           for (;;) {
-            if (mbar_try_wait_sleep(rdy1, ph1, 2000)) { fast = true; ph1 ^= 1; break; }
+            if (mbar_try_wait_sleep(rdy1, ph1, 2000)) {
+              fast = true;
+              ph1 ^= 1;
+              len = *sLen;
+              break;
+            }
             if (mbar_try_wait(rdy_slow, phs)) {
               phs ^= 1;
+              len = *sLen;   // read before the acknowledgement frees the slot
               mbar_arrive(bar_ack);
               break;
             }
             if (*sAbort || globaltimer() - w0 > kWaitNs) { ok = false; break; }
           }
         }
-        if (!ok || !fast) continue;
+        if (!ok || len < 0) break;   // len < 0: the unit is handed off
+        cs += len;
+        if (!fast) continue;
         // (1) [A;P] = [Kr;Qr] Kc^T, and the staging load of the next chunk (staging is
         // free: this chunk's gate pass has consumed it)
-        if (cs + kC < t1) issue_tma(cs + kC);
+        if (cs < t1) issue_tma(cs);
         tc_fence_after();
 #pragma unroll
         for (int s = 0; s < 16; ++s) {
@@ -400,7 +716,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // (c) first step: U^T = V'^T Tb^T, hi and lo parts of V'
         if (!(ok = mbar_wait_or_abort(rdy3, ph3, kWaitNs, sAbort))) break;
         ph3 ^= 1;
-        const uint32_t vt_cur = (((cs - t0) / kC) & 1) ? COL_VT1 : COL_VT0;
+        const uint32_t vt_cur = (ci & 1) ? COL_VT1 : COL_VT0;
         tc_fence_after();
 #pragma unroll
         for (int s = 0; s < 8; ++s)
@@ -462,7 +778,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int jrow = 32 * (warp & 3) + lane;
     const int c = jrow;
     const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
-    uint32_t tma_ph = 0, mma1_ph = 0, a_ph = 0, d_ph = 0, ack_ph = 0, r4_ph = 0, never_ph = 0;
+    // phase bits of the barriers the compute warps wait on, packed (registers are the limit)
+    enum : int { PH_TMA = 0, PH_MMA1, PH_A, PH_D, PH_ACK, PH_R4, PH_NEVER };
+    uint32_t phs = 0;
     unsigned int tma_consumed = 0;   // staging loads whose completion the compute warps saw
     // bf16 O (16 KB per chunk) is staged in T's tile and written by one TMA store;
     // fp32 O is written directly from registers
@@ -473,17 +791,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     // warp 0 polls a completion barrier; the compute warps then agree on the outcome
     // (the phase advances only on success, so after a failure it still names the phase that
     // did not complete)
-    auto cwait_for = [&](uint64_t *bar, uint32_t &ph, uint64_t limit_ns) -> bool {
+    auto cwait_for = [&](uint64_t *bar, int bit, uint64_t limit_ns) -> bool {
       bool ok = true;
-      if (warp == 0) ok = mbar_wait_or_abort(bar, ph, limit_ns, sAbort);
+      if (warp == 0) ok = mbar_wait_or_abort(bar, (phs >> bit) & 1u, limit_ns, sAbort);
       ok = bar_and(kBarC, kCompute, ok);
       if (ok) {
-        ph ^= 1;
-        if (bar == bar_tma) ++tma_consumed;
+        phs ^= 1u << bit;
+        if (bit == PH_TMA) ++tma_consumed;
       }
       return ok;
     };
-    auto cwait = [&](uint64_t *bar, uint32_t &ph) -> bool { return cwait_for(bar, ph, kWaitNs); };
+    auto cwait = [&](uint64_t *bar, int bit) -> bool { return cwait_for(bar, bit, kWaitNs); };
     // one arrival per warp, after the whole warp's writes (each thread fenced its own)
     auto announce = [&](uint64_t *bar) {
       __syncwarp();
@@ -510,169 +828,112 @@ __global__ void __launch_bounds__(kThreads, 1)
     float *sXp = reinterpret_cast<float *>(sKC);   // [8][128][2] row-group products of the gates
                                                    // and of their inverses (the solve's A is
                                                    // dead whenever a gate pass runs)
-    auto ldbf2 = [&](const uint8_t *tile, int r, float &x0, float &x1) {
-      const uint32_t u = *reinterpret_cast<const uint32_t *>(tile + swbf(r, ch0));
-      x0 = __uint_as_float(u << 16);
-      x1 = __uint_as_float(u & 0xFFFF0000u);
+    // reference exponents of this thread's two channels in the last decided chunk (0: none)
+    int eref0 = 0, eref1 = 0;
+    auto gate_pass = [&](int nrows, float *gc_out, uint32_t vcol, float b_this,
+                         __nv_bfloat16 a_this, int e0, int e1) -> bool {
+      return gate_pass_body<SG, FL>(sm, tmem, p.signed_gate, nrows, b_this, a_this, gc_out, vcol,
+                                    kc, e0, e1);
     };
-    // the gate and (KDA, CKDA) its inverse, so that the second part needs no reciprocal:
-    //   KDA   sigma(a) = 1 / (1 + e^{-a}), inverse 1 + e^{-a}
-    //   CKDA  2 sigma(a) - 1 = tanh(a/2) = sign(a) (1 - e^{-|a|}) / (1 + e^{-|a|}), inverse the
-    //         ratio upside down; both from one reciprocal r = 1 / (num den) (num r = 1 / den,
-    //         den r = 1 / num).  Small |a|: 1 - e^{-|a|} cancels, an error at fp32 rounding level
-    //         in absolute terms.  a = 0 gives 0 or NaN (0 inf): either fails the range check.
-    auto gate2 = [&](float a, float &al, float &ial) {
-      if (SG == 0) {
-        const float e = __expf(-a);
-        ial = 1.f + e;
-        al = __fdividef(1.f, ial);
-      } else if (SG == 1) {
-        const float e = __expf(-fabsf(a));
-        const float num = 1.f - e, den = 1.f + e;
-        const float r = __fdividef(1.f, num * den);
-        al = copysignf(num * (num * r), a);
-        ial = copysignf(den * (den * r), a);
-      } else {
-        ial = 1.f;
-        al = a;
-      }
-    };
-    auto gate_core = [&](float *gc_out, uint32_t vcol) -> bool {
-      {
-        // lane c of TMEM holds V^T[c][.] (V' = V - X is formed in place before (c))
-        uint32_t vt[16];
-#pragma unroll
-        for (int rr = 0; rr < 16; ++rr) vt[rr] = __float_as_uint(ldbf(stv, 16 * qg + rr, c));
-        tmem_st16(lane_addr + vcol + 16 * qg, vt);
-      }
-      float g[16], ig[16];   // [row][channel of the pair]
-      float run0 = 1.f, run1 = 1.f, irun0 = 1.f, irun1 = 1.f;
-#pragma unroll
-      for (int rr = 0; rr < 8; ++rr) {
-        float a0, a1, al0, al1, ial0, ial1;
-        if (per_head) {
-          a0 = a1 = __bfloat162float(sAh[8 * rg + rr]);
-        } else {
-          ldbf2(sta, 8 * rg + rr, a0, a1);
-        }
-        if (SG == 1) {
-          // the pair's CKDA ratios in packed fp32 pairs (same arithmetic as gate2)
-          const uint64_t one = f2pk(1.f, 1.f);
-          const uint64_t e = f2pk(__expf(-fabsf(a0)), __expf(-fabsf(a1)));
-          const uint64_t num = f2sub(one, e), den = f2add(one, e);
-          float p0, p1;
-          f2up(f2mul(num, den), p0, p1);
-          // the gate's sign rides on the shared reciprocal: num^2 r and den^2 r take it
-          const uint64_t rr2 = f2pk(copysignf(__fdividef(1.f, p0), a0),
-                                    copysignf(__fdividef(1.f, p1), a1));
-          f2up(f2mul(num, f2mul(num, rr2)), al0, al1);
-          f2up(f2mul(den, f2mul(den, rr2)), ial0, ial1);
-        } else {
-          gate2(a0, al0, ial0);
-          gate2(a1, al1, ial1);
-        }
-        run0 *= al0;
-        run1 *= al1;
-        g[2 * rr] = run0;
-        g[2 * rr + 1] = run1;
-        if (SG != 2) {
-          irun0 *= ial0;
-          irun1 *= ial1;
-          ig[2 * rr] = irun0;
-          ig[2 * rr + 1] = irun1;
-        }
-      }
-      *reinterpret_cast<float4 *>(sXp + (rg * 128 + ch0) * 2) = make_float4(run0, irun0, run1, irun1);
-      csync();
-      // products of the earlier row groups (of the gates and of their inverses)
-      float mult0 = 1.f, mult1 = 1.f, imult0 = 1.f, imult1 = 1.f;
-#pragma unroll
-      for (int x = 0; x < 7; ++x)
-        if (x < rg) {
-          const float4 v = *reinterpret_cast<const float4 *>(sXp + (x * 128 + ch0) * 2);
-          mult0 *= v.x;
-          imult0 *= v.y;
-          mult1 *= v.z;
-          imult1 *= v.w;
-        }
-      bool bad = false;
-#pragma unroll
-      for (int rr = 0; rr < 8; ++rr) {
-        const int r = 8 * rg + rr;
-        const float gam0 = g[2 * rr] * mult0, gam1 = g[2 * rr + 1] * mult1;
-        if (SG == 2 || (rr == 7 && rg == 7)) {
-          const float ag0 = fabsf(gam0), ag1 = fabsf(gam1);
-          bad |= !(ag0 >= 0x1p-100f && ag0 <= 0x1p100f && ag1 >= 0x1p-100f && ag1 <= 0x1p100f);
-        }
-        const float inv0 = SG != 2 ? ig[2 * rr] * imult0 : __fdividef(1.f, gam0);
-        const float inv1 = SG != 2 ? ig[2 * rr + 1] * imult1 : __fdividef(1.f, gam1);
-        float q0, q1, k0, k1;
-        ldbf2(stq, r, q0, q1);
-        ldbf2(stk, r, k0, k1);
-        if (l2) {
-          const float iq = sInvQ[r], ik = sInvK[r];
-          q0 *= iq;
-          q1 *= iq;
-          k0 *= ik;
-          k1 *= ik;
-        }
-        *reinterpret_cast<uint2 *>(sKQ + sw32(128, r, ch0)) =
-            make_uint2(to_tf32(k0 * gam0), to_tf32(k1 * gam1));
-        *reinterpret_cast<uint2 *>(sKQ + sw32(128, 64 + r, ch0)) =
-            make_uint2(to_tf32(q0 * gam0), to_tf32(q1 * gam1));
-        kc[2 * rr] = __uint_as_float(to_tf32(k0 * inv0));
-        kc[2 * rr + 1] = __uint_as_float(to_tf32(k1 * inv1));
-        if (rr == 7 && rg == 7) *reinterpret_cast<float2 *>(gc_out + ch0) = make_float2(gam0, gam1);
-      }
-      tmem_wait_st();
-      return bad;
-    };
-    auto gate_pass = [&](long cs, int nrows, float *gc_out, uint32_t vcol) -> bool {
-      const float b_cur = b_next;
+    // The gate pass of the chunk starting at cs (at most nmax rows) and the chunk's length and
+    // path.  The pass first takes each channel's reference from the chunk before (gc_prev,
+    // its G_63 / R, and its references; NULL: none), the decay of a channel being much the
+    // same from chunk to chunk.  If a channel leaves the range, the references are taken from
+    // the chunk's own products and the pass runs again; if a channel decays too fast for any
+    // reference, the chunk is cut after its last row group of 8 that fits and the pass runs
+    // again on the shorter chunk (rows past the cut become padding); if not even the first
+    // group fits, the chunk is its first min(8, rows) rows on the token-by-token path.  Raw
+    // gates take no references and send an out-of-range chunk to that path whole.
+    int *sTrunc = reinterpret_cast<int *>(sKC + 8192);   // beside the exchange, in the dead A
+    // Chunk lengths follow the decay (kernel with references): the fastest channel's decay over
+    // the last chunk, in bits (sDecay[parity], a block-wide max), sets the next length to the
+    // largest multiple of 8 rows expected to decay by at most kTargetBits, so that a stationary
+    // decay needs neither a second pass nor a cut.
+    constexpr int kTargetBits = 190;
+    int *sDecay = reinterpret_cast<int *>(sm + OFF_MISC + 1384);   // [2]
+    int last_rows = kC, dpar = 0;
+    auto decide_chunk = [&](long cs, int nmax, float *gc_out, uint32_t vcol, const float *gc_prev,
+                            bool &slow_out) -> int {
+      const float b_this = b_next;
+      const __nv_bfloat16 a_this = a_next;
       if (tid < kC && cs + kC + tid < t1) b_next = p.b[(size_t)(bofs + cs + kC + tid) * H + h];
-      if (tid < kC) sBeta[tid] = tid < nrows ? fast_beta(b_cur, beta_form(p.signed_gate)) : 0.f;
-      if (per_head) {
-        // the chunk's per-head gate logits (rows past the end: a gate of exactly 1)
-        const __nv_bfloat16 a_cur = a_next;
-        if (tid < kC && cs + kC + tid < t1)
-          a_next = p.a_head[(size_t)(bofs + cs + kC + tid) * H + h];
-        if (tid < kC) sAh[tid] = tid < nrows ? a_cur : __float2bfloat16_rn(SG == 2 ? 1.f : 100.f);
-      }
-      if (nrows < kC) {
-        // Rows past the sequence end hold another sequence's tokens or TMA fill.  They are
-        // overwritten in the staging copy with q = k = v = 0 and a gate of exactly 1
-        // (a = 100 gives sigma(a) = 2 sigma(a) - 1 = 1 in fp32; raw gates take a = 1), so
-        // the pass needs no per-row masking.
-        const uint32_t afill = SG == 2 ? 0x3F803F80u : 0x42C842C8u;   // bf16 pairs 1.0, 100.0
-        const int nt = (kC - nrows) * 16;   // 16-byte pieces of one array: 8 per row and box
-        for (int e = tid; e < 4 * nt; e += kCompute) {
-          const int x = e / nt, rem = e - x * nt;
-          const int row = nrows + (rem >> 4), piece = rem & 15;
-          const uint32_t f = x == 3 ? afill : 0u;
-          *reinterpret_cast<uint4 *>(sStg + x * 16384 + (piece >> 3) * 8192 + row * 128 +
-                                     (piece & 7) * 16) = make_uint4(f, f, f, f);
+      if (per_head && tid < kC && cs + kC + tid < t1)
+        a_next = p.a_head[(size_t)(bofs + cs + kC + tid) * H + h];
+      int rows = nmax;
+      bool slow;
+      if constexpr (!REFS) {
+        slow = bar_or(kBarC, kCompute, gate_pass(rows, gc_out, vcol, b_this, a_this, 0, 0));
+      } else {
+        // the length from the last chunk's decay, and each channel's reference from its own
+        // decay over the last chunk, scaled to the new length
+        rows = nmax;
+        int e0 = 0, e1 = 0;
+        if (gc_prev) {
+          const int dmax = sDecay[dpar ^ 1];
+          if (dmax > kTargetBits * last_rows / kC) {
+            int want = (kTargetBits * last_rows / dmax) & ~7;
+            want = want < 8 ? 8 : (want > kC ? kC : want);
+            rows = rows < want ? rows : want;
+          }
+          const float2 gp = *reinterpret_cast<const float2 *>(gc_prev + ch0);
+          const int E0 = (int)((__float_as_uint(gp.x) >> 23) & 255u) - 127 + eref0;
+          const int E1 = (int)((__float_as_uint(gp.y) >> 23) & 255u) - 127 + eref1;
+          e0 = ref_exponent(E0 * rows / last_rows);
+          e1 = ref_exponent(E1 * rows / last_rows);
         }
-        csync();
-      } else if (per_head || l2) {
-        csync();
-      }
-      if (l2) {
-        // 1 / ||q_r|| and 1 / ||k_r|| over the key channels: warp w takes rows w, w + 16, ...
-        // of q and of k, four channels per lane (8 bytes inside one 16-byte chunk); they are
-        // read after the gate pass's exchange barrier
-        for (int it = warp; it < 2 * kC; it += kCompute / 32) {
-          const int r = it % kC;
-          const uint8_t *tile = it < kC ? stq : stk;
-          const uint2 u = *reinterpret_cast<const uint2 *>(tile + swbf(r, 4 * lane));
-          const float x0 = __uint_as_float(u.x << 16), x1 = __uint_as_float(u.x & 0xFFFF0000u);
-          const float x2 = __uint_as_float(u.y << 16), x3 = __uint_as_float(u.y & 0xFFFF0000u);
-          float ss = fmaf(x0, x0, fmaf(x1, x1, fmaf(x2, x2, x3 * x3)));
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-          if (lane == 0) (it < kC ? sInvQ : sInvK)[r] = inv_norm(ss);
+        if (tid == 0) sDecay[dpar] = 0;   // this chunk's slot (read a chunk ago)
+        bool cut = false, retried = false;
+        if (tid == 0) *sTrunc = kC;   // ordered before any update by the pass's exchange barrier
+#pragma unroll 1
+        for (;;) {
+          slow = bar_or(kBarC, kCompute, gate_pass(rows, gc_out, vcol, b_this, a_this, e0, e1));
+          if (!slow || SG == 2) break;
+          if (!retried) {
+            // references from the chunk's own products; a chunk they do not fit gets cut
+            retried = true;
+            if (bar_and(kBarC, kCompute, chunk_refs(sXp, ch0, (rows + 7) >> 3, e0, e1))) continue;
+          }
+          if (cut) break;   // the cut chunk failed again: token by token
+          const int fail = first_failing_group(sXp, ch0);
+          if (fail < 8) atomicMin(sTrunc, 8 * fail);
+          csync();
+          const int r = *sTrunc;   // read once per chunk (at most one cut)
+          if (r == 0) rows = rows < 8 ? rows : 8;   // the token-by-token path for these rows
+          if (r == 0 || r >= rows) break;
+          rows = r;   // the cut chunk: its references from its groups, and the pass again
+          cut = true;
+          chunk_refs(sXp, ch0, r >> 3, e0, e1);
         }
+        eref0 = e0;
+        eref1 = e1;
+        if (!slow && rg == 7) {
+          // the decay of this thread's channels over the chunk: the exponent of G_63 / R plus e
+          const float2 g = *reinterpret_cast<const float2 *>(gc_out + ch0);
+          const int d0 = 127 - (int)((__float_as_uint(g.x) >> 23) & 255u) - e0;
+          const int d1 = 127 - (int)((__float_as_uint(g.y) >> 23) & 255u) - e1;
+          atomicMax(&sDecay[dpar], d0 > d1 ? d0 : d1);
+        }
+        last_rows = rows;
+        dpar ^= 1;
       }
-      return gate_core(gc_out, vcol);
+      if (rows < nmax) {
+        // the next chunk starts at the cut: its logits replace the ones fetched a chunk ahead
+        if (tid < kC) b_next = cs + rows + tid < t1 ? p.b[(size_t)(bofs + cs + rows + tid) * H + h] : 0.f;
+        if (per_head && tid < kC && cs + rows + tid < t1)
+          a_next = p.a_head[(size_t)(bofs + cs + rows + tid) * H + h];
+      }
+      slow_out = slow;
+      return rows;
+    };
+    // The reference R of the chunk just decided (a fast one), per key channel, for the threads
+    // that scale the state by it.  Over the 1 / ||q||, 1 / ||k|| factors, which a fast chunk's
+    // gate pass has consumed by the time this is written (decide_chunk ends on a barrier) and
+    // which are next written by the following chunk's gate pass, after the scaling.  R is
+    // applied as a factor of its own: multiplied into G_63 / R of the chunk before, it would
+    // fall below fp32's range for a channel decaying by more than about 2^-150 over the two.
+    float *sRn = sInvQ;   // [128] (sInvQ and sInvK)
+    auto publish_ref = [&]() {
+      if (rg == 7) *reinterpret_cast<float2 *>(sRn + ch0) = make_float2(exp2i(eref0), exp2i(eref1));
     };
     auto store_kc_tile = [&]() {  // Kc (row t, channel pair)
 #pragma unroll
@@ -707,49 +968,100 @@ __global__ void __launch_bounds__(kThreads, 1)
       announce(is_slow ? rdy_slow : rdy1);
     };
 
+    // The plain kernel hands a unit whose chunk leaves its range (gates not raw) to the kernel
+    // with references, when the caller's workspace has room: the chunk is announced with
+    // length -1 (the issuer stops) and the unit saves its state and queues its first row.
+    const bool handoff = !REFS && SG != 2 && p.saved_S != nullptr;
+    bool handed_off = false;
+    auto len_word = [&](int len, bool slow_chunk) { return handoff && slow_chunk ? -1 : len; };
+
     // ---- initial state into TMEM: thread (lane j, qg) holds S^T[j][32*qg .. +32) = S0[i][j]
     {
       uint32_t r[32];
       const int i0 = 32 * qg;
 #pragma unroll
       for (int x = 0; x < 32; ++x)
-        r[x] = __float_as_uint(p.S0 ? p.S0[sofs + (size_t)(i0 + x) * kD + jrow] : 0.f);
+        r[x] = __float_as_uint(s_init ? s_init[s_init_ofs + (size_t)(i0 + x) * kD + jrow] : 0.f);
       tmem_st32(lane_addr + COL_S + i0, r);
       tmem_wait_st();
     }
     if (tid == 0 && t1 > t0) issue_tma(t0);
     csync();
 
+    // S^ = Diag(R) S in TMEM for the fast chunk just decided
+    auto scale_state_by_ref = [&]() {
+      publish_ref();
+      csync();
+      tc_fence_after();
+      uint32_t r[32];
+      const int i0 = 32 * qg;
+      tmem_ld32(lane_addr + COL_S + i0, r);
+      tmem_wait_ld();
+#pragma unroll
+      for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * sRn[i0 + x]);
+      tmem_st32(lane_addr + COL_S + i0, r);
+      tmem_wait_st();
+    };
+
     // gate pass of the first chunk
     int gsel = 0;              // sGC / V^T buffer of the chunk being processed
     bool slow = false;
+    int len = 0;               // rows of the chunk being processed, then of the next one
     if (t1 > t0) {
-      if (!cwait(bar_tma, tma_ph)) {
+      if (!cwait(bar_tma, PH_TMA)) {
         failed = true;
       } else {
-        const bool bad = gate_pass(t0, (int)(t1 - t0 < kC ? t1 - t0 : kC), sGC, COL_VT0);
+        len = decide_chunk(t0, (int)(t1 - t0 < kC ? t1 - t0 : kC), sGC, COL_VT0, nullptr, slow);
         store_kc();
-        slow = bar_or(kBarC, kCompute, bad);
+        if (REFS && !slow) scale_state_by_ref();
+        if (tid == 0) *sLen = len_word(len, slow);
         announce_chunk(slow);
         if (!slow) announce(rdy2);
       }
     }
 
-    for (long cs = t0; cs < t1 && !failed; cs += kC) {
-      const int nrows = (int)(t1 - cs < kC ? t1 - cs : kC);
-      const bool has_next = cs + kC < t1;
-      const int nrows_next = has_next ? (int)(t1 - cs - kC < kC ? t1 - cs - kC : kC) : 0;
+    long cs = t0, cs_next = t0;
+    int len_next = 0;
+    for (int ci = 0; cs < t1 && !failed; ++ci, cs = cs_next, len = len_next) {
+      const int nrows = len;
+      cs_next = cs + nrows;
+      const bool has_next = cs_next < t1;
+      const int nmax_next = has_next ? (int)(t1 - cs_next < kC ? t1 - cs_next : kC) : 0;
+      len_next = 0;
       float *gc_cur = sGC + 128 * gsel, *gc_next = sGC + 128 * (gsel ^ 1);
       const uint32_t vt_cur = gsel ? COL_VT1 : COL_VT0, vt_next = gsel ? COL_VT0 : COL_VT1;
 
-      if (p.inject_chunk >= 0 && (cs - t0) / kC == p.inject_chunk) {
+      if (p.inject_chunk >= 0 && ci == p.inject_chunk) {
         // test hook: a wait that runs out (nothing arrives on bar_never)
-        if (!cwait_for(bar_never, never_ph, p.inject_wait_ns ? p.inject_wait_ns : kWaitNs)) {
+        if (!cwait_for(bar_never, PH_NEVER, p.inject_wait_ns ? p.inject_wait_ns : kWaitNs)) {
           failed = true;
           break;
         }
       }
 
+      if (slow && handoff) {
+        // ------------------------------------------------------------ hand-off: the state (TMEM
+        // holds S itself: the plain kernel's factors are relative to the chunk start) and the
+        // row the kernel with references resumes at
+        int *sSlot = reinterpret_cast<int *>(sKC + 8192);
+        if (tid == 0) {
+          const int slot = atomicAdd(p.queue_count, 1);
+          *sSlot = slot;
+          p.queue[slot] = make_int4(n, h, (int)cs, 0);
+        }
+        csync();
+        const int slot = *sSlot;
+        tc_fence_after();
+        uint32_t r[32];
+        const int i0 = 32 * qg;
+        tmem_ld32(lane_addr + COL_S + i0, r);
+        tmem_wait_ld();
+        float *dst = p.saved_S + (size_t)slot * kD * kD;
+#pragma unroll
+        for (int x = 0; x < 32; ++x) dst[(size_t)(i0 + x) * kD + jrow] = __uint_as_float(r[x]);
+        handed_off = true;
+        break;
+      }
       if (slow) {
         // ------------------------------------------------------------ exact token-by-token path
         // state S[i][j] in smem over Kr/Qr, gates over Kc, partial sums over [P;Kc^T]; thread
@@ -814,12 +1126,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         csync();
         if (has_next) {
-          if (tid == 0) issue_tma(cs + kC);
-          if (!cwait(bar_tma, tma_ph)) { failed = true; break; }
-          const bool bad = gate_pass(cs + kC, nrows_next, gc_next, vt_next);
+          if (tid == 0) issue_tma(cs_next);
+          if (!cwait(bar_tma, PH_TMA)) { failed = true; break; }
+          len_next = decide_chunk(cs_next, nmax_next, gc_next, vt_next, nullptr, slow);
           store_kc();
-          slow = bar_or(kBarC, kCompute, bad);
-          if (!cwait(bar_ack, ack_ph)) { failed = true; break; }   // this chunk's announcement seen
+          if (REFS && !slow) scale_state_by_ref();   // this chunk left S unscaled
+          if (!cwait(bar_ack, PH_ACK)) { failed = true; break; }   // this chunk's announcement seen
+          if (tid == 0) *sLen = len_word(len_next, slow);
           announce_chunk(slow);
           if (!slow) announce(rdy2);
           gsel ^= 1;
@@ -831,7 +1144,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // issued by the issuer once this chunk was announced
       if (tid == 0 && store_pending) bulk_wait_read();  // previous O tile (over T) has left
       store_pending = false;
-      if (!cwait(bar_mma1, mma1_ph)) { failed = true; break; }
+      if (!cwait(bar_mma1, PH_MMA1)) { failed = true; break; }
       tc_fence_after();
       // ---------------------------------------------------------------- A and P out of TMEM
       float *sA = reinterpret_cast<float *>(sKC);           // plain [64][kAS]
@@ -876,7 +1189,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // round-to-nearest tf32 hi part (over V^T) and the fp32 remainder (over [A;P])
       bool ok = true;
       if (warp >= 4 && warp < 8) {
-        ok = mbar_wait_or_abort(bar_a, a_ph, kWaitNs, sAbort);
+        ok = mbar_wait_or_abort(bar_a, (phs >> PH_A) & 1u, kWaitNs, sAbort);
         tc_fence_after();
         if (ok) {
 #pragma unroll 1
@@ -901,7 +1214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (warp >= 8 && warp < 13) solve_T(sA, sT, sm + OFF_R2, sm + OFF_R34, sBeta, warp - 8, lane);
         if (warp < 4) solve_T_zeros(sT, tid);
       }
-      a_ph ^= 1;
+      phs ^= 1u << PH_A;
       fence_proxy_async();
       tc_fence_before();
       if (!bar_and(kBarC, kCompute, ok)) { failed = true; break; }
@@ -909,20 +1222,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---------------------------------------------------------------- next chunk's gate pass,
       // overlapping (c) and (d): Kr, Qr are free ((a) is done); Kc and Kc^T are stored
       // after (d)
-      bool bad_next = false;
       if (has_next) {
-        if (!cwait(bar_tma, tma_ph)) { failed = true; break; }
-        bad_next = gate_pass(cs + kC, nrows_next, gc_next, vt_next);
+        if (!cwait(bar_tma, PH_TMA)) { failed = true; break; }
+        len_next = decide_chunk(cs_next, nmax_next, gc_next, vt_next, gc_cur, slow);
+        if (REFS && !slow) publish_ref();   // for this chunk's end-of-chunk scaling
       }
       // the next chunk's Kc tile once (c) is done with the R tiles; then (1) of the next
       // chunk can run under this chunk's (d) and read-out.  Kc^T waits for (d).
-      if (!cwait(bar_r4, r4_ph)) { failed = true; break; }
+      if (!cwait(bar_r4, PH_R4)) { failed = true; break; }
       if (has_next) {
         store_kc_tile();
-        slow = bar_or(kBarC, kCompute, bad_next);
+        if (tid == 0) *sLen = len_word(len_next, slow);
         announce_chunk(slow);
       }
-      if (!cwait(bar_d, d_ph)) { failed = true; break; }
+      if (!cwait(bar_d, PH_D)) { failed = true; break; }
       tc_fence_after();
       if (has_next) store_kct_tile();
       // ---------------------------------------------------------------- O out; S^T columns scaled by G_63
@@ -948,13 +1261,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int i0 = 32 * qg;
         tmem_ld32(lane_addr + COL_S + i0, r);
         tmem_wait_ld();
+        // S' = (G_63 / R) S^, then S^ for the next chunk = R' S' (R' = 1 if it is token by
+        // token or there is none)
+        const bool rnext = REFS && has_next && !slow;
 #pragma unroll
         for (int x = 0; x < 32; x += 4) {
           const float4 gv = *reinterpret_cast<const float4 *>(gc_cur + i0 + x);
-          r[x] = __float_as_uint(__uint_as_float(r[x]) * gv.x);
-          r[x + 1] = __float_as_uint(__uint_as_float(r[x + 1]) * gv.y);
-          r[x + 2] = __float_as_uint(__uint_as_float(r[x + 2]) * gv.z);
-          r[x + 3] = __float_as_uint(__uint_as_float(r[x + 3]) * gv.w);
+          float4 rv = make_float4(1.f, 1.f, 1.f, 1.f);
+          if (rnext) rv = *reinterpret_cast<const float4 *>(sRn + i0 + x);
+          r[x] = __float_as_uint(__uint_as_float(r[x]) * gv.x * rv.x);
+          r[x + 1] = __float_as_uint(__uint_as_float(r[x + 1]) * gv.y * rv.y);
+          r[x + 2] = __float_as_uint(__uint_as_float(r[x + 2]) * gv.z * rv.z);
+          r[x + 3] = __float_as_uint(__uint_as_float(r[x + 3]) * gv.w * rv.w);
         }
         tmem_st32(lane_addr + COL_S + i0, r);
         tmem_wait_st();
@@ -972,14 +1290,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (tid == 0) bulk_wait_all();
 
-    tma_ph_out = tma_ph;
+    tma_ph_out = phs & 1u;
     tma_consumed_out = tma_consumed;
     if (failed) {
       if (tid == 0) {
         set_status(p.status, CKDA_ERR_TIMEOUT);
         *sAbort = 1;   // the issuer leaves its loop at its next wait
       }
-    } else if (p.S_T) {
+    } else if (p.S_T && !handed_off) {
       tc_fence_after();
       uint32_t r[32];
       const int i0 = 32 * qg;
@@ -1002,6 +1320,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  // the plain kernel's work is done: the launch of the kernel with references (programmatic
+  // dependent launch) may start once every CTA got here; it waits for this grid's completion
+  // before it reads the queue
+  if constexpr (!REFS) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
@@ -1045,12 +1367,14 @@ bool make_out_map(CUtensorMap *map, void *base, int H, long rows, bool bf16) {
              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Workspace of the hand-off (after the 256-byte header, whose word at byte 64 counts the queued
+// units): the queue, then the saved states.
+constexpr size_t kQueueCountOffset = 64;
+inline size_t handoff_queue_bytes(long units) { return ((size_t)units * 16 + 255) & ~(size_t)255; }
+
 template <typename TOut, int SG, int FL>
 int launch_typed(const ChunkArgs &g, cudaStream_t stream) {
   const long rows = (long)g.B * g.T;
-  if (rows == 0) {
-    // no tokens: S_T = S0 (or zero) is still produced by the kernel below
-  }
   CUtensorMap mq, mk, mv, ma, mo;
   const long map_rows = rows > 0 ? rows : 1;
   const bool per_head = per_head_gate(g.signed_gate);   // a is [rows, H]: no tile map
@@ -1066,15 +1390,50 @@ int launch_typed(const ChunkArgs &g, cudaStream_t stream) {
   p.inject_chunk = g.inject_chunk;
   p.inject_wait_ns = g.inject_wait_ns;
   p.a_head = per_head ? static_cast<const __nv_bfloat16 *>(g.a) : nullptr;
-  auto kern = chunk_tc_kernel<TOut, SG, FL>;
+  const long units = (long)g.n_seqs * g.H;
+  const bool handoff = SG != 2 && g.workspace &&
+                       g.workspace_bytes >= chunk_tc_handoff_bytes(g.n_seqs, g.H);
+  uint8_t *ws = static_cast<uint8_t *>(g.workspace);
+  p.queue_count = handoff ? reinterpret_cast<int *>(ws + kQueueCountOffset) : nullptr;
+  p.queue = handoff ? reinterpret_cast<int4 *>(ws + kWorkspaceHeader) : nullptr;
+  p.saved_S = handoff ? reinterpret_cast<float *>(ws + kWorkspaceHeader + handoff_queue_bytes(units))
+                      : nullptr;
+  auto kern = chunk_tc_kernel<TOut, SG, FL, false>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) !=
       cudaSuccess)
     return CKDA_ERR_CUDA;
-  kern<<<g.n_seqs * g.H, kThreads, kSmemBytes, stream>>>(mq, mk, mv, ma, mo, p);
-  return cudaGetLastError() == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
+  kern<<<(unsigned)units, kThreads, kSmemBytes, stream>>>(mq, mk, mv, ma, mo, p);
+  if (cudaGetLastError() != cudaSuccess) return CKDA_ERR_CUDA;
+  if constexpr (SG != 2) {
+    if (handoff) {
+      // the units handed off (CTAs past the queue's count return at once)
+      auto kern_r = chunk_tc_kernel<TOut, SG, FL, true>;
+      if (cudaFuncSetAttribute(kern_r, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)kSmemBytes) != cudaSuccess)
+        return CKDA_ERR_CUDA;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)units);
+      cfg.blockDim = dim3(kThreads);
+      cfg.dynamicSmemBytes = kSmemBytes;
+      cfg.stream = stream;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // launch early
+      attr[0].val.programmaticStreamSerializationAllowed = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      if (cudaLaunchKernelEx(&cfg, kern_r, mq, mk, mv, ma, mo, p) != cudaSuccess)
+        return CKDA_ERR_CUDA;
+    }
+  }
+  return CKDA_OK;
 }
 
 }  // namespace
+
+size_t chunk_tc_handoff_bytes(int n_seqs, int H) {
+  const long units = (long)n_seqs * H;
+  return kWorkspaceHeader + handoff_queue_bytes(units) + (size_t)units * kD * kD * sizeof(float);
+}
 
 bool chunk_tc_supported(const ChunkArgs &g) {
   return g.dk == kD && g.dv == kD && g.chunk == kC && g.io_dtype == CKDA_BF16 &&

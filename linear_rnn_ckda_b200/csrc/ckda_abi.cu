@@ -4,6 +4,7 @@
 // status read-back, which says so).
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <climits>
 #include <cstdint>
@@ -100,7 +101,10 @@ const char *ckda_status_string(int status) {
 int ckda_version(void) { return 100; }
 
 size_t ckda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int chunk, int n_seqs) {
-  (void)B; (void)T; (void)H; (void)dk; (void)dv; (void)chunk; (void)n_seqs;
+  (void)T;
+  const int N = n_seqs > 0 ? n_seqs : B;
+  if (dk == 128 && dv == 128 && chunk == 64 && N > 0 && H > 0)
+    return std::max(ckda::kWorkspaceHeader, ckda::chunk_tc_handoff_bytes(N, H));
   return ckda::kWorkspaceHeader;
 }
 
@@ -112,8 +116,10 @@ int ckda_chunk_fwd(const void *q, const void *k, const void *v, const void *a, c
                                             chunk, signed_gate, io_dtype, o_dtype, o, S_T);
   if (arg_rc != CKDA_OK) return arg_rc;
   const int N = cu_seqlens ? n_seqs : B;
-  const size_t need = ckda_chunk_fwd_workspace_size(B, T, H, dk, dv, chunk, n_seqs);
-  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+  // the header is the minimum; ckda_chunk_fwd_workspace_size() bytes also let fast-decaying
+  // gates stay on the tensor cores
+  if (!workspace || workspace_bytes < ckda::kWorkspaceHeader ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return CKDA_ERR_WORKSPACE;
   const int dev_rc = check_device();
   if (dev_rc != CKDA_OK) return dev_rc;
@@ -129,7 +135,6 @@ int ckda_chunk_fwd(const void *q, const void *k, const void *v, const void *a, c
   g.workspace_bytes = workspace_bytes;
   g.inject_chunk = g_inject_chunk.load(std::memory_order_relaxed);
   g.inject_wait_ns = g_inject_wait_ns.load(std::memory_order_relaxed);
-  g.S_chunks = nullptr;
   if (ckda::chunk_tc_supported(g)) return ckda::launch_chunk_tc(g, s);
   return ckda::launch_chunk_simt(g, s);
 }
@@ -139,7 +144,8 @@ size_t ckda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int n_
   const bool packed = n_seqs > 0;
   const long slots = ckda::chunk_slots(packed, packed ? 1 : B, (long)(packed ? T : T),
                                        packed ? n_seqs : B, ckda::bwd_chunk_rows());
-  return ckda::kWorkspaceHeader + 2 * (size_t)slots * H * dk * dv * sizeof(float);
+  const size_t per_slot_head = 2 * (size_t)dk * dv + ckda::bwd_record_floats(ckda::bwd_chunk_rows(), dk);
+  return ckda::kWorkspaceHeader + (size_t)slots * H * per_slot_head * sizeof(float);
 }
 
 int ckda_chunk_bwd(const void *q, const void *k, const void *v, const void *a, const float *b,
@@ -172,6 +178,7 @@ int ckda_chunk_bwd(const void *q, const void *k, const void *v, const void *a, c
   g.dO = dO; g.gq = dq; g.gk = dk_out; g.gv = dv_out; g.ga = da; g.gb = db; g.gS0 = dS0;
   g.S_chunks = base;
   g.dS_chunks = base + (size_t)slots * H * dk * dv;
+  g.rec = base + 2 * (size_t)slots * H * dk * dv;
   g.status = static_cast<int *>(workspace);
   g.n_seqs = N; g.B = B; g.T = T; g.H = H; g.dk = dk; g.dv = dv; g.signed_gate = signed_gate;
   g.io_dtype = io_dtype; g.do_dtype = do_dtype; g.n_slots = slots;

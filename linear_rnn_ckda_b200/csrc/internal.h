@@ -23,9 +23,6 @@ struct ChunkArgs {
   // tensor-core kernel waits on a barrier nothing arrives on (-1: off), and that wait's bound
   int inject_chunk;
   unsigned long long inject_wait_ns;
-  // backward only: the exact kernel saves every chunk's incoming state here,
-  // [slot][H][dk][dv] with slot = chunk_slot_base(sequence) + chunk index (NULL: not saved)
-  float *S_chunks;
 };
 
 struct DecodeArgs {
@@ -48,6 +45,10 @@ int launch_chunk_simt(const ChunkArgs &args, cudaStream_t stream);
 
 // Tensor-core chunkwise forward (tcgen05, dk = dv = 128, chunk 64, bf16 io).
 bool chunk_tc_supported(const ChunkArgs &args);
+// Workspace bytes that let the tensor-core kernel hand units whose gates decay past its range to
+// its variant with per-channel references (the header, a queue and one saved state per unit);
+// with less, such chunks run token by token.
+size_t chunk_tc_handoff_bytes(int n_seqs, int H);
 int launch_chunk_tc(const ChunkArgs &args, cudaStream_t stream);
 
 // First chunk slot of sequence n when chunks of C tokens of every sequence are numbered in one
@@ -69,11 +70,18 @@ struct BwdArgs {
   const void *dO;             // may be NULL (zero)
   float *gq, *gk, *gv, *ga, *gb, *gS0;   // gS0 may be NULL
   float *S_chunks, *dS_chunks;           // workspace: [n_slots][H][dk][dv] each
+  float *rec;                            // workspace: [n_slots][H][bwd_record_floats]
   int *status;
   int n_seqs, B, T, H, dk, dv, signed_gate, io_dtype, do_dtype;
   long n_slots;
 };
 int launch_chunk_bwd(const BwdArgs &args, cudaStream_t stream);
+// Floats of one (chunk slot, head) record of the backward: the chunk's state-independent
+// factors Kr, Kd, Qr ([C][dk] each), Li, P, M ([C][C] each), beta [C] and g [dk], rounded up
+// to 16 bytes.
+__host__ __device__ __forceinline__ long bwd_record_floats(int C, int dk) {
+  return (3L * C * dk + 3L * C * C + C + dk + 3) & ~3L;
+}
 int bwd_chunk_rows();   // the backward's chunk size (its saved states are every this many rows)
 
 // One decode step.  Returns a CKDA_* code.

@@ -45,8 +45,6 @@ extern "C" int ckda_chunk_fwd_noalloc(const void *q, const void *k, const void *
   const int arg_rc = ckda::check_chunk_args(q, k, v, a, b, S0, cu_seqlens, n_seqs, B, T, H, dk, dv,
                                             chunk, signed_gate, io_dtype, o_dtype, o, S_T);
   if (arg_rc != CKDA_OK) return arg_rc;
-  const size_t need = ckda_chunk_fwd_workspace_size(B, T, H, dk, dv, chunk, n_seqs);
-  if (need > kNoAllocScratchBytes) return CKDA_ERR_WORKSPACE;
   void *scratch = nullptr;
   const int rc = scratch_for_current_device(&scratch);
   if (rc != CKDA_OK) return rc;

@@ -170,6 +170,15 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, const void 
       "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
+// global -> smem copy of `bytes` contiguous bytes (both addresses 16-byte aligned, bytes a
+// multiple of 16), completing on an mbarrier's transaction count (no multicast)
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // the smem sources of every committed bulk store have been read
 __device__ __forceinline__ void bulk_wait_read() {

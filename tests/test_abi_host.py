@@ -61,8 +61,17 @@ def test_status_strings(lib):
 
 
 def test_workspace_size(lib):
-    assert lib.ckda_chunk_fwd_workspace_size(4, 4096, 16, 128, 128, 64, 0) >= 256
-    assert lib.ckda_chunk_fwd_workspace_size(1, 0, 1, 16, 16, 16, 0) >= 256
+    """The 256-byte header; for the tensor-core shapes also the hand-off's queue (16 bytes per
+    (sequence, head), rounded up to 256) and one fp32 128 x 128 state per (sequence, head)."""
+    assert lib.ckda_chunk_fwd_workspace_size(1, 0, 1, 16, 16, 16, 0) == 256
+    assert lib.ckda_chunk_fwd_workspace_size(2, 100, 3, 64, 64, 64, 0) == 256
+    assert lib.ckda_chunk_fwd_workspace_size(4, 4096, 16, 128, 128, 32, 0) == 256
+    units = 4 * 16
+    assert lib.ckda_chunk_fwd_workspace_size(4, 4096, 16, 128, 128, 64, 0) == \
+        256 + 1024 + units * 65536
+    units = 3 * 2   # packed: n_seqs sequences
+    assert lib.ckda_chunk_fwd_workspace_size(1, 1000, 2, 128, 128, 64, 3) == \
+        256 + 256 + units * 65536
 
 
 # Fake, aligned, never-dereferenced host addresses: every call below has exactly
@@ -240,8 +249,13 @@ def test_chunk_bwd_rejects(lib, kw, code):
 
 
 def test_bwd_workspace_size(lib):
-    """Two fp32 [slots][H][dk][dv] arrays (the state and its gradient at every 32-row chunk)
-    plus the 256-byte header; a packed batch allows one extra slot per sequence."""
-    per = 128 * 128 * 4 * 16
-    assert lib.ckda_chunk_bwd_workspace_size(4, 4096, 16, 128, 128, 0) == 256 + 2 * 512 * per
-    assert lib.ckda_chunk_bwd_workspace_size(1, 4096, 16, 128, 128, 3) == 256 + 2 * (128 + 4) * per
+    """Per 32-row chunk slot and head: the state and its gradient (fp32 [dk][dv] each) and the
+    chunk's record (Kr, Kd, Qr [32][dk], Li, P, M [32][32], beta [32], g [dk], fp32, rounded
+    to 16 bytes), plus the 256-byte header; a packed batch allows one extra slot per
+    sequence."""
+    rec = 3 * 32 * 128 + 3 * 32 * 32 + 32 + 128
+    per = (2 * 128 * 128 + rec) * 4 * 16
+    assert lib.ckda_chunk_bwd_workspace_size(4, 4096, 16, 128, 128, 0) == 256 + 512 * per
+    assert lib.ckda_chunk_bwd_workspace_size(1, 4096, 16, 128, 128, 3) == 256 + (128 + 4) * per
+    rec16 = (3 * 32 * 16 + 3 * 32 * 32 + 32 + 16 + 3) // 4 * 4
+    assert lib.ckda_chunk_bwd_workspace_size(1, 32, 1, 16, 48, 0) == 256 + (2 * 16 * 48 + rec16) * 4

@@ -341,11 +341,71 @@ def test_tc_small_gate_logits(cuda_lib, sg):
 
 
 def test_tc_fast_forgetting_channels(cuda_lib):
-    """KDA gates with every fourth key channel forgetting fast (logits N(-2, 1)): most chunks
-    decay past the factorised path's range and run token by token on the tensor-core kernel's
-    state; the result matches the oracle whatever path each chunk took."""
+    """KDA gates with every fourth key channel forgetting fast (logits N(-2, 1)): those
+    channels decay by about 2^-211 over a chunk, so they take a power-of-two reference and some
+    chunks are cut short; the result matches the oracle whatever each chunk did."""
     w = synth.KDA_FAST.with_(B=2, T=400, H=2, o_dtype="f32")
     check(cuda_lib, w, seed=16)
+
+
+@pytest.mark.parametrize("sg", [0, 1])
+def test_tc_range_cuts(cuda_lib, sg):
+    """Decay that leaves the factorisation's range at known row groups: gates of 2^-8 per row
+    in one channel (a chunk fits 24 rows), of 2^-20 (8 rows), of 2^-30 (not even 8 rows: token
+    by token), zero gates 0, 7, 8 and 63 rows apart, and stretches of ordinary gates between
+    them, so that chunks start at unaligned rows and the sequence ends inside a cut chunk.
+    Every row of o and S_T matches the oracle."""
+    T, H = 701, 2
+    rng = np.random.default_rng(60 + sg)
+    a = rng.standard_normal((1, T, H, 128)) * 0.5 + (3.0 if sg == 0 else 4.0)
+    if sg:
+        a *= np.where(rng.random(a.shape) < 0.5, 1.0, -1.0)
+
+    def logit(log2_alpha):  # a whose gate is 2^log2_alpha (KDA: sigma(a); CKDA: tanh(a/2))
+        x = 2.0 ** log2_alpha
+        return math.log(x / (1 - x)) if sg == 0 else 2 * math.atanh(x)
+
+    a[0, 0:300, 0, 3] = logit(-8)
+    a[0, 300:400, :, 7] = logit(-20)
+    a[0, 520:545, 1, 11] = logit(-30)
+    zero = -INF if sg == 0 else 0.0
+    for r in (448, 455, 456, 511):
+        a[0, r, r % 2, 9 + r % 5] = zero
+    a[0, 640:701, 0, 20] = logit(-8)      # a cut chunk runs into the end of the sequence
+    b = rng.standard_normal((1, T, H))
+    inp = _bf16_raw_case(T, a, b, seed=70 + sg)
+    w = synth.CKDA_SPREAD.with_(B=1, T=T, H=H, signed_gate=sg, o_dtype="f32")
+    o, S = run_gpu(cuda_lib, inp, w)
+    ro, rS = oracle_prefill(inp, sg)
+    close(o, ro, TOL_BF16, "o")
+    close(S, rS, TOL_BF16, "S_T")
+
+
+def test_tc_fast_forgetting_without_handoff(cuda_lib):
+    """With only the 256-byte workspace header there is no room for the hand-off to the kernel
+    with references: chunks past the plain kernel's range run token by token, exactly."""
+    w = synth.KDA_FAST.with_(B=2, T=200, H=2, o_dtype="f32")
+    inp = synth.make_prefill(w, seed=18)
+    d = to_device(inp)
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    o, S = cuda_lib.chunk_fwd(d["q"], d["k"], d["v"], d["a"], d["b"], d["S0"], None, chunk=64,
+                              signed_gate=w.signed_gate, o_dtype=torch.float32, workspace=ws)
+    torch.cuda.synchronize()
+    ro, rS = oracle_prefill(inp, w.signed_gate)
+    close(o, ro, TOL_BF16, "o")
+    close(S, rS, TOL_BF16, "S_T")
+
+
+def test_tc_fast_forgetting_varlen_alias(cuda_lib):
+    """The fast-forgetting gates in a packed batch (cut chunks cross no sequence boundary)
+    with S_T written over S0."""
+    lens = (0, 1, 63, 64, 65, 200, 7, 333)
+    w = synth.KDA_FAST.with_(B=1, H=2, seq_lens=lens, T=sum(lens), o_dtype="f32")
+    inp = synth.make_prefill(w, seed=17)
+    ro, rS = oracle_prefill(inp, w.signed_gate)
+    o, S = run_gpu(cuda_lib, inp, w, S0_alias=True)
+    close(o, ro, TOL_BF16, "o")
+    close(S, rS, TOL_BF16, "S_T")
 
 
 @pytest.mark.parametrize("signed_gate", [3, 4], ids=["gate_range", "strength_range"])

@@ -91,6 +91,14 @@ def test_tensor_core_varlen_per_head(cuda_lib):
     _fwd_check(cuda_lib, w, seed=31, flags=PH | L2, tol=TOL_BF16)
 
 
+@pytest.mark.parametrize("flags", [PH, PH | L2], ids=["per_head", "both"])
+def test_tensor_core_per_head_fast_decay(cuda_lib, flags):
+    """A per-head gate that forgets fast (the fast channel's logits, N(-2, 1)): every key
+    channel decays by about 2^-211 per chunk, so all take a reference and chunks are cut."""
+    w = synth.KDA_FAST.with_(B=2, T=300, H=3)
+    _fwd_check(cuda_lib, w, seed=32, flags=flags, tol=TOL_BF16)
+
+
 @pytest.mark.parametrize("flags", [PH, L2, PH | L2], ids=["per_head", "l2norm", "both"])
 @pytest.mark.parametrize("io", ["f32", "bf16"])
 def test_decode(cuda_lib, flags, io):
