@@ -247,7 +247,7 @@ __device__ __forceinline__ void gate_pair(float a, float &al, float &ial) {
   }
 }
 
-template <int SG, int FL>
+template <int SG, int FL, bool REFS>
 __device__ __forceinline__ bool gate_pass_body(uint8_t *sm, uint32_t tmem, int signed_gate,
                                                int nrows, float b_this, __nv_bfloat16 a_this,
                                                float *gc_out, uint32_t vcol, float (&kc)[16],
@@ -316,7 +316,10 @@ __device__ __forceinline__ bool gate_pass_body(uint8_t *sm, uint32_t tmem, int s
     for (int rr = 0; rr < 16; ++rr) vt[rr] = __float_as_uint(ldbf(stv, 16 * qg + rr, c));
     tmem_st16(lane_addr + vcol + 16 * qg, vt);
   }
-  float g[16];   // [row][channel of the pair]; the inverse factors are formed from them
+  // [row][channel of the pair]: the gates' running products within the row group and (plain
+  // kernel) those of their inverses; the kernel with references, which runs closer to the
+  // register limit, forms the inverse factors from g by one reciprocal each instead
+  float g[16], ig[REFS ? 1 : 16];
   float run0 = 1.f, run1 = 1.f, irun0 = 1.f, irun1 = 1.f;
 #pragma unroll
   for (int rr = 0; rr < 8; ++rr) {
@@ -349,6 +352,10 @@ __device__ __forceinline__ bool gate_pass_body(uint8_t *sm, uint32_t tmem, int s
     if (SG != 2) {
       irun0 *= ial0;
       irun1 *= ial1;
+      if constexpr (!REFS) {
+        ig[2 * rr] = irun0;
+        ig[2 * rr + 1] = irun1;
+      }
     }
   }
   *reinterpret_cast<float4 *>(sXp + (rg * 128 + ch0) * 2) = make_float4(run0, irun0, run1, irun1);
@@ -376,10 +383,20 @@ __device__ __forceinline__ bool gate_pass_body(uint8_t *sm, uint32_t tmem, int s
       const float ag0 = fabsf(gam0), ag1 = fabsf(gam1);
       bad |= !(ag0 >= 0x1p-100f && ag0 <= 0x1p100f && ag1 >= 0x1p-100f && ag1 <= 0x1p100f);
     }
-    // R / G_t: the earlier groups' inverse product over this group's running product (a
-    // normal number, checked) -- one reciprocal, accurate to a few ulp like the product itself
-    const float inv0 = SG != 2 ? __fdividef(imult0, g[2 * rr]) : __fdividef(1.f, gam0);
-    const float inv1 = SG != 2 ? __fdividef(imult1, g[2 * rr + 1]) : __fdividef(1.f, gam1);
+    // R / G_t: the earlier groups' inverse product times this group's inverse running product
+    // (or, with references, over this group's running product -- a normal number, checked --
+    // by one reciprocal, accurate to a few ulp like the product itself)
+    float inv0, inv1;
+    if constexpr (SG == 2) {
+      inv0 = __fdividef(1.f, gam0);
+      inv1 = __fdividef(1.f, gam1);
+    } else if constexpr (REFS) {
+      inv0 = __fdividef(imult0, g[2 * rr]);
+      inv1 = __fdividef(imult1, g[2 * rr + 1]);
+    } else {
+      inv0 = ig[2 * rr] * imult0;
+      inv1 = ig[2 * rr + 1] * imult1;
+    }
     if (SG != 2 && rr == 7 && rg == 7) {
       // |alpha| <= 1: G/R falls and R/G grows along the chunk, so the last row decides (a NaN
       // gate reaches it too)
@@ -832,8 +849,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int eref0 = 0, eref1 = 0;
     auto gate_pass = [&](int nrows, float *gc_out, uint32_t vcol, float b_this,
                          __nv_bfloat16 a_this, int e0, int e1) -> bool {
-      return gate_pass_body<SG, FL>(sm, tmem, p.signed_gate, nrows, b_this, a_this, gc_out, vcol,
-                                    kc, e0, e1);
+      return gate_pass_body<SG, FL, REFS>(sm, tmem, p.signed_gate, nrows, b_this, a_this, gc_out,
+                                          vcol, kc, e0, e1);
     };
     // The gate pass of the chunk starting at cs (at most nmax rows) and the chunk's length and
     // path.  The pass first takes each channel's reference from the chunk before (gc_prev,
