@@ -401,8 +401,10 @@ def main():
         case.check("the headline leg")
         ms_step = ms / args.steps
         value = tokens * args.steps / (ms / 1000.0)
-        # dominant kernel: the chunk kernel, one launch per step (the 256-byte status memset
-        # before it is included, < 2 us)
+        # dominant kernel: the chunk kernel.  A step is two launches (the 256-byte status memset
+        # before them is included, < 2 us): the plain tensor-core kernel, then the kernel with
+        # per-channel references for the units it handed off (none here: its CTAs return at once,
+        # ~6 us with the programmatic dependent launch)
         roofline = prefill_roofline(w, ms_step, peaks, "chunk_tc_kernel/" + w.name)
 
     # ------------------------------------------------------------ e2e (host buffers)
@@ -582,7 +584,7 @@ def main():
             "config": headline_config(w),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "workloads": workloads, "fwd_bwd": fwd_bwd, "decode": decode_obj,
-            "gpu_launches": args.steps, "clocks": clocks, "peaks_source": peaks["source"],
+            "gpu_launches": 2 * args.steps, "clocks": clocks, "peaks_source": peaks["source"],
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -59,7 +59,7 @@ constexpr int kBC = 32;          // backward chunk rows
 constexpr int kBThreads = 256;   // the state passes
 constexpr int kGThreads = 512;   // the record and gradient passes (one chunk per block)
 constexpr int kJS = 32;          // value columns per slice in the gradient pass
-constexpr int kJP = kJS + 1;     // their row stride (threads that differ in the row hit distinct banks)
+constexpr int kJP = kJS + 4;     // their row stride: 16-byte rows that start on distinct 16-byte bank groups
 constexpr int kBP = kBC + 1;     // row stride of the gradient pass's [kBC][kBC] arrays (the same)
 constexpr uint64_t kWaitNs = 2000000000ull;   // bound on a record copy's wait (2 s)
 
@@ -139,11 +139,11 @@ __device__ __forceinline__ bool slot_chunk(const BwdParams &p, long slot, int &n
 //   sBeta  [kBC], sGC [dk] = g (exact), sLC [dk], sZC [dk]
 //   (CKDA_QK_L2NORM: q and k divided by their norms; the factors go to sInvQ / sInvK)
 template <typename TIn>
-__device__ void load_chunk(const BwdParams &p, long row0, int nrows, int h, float *sQ, float *sK,
-                           float *sL, uint8_t *sZ, float *sBeta, float *sGC, float *sLC, int *sZC,
-                           float *sInvQ, float *sInvK) {
+__device__ void load_chunk(const BwdParams &p, long row0, int nrows, int h, int ldk, float *sQ,
+                           float *sK, float *sL, uint8_t *sZ, float *sBeta, float *sGC, float *sLC,
+                           int *sZC, float *sInvQ, float *sInvK) {
   const bool per_head = per_head_gate(p.signed_gate);
-  const int dk = p.dk, ldk = dk + 1, ldz = dk + 4, H = p.H, tid = threadIdx.x;
+  const int dk = p.dk, ldz = dk + 4, H = p.H, tid = threadIdx.x;
   const TIn *q = static_cast<const TIn *>(p.q);
   const TIn *k = static_cast<const TIn *>(p.k);
   const TIn *a = static_cast<const TIn *>(p.a);
@@ -288,7 +288,8 @@ __global__ void __launch_bounds__(kGThreads) bwd_prep_kernel(BwdParams p) {
   if (!slot_chunk(p, slot, n, t0, t1, bofs, ci)) return;
   const long cs = t0 + ci * kBC;
   const int nrows = (int)(t1 - cs < kBC ? t1 - cs : kBC);
-  load_chunk<TIn>(p, bofs + cs, nrows, h, sQ, sK, sL, sZ, sBeta, sGC, sLC, sZC, sInv, sInv + kBC);
+  load_chunk<TIn>(p, bofs + cs, nrows, h, ldk, sQ, sK, sL, sZ, sBeta, sGC, sLC, sZC, sInv,
+                  sInv + kBC);
   pair_products(dk, sQ, sK, sL, sZ, sM, sP);
   // warp 0 inverts while the others write the gated rows
   if (tid < 32) unit_lower_inverse_warp(sM, sBeta, sLi);
@@ -614,7 +615,9 @@ __global__ void __launch_bounds__(kBThreads) bwd_state_rev_kernel(BwdParams p) {
 template <typename TIn, typename TG>
 __global__ void __launch_bounds__(kGThreads, 1) bwd_grad_kernel(BwdParams p) {
   extern __shared__ float smem[];
-  const int dk = p.dk, dv = p.dv, ldk = dk + 1, ldz = dk + 4, H = p.H, tid = threadIdx.x;
+  // rows of dk + 8 floats: the gate gradient's four threads per channel read rows t = 4i + sub,
+  // which then fall on distinct banks for the eight channels of a warp
+  const int dk = p.dk, dv = p.dv, ldk = dk + 8, ldz = dk + 4, H = p.H, tid = threadIdx.x;
   float *sQ = smem;                                   // [kBC][ldk] q
   float *sK = sQ + kBC * ldk;                         // [kBC][ldk] k
   float *sL = sK + kBC * ldk;                         // [kBC][ldk] gate prefix
@@ -663,7 +666,7 @@ __global__ void __launch_bounds__(kGThreads, 1) bwd_grad_kernel(BwdParams p) {
   const float *dSo = p.dS_out + ((size_t)slot * H + h) * dk * dv;
 
   const bool per_head = per_head_gate(p.signed_gate), l2 = qk_l2norm(p.signed_gate);
-  load_chunk<TIn>(p, row0, nrows, h, sQ, sK, sL, sZ, sBeta, sGC, sLC, sZC, sInvQ, sInvK);
+  load_chunk<TIn>(p, row0, nrows, h, ldk, sQ, sK, sL, sZ, sBeta, sGC, sLC, sZC, sInvQ, sInvK);
   for (int r = tid; r < kBC; r += kGThreads) sDaRow[r] = 0.f;
   // M, P, Li, Kr and Kd from the chunk's record
   const RecLayout R = rec_layout(dk);
@@ -766,7 +769,7 @@ __global__ void __launch_bounds__(kGThreads, 1) bwd_grad_kernel(BwdParams p) {
     }
     __syncthreads();
     // sums over this slice's value columns: rows r0, r0 + 1 and the key channels
-    // cl, cl + 32, cl + 64, cl + 96 per thread
+    // cl, cl + 32, cl + 64, cl + 96 per thread, four columns per step (16-byte loads)
     for (int ti = tid; ti < (kBC / 2) * 32; ti += kGThreads) {
       const int r0 = 2 * (ti >> 5), cl = ti & 31;
       float akd[2][4], aqr[2][4], akr[2][4];
@@ -774,21 +777,31 @@ __global__ void __launch_bounds__(kGThreads, 1) bwd_grad_kernel(BwdParams p) {
       for (int y = 0; y < 2; ++y)
 #pragma unroll
         for (int x = 0; x < 4; ++x) akd[y][x] = aqr[y][x] = akr[y][x] = 0.f;
-      for (int j = 0; j < js; ++j) {
-        const float u0 = sU[r0 * kJP + j], u1 = sU[(r0 + 1) * kJP + j];
-        const float o0 = sdO[r0 * kJP + j], o1 = sdO[(r0 + 1) * kJP + j];
-        const float w0 = sdV[r0 * kJP + j], w1 = sdV[(r0 + 1) * kJP + j];
+      for (int j = 0; j < js; j += 4) {
+        const float4 u0 = *reinterpret_cast<const float4 *>(sU + r0 * kJP + j);
+        const float4 u1 = *reinterpret_cast<const float4 *>(sU + (r0 + 1) * kJP + j);
+        const float4 o0 = *reinterpret_cast<const float4 *>(sdO + r0 * kJP + j);
+        const float4 o1 = *reinterpret_cast<const float4 *>(sdO + (r0 + 1) * kJP + j);
+        const float4 w0 = *reinterpret_cast<const float4 *>(sdV + r0 * kJP + j);
+        const float4 w1 = *reinterpret_cast<const float4 *>(sdV + (r0 + 1) * kJP + j);
+        const float ua[2][4] = {{u0.x, u0.y, u0.z, u0.w}, {u1.x, u1.y, u1.z, u1.w}};
+        const float oa[2][4] = {{o0.x, o0.y, o0.z, o0.w}, {o1.x, o1.y, o1.z, o1.w}};
+        const float wa[2][4] = {{w0.x, w0.y, w0.z, w0.w}, {w1.x, w1.y, w1.z, w1.w}};
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
           const int c = cl + 32 * x;
           if (c < dk) {
-            const float sv = sS[c * kJP + j], dsv = sdS[c * kJP + j];
-            akd[0][x] = fmaf(u0, dsv, akd[0][x]);
-            akd[1][x] = fmaf(u1, dsv, akd[1][x]);
-            aqr[0][x] = fmaf(o0, sv, aqr[0][x]);
-            aqr[1][x] = fmaf(o1, sv, aqr[1][x]);
-            akr[0][x] = fmaf(-w0, sv, akr[0][x]);
-            akr[1][x] = fmaf(-w1, sv, akr[1][x]);
+            const float4 sv = *reinterpret_cast<const float4 *>(sS + c * kJP + j);
+            const float4 dv4 = *reinterpret_cast<const float4 *>(sdS + c * kJP + j);
+            const float sa[4] = {sv.x, sv.y, sv.z, sv.w}, da[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+              for (int y = 0; y < 2; ++y) {
+                akd[y][x] = fmaf(ua[y][i], da[i], akd[y][x]);
+                aqr[y][x] = fmaf(oa[y][i], sa[i], aqr[y][x]);
+                akr[y][x] = fmaf(-wa[y][i], sa[i], akr[y][x]);
+              }
           }
         }
       }
@@ -808,16 +821,24 @@ __global__ void __launch_bounds__(kGThreads, 1) bwd_grad_kernel(BwdParams p) {
       const int r = e / kBC, m = e % kBC;
       if (m > r) continue;
       float adp = 0.f, adt = 0.f;
-      for (int j = 0; j < js; ++j) {
-        adp = fmaf(sdO[r * kJP + j], sU[m * kJP + j], adp);
-        adt = fmaf(sdU[r * kJP + j], sVp[m * kJP + j], adt);
+      for (int j = 0; j < js; j += 4) {
+        const float4 o = *reinterpret_cast<const float4 *>(sdO + r * kJP + j);
+        const float4 u = *reinterpret_cast<const float4 *>(sU + m * kJP + j);
+        const float4 du = *reinterpret_cast<const float4 *>(sdU + r * kJP + j);
+        const float4 vp = *reinterpret_cast<const float4 *>(sVp + m * kJP + j);
+        adp = fmaf(o.x, u.x, fmaf(o.y, u.y, fmaf(o.z, u.z, fmaf(o.w, u.w, adp))));
+        adt = fmaf(du.x, vp.x, fmaf(du.y, vp.y, fmaf(du.z, vp.z, fmaf(du.w, vp.w, adt))));
       }
       sdP[r * kBP + m] += adp;
       sdT[r * kBP + m] += adt;
     }
     for (int c = tid; c < dk; c += kGThreads) {
       float acc = 0.f;
-      for (int j = 0; j < js; ++j) acc = fmaf(sdS[c * kJP + j], sS[c * kJP + j], acc);
+      for (int j = 0; j < js; j += 4) {
+        const float4 a4 = *reinterpret_cast<const float4 *>(sdS + c * kJP + j);
+        const float4 b4 = *reinterpret_cast<const float4 *>(sS + c * kJP + j);
+        acc = fmaf(a4.x, b4.x, fmaf(a4.y, b4.y, fmaf(a4.z, b4.z, fmaf(a4.w, b4.w, acc))));
+      }
       sCarry[c] += acc;
     }
     __syncthreads();
@@ -1011,7 +1032,7 @@ size_t state_rev_smem(int dk, int dvs) {
   return sizeof(float) * (2 * (size_t)rec_layout(dk).m + (size_t)dk * dvs + 3 * kBC * dvs) + 16;
 }
 size_t grad_smem(int dk) {
-  const int ldk = dk + 1, ldz = dk + 4;
+  const int ldk = dk + 8, ldz = dk + 4;
   return sizeof(float) * ((size_t)8 * kBC * ldk + 6 * kBC * kBP + 2 * dk * kJP + 5 * kBC * kJP +
                           2 * kBC + 3 * dk + 3 * kBC) +
          (size_t)kBC * ldz + sizeof(int) * dk + 64;

@@ -316,10 +316,10 @@ __device__ __forceinline__ bool gate_pass_body(uint8_t *sm, uint32_t tmem, int s
     for (int rr = 0; rr < 16; ++rr) vt[rr] = __float_as_uint(ldbf(stv, 16 * qg + rr, c));
     tmem_st16(lane_addr + vcol + 16 * qg, vt);
   }
-  // [row][channel of the pair]: the gates' running products within the row group and (plain
-  // kernel) those of their inverses; the kernel with references, which runs closer to the
-  // register limit, forms the inverse factors from g by one reciprocal each instead
-  float g[16], ig[REFS ? 1 : 16];
+  // [row][channel of the pair]: the running products of the gates and of their inverses within
+  // the row group (the inverse factors need no reciprocal: the gate pass is sensitive to the
+  // special-function unit's throughput)
+  float g[16], ig[16];
   float run0 = 1.f, run1 = 1.f, irun0 = 1.f, irun1 = 1.f;
 #pragma unroll
   for (int rr = 0; rr < 8; ++rr) {
@@ -352,10 +352,8 @@ __device__ __forceinline__ bool gate_pass_body(uint8_t *sm, uint32_t tmem, int s
     if (SG != 2) {
       irun0 *= ial0;
       irun1 *= ial1;
-      if constexpr (!REFS) {
-        ig[2 * rr] = irun0;
-        ig[2 * rr + 1] = irun1;
-      }
+      ig[2 * rr] = irun0;
+      ig[2 * rr + 1] = irun1;
     }
   }
   *reinterpret_cast<float4 *>(sXp + (rg * 128 + ch0) * 2) = make_float4(run0, irun0, run1, irun1);
@@ -384,15 +382,10 @@ __device__ __forceinline__ bool gate_pass_body(uint8_t *sm, uint32_t tmem, int s
       bad |= !(ag0 >= 0x1p-100f && ag0 <= 0x1p100f && ag1 >= 0x1p-100f && ag1 <= 0x1p100f);
     }
     // R / G_t: the earlier groups' inverse product times this group's inverse running product
-    // (or, with references, over this group's running product -- a normal number, checked --
-    // by one reciprocal, accurate to a few ulp like the product itself)
     float inv0, inv1;
     if constexpr (SG == 2) {
       inv0 = __fdividef(1.f, gam0);
       inv1 = __fdividef(1.f, gam1);
-    } else if constexpr (REFS) {
-      inv0 = __fdividef(imult0, g[2 * rr]);
-      inv1 = __fdividef(imult1, g[2 * rr + 1]);
     } else {
       inv0 = ig[2 * rr] * imult0;
       inv1 = ig[2 * rr + 1] * imult1;
