@@ -615,8 +615,8 @@ __global__ void __launch_bounds__(kBThreads) bwd_state_rev_kernel(BwdParams p) {
 template <typename TIn, typename TG>
 __global__ void __launch_bounds__(kGThreads, 1) bwd_grad_kernel(BwdParams p) {
   extern __shared__ float smem[];
-  // rows of dk + 8 floats: the gate gradient's four threads per channel read rows t = 4i + sub,
-  // which then fall on distinct banks for the eight channels of a warp
+  // rows of dk + 8 floats: 16-byte aligned, and the gate gradient's four threads per channel
+  // read rows t = 4i + sub, which then fall on distinct banks for the eight channels of a warp
   const int dk = p.dk, dv = p.dv, ldk = dk + 8, ldz = dk + 4, H = p.H, tid = threadIdx.x;
   float *sQ = smem;                                   // [kBC][ldk] q
   float *sK = sQ + kBC * ldk;                         // [kBC][ldk] k
@@ -712,12 +712,17 @@ __global__ void __launch_bounds__(kGThreads, 1) bwd_grad_kernel(BwdParams p) {
     for (int ti = tid; ti < (kBC / 2) * js; ti += kGThreads) {
       const int r0 = 2 * (ti / js), j = ti % js;
       float a0 = sVp[r0 * kJP + j], a1 = sVp[(r0 + 1) * kJP + j];
-      const float *k0 = sKr + r0 * ldk, *k1 = k0 + ldk;
-#pragma unroll 4
-      for (int c = 0; c < dk; ++c) {
-        const float sv = sS[c * kJP + j];
-        a0 = fmaf(-k0[c], sv, a0);
-        a1 = fmaf(-k1[c], sv, a1);
+      const float *k0 = sKr + r0 * ldk, *k1 = k0 + ldk;   // rows 16-byte aligned (ldk % 4 == 0)
+      for (int c = 0; c < dk; c += 4) {
+        const float4 x0 = *reinterpret_cast<const float4 *>(k0 + c);
+        const float4 x1 = *reinterpret_cast<const float4 *>(k1 + c);
+        const float xa[4] = {x0.x, x0.y, x0.z, x0.w}, xb[4] = {x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float sv = sS[(c + i) * kJP + j];
+          a0 = fmaf(-xa[i], sv, a0);
+          a1 = fmaf(-xb[i], sv, a1);
+        }
       }
       sVp[r0 * kJP + j] = a0;
       sVp[(r0 + 1) * kJP + j] = a1;
@@ -736,11 +741,16 @@ __global__ void __launch_bounds__(kGThreads, 1) bwd_grad_kernel(BwdParams p) {
       sU[(r0 + 1) * kJP + j] = u1;
       float d0 = 0.f, d1 = 0.f;
       const float *k0 = sKd + r0 * ldk, *k1 = k0 + ldk;
-#pragma unroll 4
-      for (int c = 0; c < dk; ++c) {
-        const float sv = sdS[c * kJP + j];
-        d0 = fmaf(k0[c], sv, d0);
-        d1 = fmaf(k1[c], sv, d1);
+      for (int c = 0; c < dk; c += 4) {
+        const float4 x0 = *reinterpret_cast<const float4 *>(k0 + c);
+        const float4 x1 = *reinterpret_cast<const float4 *>(k1 + c);
+        const float xa[4] = {x0.x, x0.y, x0.z, x0.w}, xb[4] = {x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float sv = sdS[(c + i) * kJP + j];
+          d0 = fmaf(xa[i], sv, d0);
+          d1 = fmaf(xb[i], sv, d1);
+        }
       }
       for (int t = r0; t < kBC; ++t) {   // P[r0][r0 + 1] = 0
         const float o = sdO[t * kJP + j];

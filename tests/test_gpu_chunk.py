@@ -381,6 +381,32 @@ def test_tc_range_cuts(cuda_lib, sg):
     close(S, rS, TOL_BF16, "S_T")
 
 
+def test_tc_handoff_positions(cuda_lib):
+    """Units handed to the kernel with references at their first chunk (head 0), in the middle
+    (head 1, fast gates from row 150) and in the ragged last chunk (head 2, from row 262 of
+    273); S_T written over S0.  The workspace header's hand-off count says all three moved."""
+    T, H = 273, 3
+    rng = np.random.default_rng(80)
+    a = rng.standard_normal((1, T, H, 128)) * 0.5 + 3.0
+    fast = math.log(2.0 ** -5 / (1 - 2.0 ** -5))      # KDA gate 2^-5: 320 bits per 64 rows
+    a[0, :, 0, 17] = fast
+    a[0, 150:, 1, 40:44] = fast
+    a[0, 262:, 2, 99] = -60.0                          # 2^-87 per row: not even 8 rows fit
+    b = rng.standard_normal((1, T, H))
+    inp = _bf16_raw_case(T, a, b, seed=81, H=H)
+    w = synth.KDA_STD.with_(B=1, T=T, H=H, o_dtype="f32")
+    d = to_device(inp)
+    ws = cuda_lib.new_workspace(1, T, H, 128, 128, 64, 0, torch.device("cuda"))
+    S = d["S0"].clone()
+    o, S = cuda_lib.chunk_fwd(d["q"], d["k"], d["v"], d["a"], d["b"], S, None, chunk=64,
+                              signed_gate=0, o_dtype=torch.float32, S_T=S, workspace=ws)
+    torch.cuda.synchronize()
+    assert int(ws[64:68].view(torch.int32).item()) == 3
+    ro, rS = oracle_prefill(inp, 0)
+    close(o, ro, TOL_BF16, "o")
+    close(S, rS, TOL_BF16, "S_T")
+
+
 def test_tc_fast_forgetting_without_handoff(cuda_lib):
     """With only the 256-byte workspace header there is no room for the hand-off to the kernel
     with references: chunks past the plain kernel's range run token by token, exactly."""
