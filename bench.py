@@ -323,7 +323,8 @@ class PrefillCase:
         B, T = host["q"].shape[:2]
         self.o = torch.empty((B, T, w.H, w.dv), dtype=torch.bfloat16, device=dev)
         self.S_T = torch.empty((w.n_seqs, w.H, w.dk, w.dv), dtype=torch.float32, device=dev)
-        self.ws = ops.new_workspace(B, T, w.H, w.dk, w.dv, w.chunk, w.n_seqs, dev)
+        self.ws = ops.new_workspace(B, T, w.H, w.dk, w.dv, w.chunk,
+                                    w.n_seqs if w.seq_lens is not None else 0, dev)
 
     def __call__(self):
         d = self.d
@@ -401,10 +402,12 @@ def main():
         case.check("the headline leg")
         ms_step = ms / args.steps
         value = tokens * args.steps / (ms / 1000.0)
-        # dominant kernel: the chunk kernel.  A step is two launches (the 256-byte status memset
-        # before them is included, < 2 us): the plain tensor-core kernel, then the kernel with
-        # per-channel references for the units it handed off (none here: its CTAs return at once,
-        # ~6 us with the programmatic dependent launch)
+        # dominant kernel: the chunk kernel.  A packed step is six launches (the 256-byte status
+        # memset before them is included, < 2 us): the unit planner, the first launch of the
+        # plain tensor-core kernel and of the kernel with per-channel references for the units
+        # it handed off (none here: its CTAs return at once, ~6 us with the programmatic
+        # dependent launch), the state chain of the cut sequence, and the second pair; an
+        # unpacked step without a cut is the first pair alone
         roofline = prefill_roofline(w, ms_step, peaks, "chunk_tc_kernel/" + w.name)
 
     # ------------------------------------------------------------ e2e (host buffers)
@@ -584,7 +587,7 @@ def main():
             "config": headline_config(w),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "workloads": workloads, "fwd_bwd": fwd_bwd, "decode": decode_obj,
-            "gpu_launches": 2 * args.steps, "clocks": clocks, "peaks_source": peaks["source"],
+            "gpu_launches": (6 if w.seq_lens is not None else 2) * args.steps, "clocks": clocks, "peaks_source": peaks["source"],
         }
         print(json.dumps(line), flush=True)
     if world > 1:

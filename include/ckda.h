@@ -114,10 +114,18 @@ extern "C" {
  *            status header); owned by the caller, reused freely between calls
  *            on the same stream, never shared by two calls in flight at once.
  *            With ckda_chunk_fwd_workspace_size() bytes, the tensor-core path
- *            hands a (sequence, head) whose gates decay faster than its range
+ *            (1) hands a (sequence, head) whose gates decay faster than its range
  *            (a chunk product below 2^-100 in some channel) to a second launch
  *            that carries per-channel references and stays on the tensor
- *            cores; with less, such chunks run token by token (exact, slower).
+ *            cores; with less, such chunks run token by token (exact, slower);
+ *            (2) cuts the one or two longest sequences of a batch into
+ *            segments when their serial chunk walk would bound the call (a
+ *            packed batch with one long document, a short batch of long
+ *            sequences): the segments run in parallel from a zero and an
+ *            identity state, their affine state maps are chained on the
+ *            device, and the segments run again from their true states (the
+ *            DPR1 transition of the CKDA review is linear in the state).  The
+ *            result is the same recurrence; with less workspace nothing is cut.
  *   stream  : cudaStream_t.
  * Returns CKDA_OK or a negative CKDA_ERR_* code.
  */
@@ -128,10 +136,13 @@ int ckda_chunk_fwd(const void *q, const void *k, const void *v, const void *a, c
 
 /*
  * Bytes of workspace ckda_chunk_fwd uses in full for these sizes (same
- * meaning as there; n_seqs is ignored when the batch is not packed): 256 for
- * the exact path; for dk = dv = 128 and chunk 64 also a 16-byte queue entry
- * and a 64 KB saved state per (sequence, head) for the hand-off above.  Pure
- * host arithmetic, no CUDA call.
+ * meaning as there; n_seqs > 0 means a packed batch of n_seqs sequences, else
+ * B sequences of T tokens): 256 for the exact path; for dk = dv = 128 and
+ * chunk 64 also a 16-byte queue entry and a 64 KB saved state per unit of
+ * one launch for the hand-off above, and, where sequences may be cut (every
+ * packed batch of at most 1024 sequences; an unpacked batch whose walk the cut
+ * shortens on a 148-SM B200), the unit lists and 26 state slots per head.
+ * Pure host arithmetic, no CUDA call.
  */
 size_t ckda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int chunk,
                                      int n_seqs);
@@ -250,6 +261,19 @@ int ckda_workspace_status(const void *workspace, int *status, void *stream);
  * the hook off (the default).  Process-wide; takes effect at the next launch.
  */
 void ckda_debug_wait_injection(int chunk_index, unsigned long long wait_ns);
+
+/*
+ * TEST HOOK for the segment cut of ckda_chunk_fwd (workspace item (2));
+ * not needed in normal use.  After ckda_debug_segment_split(n_split,
+ * n_segments) with 1 <= n_split <= 2 and 3 <= n_segments <= 8, every later
+ * packed ckda_chunk_fwd call on the tensor-core kernel whose workspace has
+ * ckda_chunk_fwd_workspace_size() bytes cuts its n_split longest sequences
+ * into n_segments segments (fewer when a sequence has fewer chunks; a
+ * sequence of under three chunks is not cut) whatever the cost model says.
+ * Other arguments switch the hook off (the default: the cost model decides).
+ * Process-wide; takes effect at the next launch.
+ */
+void ckda_debug_segment_split(int n_split, int n_segments);
 
 /* Static, human-readable text for a status code (never NULL). */
 const char *ckda_status_string(int status);

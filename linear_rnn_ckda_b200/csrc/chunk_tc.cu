@@ -119,6 +119,11 @@ struct TcParams {
   int *queue_count;
   int4 *queue;
   float *saved_S;
+  // Unit list of a planned launch (NULL: unit = (sequence, head) in length order): CTA x runs
+  // entry x / H for head x % H when x / H < *plan_count.  slots holds the cut sequences' states.
+  const SegDesc *plan;
+  const int *plan_count;
+  float *slots;
 };
 
 // byte offset of fp32 element (r, c) in a 128-byte-swizzled tile of R rows
@@ -582,10 +587,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = p.H;
   const int unit = blockIdx.x;
-  int n, h;
+  int n, h, mode = 0;
   long t0, t1, bofs;
-  const float *s_init = p.S0;   // the state the unit starts from ([dk][dv] at s_init + s_init_ofs)
-  size_t sofs;
+  const float *s_init = nullptr;   // the state the unit starts from ([dk][dv]; NULL: zero)
+  int out_slot = 0;
+  auto slot_state = [&](int slot) { return p.slots + ((size_t)slot * H + h) * kD * kD; };
   if constexpr (REFS) {
     // a unit the plain kernel handed off: from its first row on, from the state it saved (this
     // grid may start before the plain one has finished: wait for it, and for its writes)
@@ -595,10 +601,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     n = e.x;
     h = e.y;
     t0 = e.z;
-    t1 = p.cu ? p.cu[n + 1] : p.T;
-    bofs = p.cu ? 0 : (long)n * p.T;
+    if (p.plan && e.w >= 0) {
+      const SegDesc d = p.plan[e.w];
+      t1 = d.t1;
+      mode = d.mode & ~(kSegInZero | kSegInIdent | kSegInSlot);
+      out_slot = d.out_slot;
+    } else {
+      t1 = p.cu ? p.cu[n + 1] : p.T;
+    }
     s_init = p.saved_S + (size_t)unit * kD * kD;
-    sofs = ((size_t)n * H + h) * kD * kD;
+  } else if (p.plan) {
+    // an entry of the unit list (offsets were checked by the planner)
+    const int di = unit / H;
+    if (di >= *p.plan_count) return;
+    const SegDesc d = p.plan[di];
+    h = unit - di * H;
+    n = d.n;
+    t0 = d.t0;
+    t1 = d.t1;
+    mode = d.mode;
+    out_slot = d.out_slot;
+    if (mode & kSegInSlot) s_init = slot_state(d.in_slot);
+    else if (!(mode & (kSegInZero | kSegInIdent)) && p.S0)
+      s_init = p.S0 + ((size_t)n * H + h) * kD * kD;
   } else {
     h = unit % H;
     // CTAs start in blockIdx order: in a packed batch the longest sequences go first, so that
@@ -609,7 +634,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (p.cu) {
       t0 = p.cu[n];
       t1 = p.cu[n + 1];
-      bofs = 0;
       if (t0 < 0 || t1 < t0 || t1 > p.T || (n == 0 && t0 != 0) ||
           (n == p.n_seqs - 1 && t1 != p.T)) {
         if (tid == 0) set_status(p.status, CKDA_ERR_SEQLENS);
@@ -618,12 +642,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
       t0 = 0;
       t1 = p.T;
-      bofs = (long)n * p.T;
     }
-    sofs = ((size_t)n * H + h) * kD * kD;
+    if (p.S0) s_init = p.S0 + ((size_t)n * H + h) * kD * kD;
   }
-  const size_t s_init_ofs = REFS ? 0 : sofs;
-  TOut *o = static_cast<TOut *>(p.o);
+  bofs = p.cu ? 0 : (long)n * p.T;
+  // where the end state goes (NULL: nowhere)
+  float *const s_out = (mode & kSegOutSlot) ? slot_state(out_slot)
+                       : (!(mode & kSegOutNone) && p.S_T) ? p.S_T + ((size_t)n * H + h) * kD * kD
+                                                          : nullptr;
+  const bool vzero = (mode & kSegVZero) != 0;   // v = 0 (the v tile is not loaded)
+  TOut *o = (mode & kSegNoO) ? nullptr : static_cast<TOut *>(p.o);
 
   if (tid == 0) {
     for (int x = 0; x < 6; ++x) mbar_init(bars + x, 1);
@@ -653,12 +681,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto issue_tma = [&](long cs) {   // q, k, v and (per-channel gates) a of one chunk
     atomicAdd(sTmaIssued, 1u);
     const int ntens = per_head ? 3 : 4;
-    mbar_arrive_expect_tx(bar_tma, ntens * 2 * 8192);
+    mbar_arrive_expect_tx(bar_tma, (ntens - (vzero ? 1 : 0)) * 2 * 8192);
     const int row = (int)(bofs + cs);
     const CUtensorMap *maps[4] = {&tm_q, &tm_k, &tm_v, &tm_a};
 #pragma unroll
     for (int x = 0; x < 4; ++x)
-      if (x < ntens) {
+      if (x < ntens && !(x == 2 && vzero)) {
 #pragma unroll
         for (int bx = 0; bx < 2; ++bx)
           tma_load_3d(sStg + x * 16384 + bx * 8192, maps[x], bar_tma, bx * 64, h, row);
@@ -989,11 +1017,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     {
       uint32_t r[32];
       const int i0 = 32 * qg;
+      const bool ident = (mode & kSegInIdent) != 0;
 #pragma unroll
       for (int x = 0; x < 32; ++x)
-        r[x] = __float_as_uint(s_init ? s_init[s_init_ofs + (size_t)(i0 + x) * kD + jrow] : 0.f);
+        r[x] = __float_as_uint(ident    ? (i0 + x == jrow ? 1.f : 0.f)
+                               : s_init ? s_init[(size_t)(i0 + x) * kD + jrow]
+                                        : 0.f);
       tmem_st32(lane_addr + COL_S + i0, r);
       tmem_wait_st();
+    }
+    if (vzero) {
+      // the v tile is never loaded: zero once (rows past a chunk's end are zeroed anyway)
+      for (int e = tid; e < 1024; e += kCompute)
+        reinterpret_cast<uint4 *>(sStg + 32768)[e] = make_uint4(0u, 0u, 0u, 0u);
     }
     if (tid == 0 && t1 > t0) issue_tma(t0);
     csync();
@@ -1057,7 +1093,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (tid == 0) {
           const int slot = atomicAdd(p.queue_count, 1);
           *sSlot = slot;
-          p.queue[slot] = make_int4(n, h, (int)cs, 0);
+          p.queue[slot] = make_int4(n, h, (int)cs, p.plan ? (int)(blockIdx.x / H) : -1);
         }
         csync();
         const int slot = *sSlot;
@@ -1307,15 +1343,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         set_status(p.status, CKDA_ERR_TIMEOUT);
         *sAbort = 1;   // the issuer leaves its loop at its next wait
       }
-    } else if (p.S_T && !handed_off) {
+    } else if (s_out && !handed_off) {
       tc_fence_after();
       uint32_t r[32];
       const int i0 = 32 * qg;
       tmem_ld32(lane_addr + COL_S + i0, r);
       tmem_wait_ld();
 #pragma unroll
-      for (int x = 0; x < 32; ++x)
-        p.S_T[sofs + (size_t)(i0 + x) * kD + jrow] = __uint_as_float(r[x]);
+      for (int x = 0; x < 32; ++x) s_out[(size_t)(i0 + x) * kD + jrow] = __uint_as_float(r[x]);
     }
   }
   tc_fence_before();
@@ -1377,10 +1412,18 @@ bool make_out_map(CUtensorMap *map, void *base, int H, long rows, bool bf16) {
              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Workspace of the hand-off (after the 256-byte header, whose word at byte 64 counts the queued
-// units): the queue, then the saved states.
+// The workspace (tc_workspace_layout): the 256-byte header (status word; at byte 64 the count
+// of handed-off units; at kSegHeaderOffset the plan's header), the hand-off queue and saved
+// states, and for a planned call the two unit lists and the cut sequences' state slots.
 constexpr size_t kQueueCountOffset = 64;
-inline size_t handoff_queue_bytes(long units) { return ((size_t)units * 16 + 255) & ~(size_t)255; }
+
+int sm_count() {
+  int dev = 0, P = kSegAssumedSMs;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&P, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || P <= 0)
+    P = kSegAssumedSMs;
+  return P;
+}
 
 template <typename TOut, int SG, int FL>
 int launch_typed(const ChunkArgs &g, cudaStream_t stream) {
@@ -1400,50 +1443,74 @@ int launch_typed(const ChunkArgs &g, cudaStream_t stream) {
   p.inject_chunk = g.inject_chunk;
   p.inject_wait_ns = g.inject_wait_ns;
   p.a_head = per_head ? static_cast<const __nv_bfloat16 *>(g.a) : nullptr;
-  const long units = (long)g.n_seqs * g.H;
-  const bool handoff = SG != 2 && g.workspace &&
-                       g.workspace_bytes >= chunk_tc_handoff_bytes(g.n_seqs, g.H);
+  p.plan = nullptr;
+  p.plan_count = nullptr;
+  p.slots = nullptr;
+
+  // plan (cut the longest sequences) when the cost model may gain and the workspace has room
+  const bool packed = g.cu_seqlens != nullptr;
+  const int P = sm_count();
+  const bool want_plan = g.n_seqs <= kSegMaxSeqs &&
+                         (g.force_split > 0 ? packed : tc_plans(packed, g.B, g.T, g.H, g.n_seqs, P));
+  TcWorkspace L = tc_workspace_layout(g.n_seqs, g.H, true);
+  const bool plan = want_plan && g.workspace && g.workspace_bytes >= L.total;
+  if (!plan) L = tc_workspace_layout(g.n_seqs, g.H, false);
+  const bool handoff = SG != 2 && g.workspace && g.workspace_bytes >= L.total;
   uint8_t *ws = static_cast<uint8_t *>(g.workspace);
   p.queue_count = handoff ? reinterpret_cast<int *>(ws + kQueueCountOffset) : nullptr;
-  p.queue = handoff ? reinterpret_cast<int4 *>(ws + kWorkspaceHeader) : nullptr;
-  p.saved_S = handoff ? reinterpret_cast<float *>(ws + kWorkspaceHeader + handoff_queue_bytes(units))
-                      : nullptr;
+  p.queue = handoff ? reinterpret_cast<int4 *>(ws + L.queue_off) : nullptr;
+  p.saved_S = handoff ? reinterpret_cast<float *>(ws + L.saved_off) : nullptr;
+
   auto kern = chunk_tc_kernel<TOut, SG, FL, false>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) !=
       cudaSuccess)
     return CKDA_ERR_CUDA;
-  kern<<<(unsigned)units, kThreads, kSmemBytes, stream>>>(mq, mk, mv, ma, mo, p);
-  if (cudaGetLastError() != cudaSuccess) return CKDA_ERR_CUDA;
-  if constexpr (SG != 2) {
-    if (handoff) {
-      // the units handed off (CTAs past the queue's count return at once)
-      auto kern_r = chunk_tc_kernel<TOut, SG, FL, true>;
-      if (cudaFuncSetAttribute(kern_r, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)kSmemBytes) != cudaSuccess)
-        return CKDA_ERR_CUDA;
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3((unsigned)units);
-      cfg.blockDim = dim3(kThreads);
-      cfg.dynamicSmemBytes = kSmemBytes;
-      cfg.stream = stream;
-      cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // launch early
-      attr[0].val.programmaticStreamSerializationAllowed = 1;
-      cfg.attrs = attr;
-      cfg.numAttrs = 1;
-      if (cudaLaunchKernelEx(&cfg, kern_r, mq, mk, mv, ma, mo, p) != cudaSuccess)
-        return CKDA_ERR_CUDA;
+  // one launch of the plain kernel over `units` CTAs, then (hand-off) the kernel with references
+  // on the units it queued
+  auto run = [&](long units) -> int {
+    kern<<<(unsigned)units, kThreads, kSmemBytes, stream>>>(mq, mk, mv, ma, mo, p);
+    if (cudaGetLastError() != cudaSuccess) return CKDA_ERR_CUDA;
+    if constexpr (SG != 2) {
+      if (handoff) {
+        // CTAs past the queue's count return at once
+        auto kern_r = chunk_tc_kernel<TOut, SG, FL, true>;
+        if (cudaFuncSetAttribute(kern_r, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kSmemBytes) != cudaSuccess)
+          return CKDA_ERR_CUDA;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)units);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = kSmemBytes;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // launch early
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, kern_r, mq, mk, mv, ma, mo, p) != cudaSuccess)
+          return CKDA_ERR_CUDA;
+      }
     }
-  }
-  return CKDA_OK;
+    return CKDA_OK;
+  };
+  if (!plan) return run((long)g.n_seqs * g.H);
+
+  SegHeader *hdr = reinterpret_cast<SegHeader *>(ws + kSegHeaderOffset);
+  SegDesc *d1 = reinterpret_cast<SegDesc *>(ws + L.desc_off), *d3 = d1 + L.max_desc;
+  p.slots = reinterpret_cast<float *>(ws + L.slot_off);
+  int rc = launch_seg_plan(g.cu_seqlens, g.n_seqs, g.T, g.H, P, g.force_split, g.force_nseg, hdr,
+                           d1, d3, g.status, stream);
+  if (rc != CKDA_OK) return rc;
+  p.plan = d1;
+  p.plan_count = &hdr->n1;
+  if ((rc = run((long)L.max_desc * g.H)) != CKDA_OK) return rc;
+  if ((rc = launch_seg_combine(hdr, p.slots, p.queue_count, g.H, stream)) != CKDA_OK) return rc;
+  p.plan = d3;
+  p.plan_count = &hdr->n3;
+  return run((long)L.max_desc * g.H);
 }
 
 }  // namespace
-
-size_t chunk_tc_handoff_bytes(int n_seqs, int H) {
-  const long units = (long)n_seqs * H;
-  return kWorkspaceHeader + handoff_queue_bytes(units) + (size_t)units * kD * kD * sizeof(float);
-}
 
 bool chunk_tc_supported(const ChunkArgs &g) {
   return g.dk == kD && g.dv == kD && g.chunk == kC && g.io_dtype == CKDA_BF16 &&

@@ -46,6 +46,9 @@ int check_device() {
 // ckda_debug_wait_injection's settings (process-wide, read at each launch)
 std::atomic<int> g_inject_chunk{-1};
 std::atomic<unsigned long long> g_inject_wait_ns{0};
+// ckda_debug_segment_split's settings (process-wide, read at each launch)
+std::atomic<int> g_force_split{0};
+std::atomic<int> g_force_nseg{0};
 
 }  // namespace
 
@@ -81,6 +84,13 @@ void ckda_debug_wait_injection(int chunk_index, unsigned long long wait_ns) {
   g_inject_chunk.store(chunk_index < 0 ? -1 : chunk_index, std::memory_order_relaxed);
 }
 
+void ckda_debug_segment_split(int n_split, int n_segments) {
+  const bool on = n_split > 0 && n_split <= ckda::kSegMaxSplit && n_segments >= 3 &&
+                  n_segments <= ckda::kSegMaxSeg;
+  g_force_nseg.store(on ? n_segments : 0, std::memory_order_relaxed);
+  g_force_split.store(on ? n_split : 0, std::memory_order_relaxed);
+}
+
 const char *ckda_status_string(int status) {
   switch (status) {
     case CKDA_OK: return "ok";
@@ -101,10 +111,12 @@ const char *ckda_status_string(int status) {
 int ckda_version(void) { return 100; }
 
 size_t ckda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int chunk, int n_seqs) {
-  (void)T;
-  const int N = n_seqs > 0 ? n_seqs : B;
-  if (dk == 128 && dv == 128 && chunk == 64 && N > 0 && H > 0)
-    return std::max(ckda::kWorkspaceHeader, ckda::chunk_tc_handoff_bytes(N, H));
+  const bool packed = n_seqs > 0;
+  const int N = packed ? n_seqs : B;
+  if (dk == 128 && dv == 128 && chunk == 64 && N > 0 && H > 0) {
+    const bool plan = ckda::tc_plans(packed, B, T, H, N, ckda::kSegAssumedSMs);
+    return std::max(ckda::kWorkspaceHeader, ckda::tc_workspace_layout(N, H, plan).total);
+  }
   return ckda::kWorkspaceHeader;
 }
 
@@ -135,6 +147,8 @@ int ckda_chunk_fwd(const void *q, const void *k, const void *v, const void *a, c
   g.workspace_bytes = workspace_bytes;
   g.inject_chunk = g_inject_chunk.load(std::memory_order_relaxed);
   g.inject_wait_ns = g_inject_wait_ns.load(std::memory_order_relaxed);
+  g.force_split = g_force_split.load(std::memory_order_relaxed);
+  g.force_nseg = g_force_nseg.load(std::memory_order_relaxed);
   if (ckda::chunk_tc_supported(g)) return ckda::launch_chunk_tc(g, s);
   return ckda::launch_chunk_simt(g, s);
 }

@@ -23,7 +23,130 @@ struct ChunkArgs {
   // tensor-core kernel waits on a barrier nothing arrives on (-1: off), and that wait's bound
   int inject_chunk;
   unsigned long long inject_wait_ns;
+  // test hook (ckda_debug_segment_split): cut the force_split longest sequences into
+  // force_nseg segments whatever the cost model says (0: the cost model decides)
+  int force_split, force_nseg;
 };
+
+// ---------------------------------------------------------------- segment plan (tensor-core path)
+// A sequence's chunk walk is serial, so a batch whose longest sequence holds far more chunks than
+// the batch's work per SM is bound by that one walk.  The state map of a segment of the
+// recurrence is affine in the state it starts from: S_end = A S_in + B, A the product of the
+// segment's transitions (the end state from S_in = I with v = 0) and B the end state from
+// S_in = 0.  A long sequence cut into segments 0 .. m-1 then runs in two launches:
+//   first:   X_0 = segment 0 from the caller's S0 (o written); for s = 1 .. m-2 X_s from 0 and
+//            Y_s from I with v = 0 (o not written);
+//   combine: X_s <- Y_s X_{s-1} + X_s for s = 1 .. m-2 (X_s: the state entering segment s + 1);
+//   second:  segments 1 .. m-1 from X_{s-1}, o written, the last one writes S_T.
+// Every other sequence runs whole in one of the two launches, chosen to balance them.
+constexpr int kSegMaxSplit = 2;                       // sequences cut at most
+constexpr int kSegMaxSeg = 8;                         // segments per cut sequence at most
+constexpr int kSegSlotsPerSplit = 2 * kSegMaxSeg - 3; // X_0 .. X_{m-2}, Y_1 .. Y_{m-2}
+constexpr int kSegMinChunks = 48;                     // shorter sequences are never cut
+constexpr int kSegMaxSeqs = 1024;                     // larger packed batches are not planned
+constexpr int kSegAssumedSMs = 148;                   // SM count the workspace size assumes
+
+// one unit list entry: rows [t0, t1) of sequence n (packed rows, or rows of batch row n), run
+// for every head; states in slots are [slot][H][dk][dv]
+struct SegDesc {
+  int t0, t1, n, mode, in_slot, out_slot, pad0, pad1;
+};
+enum : int {
+  kSegInZero = 1,    // start from S = 0 (else the caller's S0)
+  kSegInIdent = 2,   // start from S = I
+  kSegInSlot = 4,    // start from slot in_slot
+  kSegOutSlot = 8,   // end state to slot out_slot (else the caller's S_T)
+  kSegOutNone = 16,  // end state not written
+  kSegVZero = 32,    // v = 0
+  kSegNoO = 64,      // o not written
+};
+struct SegSplit {
+  int m, seg_rows, slot_base, pad;
+};
+// in the workspace header at byte kSegHeaderOffset
+struct SegHeader {
+  int n1, n3, nsplit, pad;
+  SegSplit split[kSegMaxSplit];
+};
+constexpr size_t kSegHeaderOffset = 128;
+
+// The cost model: given the chunk counts of the longest sequences (top[0] >= top[1] >= ...,
+// min(nv, kSegMaxSplit + 1) of them), the batch's total chunk count over all heads W, H and
+// the SM count P, how many sequences to cut (k, 0: none) and into how many segments each (m[i]
+// of seg[i] chunks), and the estimated walk (in chunk times) with and without the cut.
+struct SegChoice {
+  int k;
+  int m[kSegMaxSplit], seg[kSegMaxSplit];
+  long est, est0;
+  int w1, w3;   // waves of the cut sequences' units in the first and second launch
+};
+__host__ __device__ inline long seg_cdiv(long a, long b) { return (a + b - 1) / b; }
+__host__ __device__ inline SegChoice seg_choose(const int *top, int nv, long W, int H, int P,
+                                                int force_k, int force_m) {
+  SegChoice best;
+  best.k = 0;
+  best.w1 = best.w3 = 0;
+  best.est0 = nv > 0 ? (top[0] > seg_cdiv(W, P) ? (long)top[0] : seg_cdiv(W, P)) : 0;
+  best.est = best.est0;
+  const int kmax = nv < kSegMaxSplit ? nv : kSegMaxSplit;
+  for (int k = 1; k <= kmax; ++k) {
+    for (int nseg = 3; nseg <= kSegMaxSeg; ++nseg) {
+      if (force_k > 0 && (k != force_k || nseg != force_m)) continue;
+      SegChoice c;
+      c.k = k;
+      long U1 = 0, U3 = 0, extra = 0;
+      bool ok = true;
+      for (int i = 0; i < k; ++i) {
+        const int ch = top[i];
+        if (force_k <= 0 && ch < kSegMinChunks) ok = false;
+        const int L = ch > 0 ? (int)seg_cdiv(ch, nseg) : 1;
+        const int mm = (int)seg_cdiv(ch, L);
+        if (mm < 3) ok = false;
+        c.m[i] = mm;
+        c.seg[i] = L;
+        U1 += (long)H * (2 * mm - 3);
+        U3 += (long)H * (mm - 1);
+        extra += (long)H * L * (2 * mm - 4);
+      }
+      if (!ok) continue;
+      const long L0 = c.seg[0];
+      c.w1 = (int)seg_cdiv(U1, P);
+      c.w3 = (int)seg_cdiv(U3, P);
+      long chain = L0 * (c.w1 + c.w3);
+      if (k < nv) {
+        const long wsmall = c.w1 < c.w3 ? c.w1 : c.w3;
+        const long alt = L0 * wsmall + (long)top[k];
+        if (alt > chain) chain = alt;
+      }
+      const long work = seg_cdiv(W + extra, P);
+      c.est = chain > work ? chain : work;
+      c.est0 = best.est0;
+      if (force_k > 0 || c.est < best.est) best = c;
+    }
+  }
+  // a cut costs two more launches and up to twice the work of the cut sequences: only for a
+  // clear gain
+  if (force_k <= 0 && best.k > 0 && best.est * 10 > best.est0 * 9) best.k = 0;
+  return best;
+}
+
+// Workspace of the tensor-core path: the header, the hand-off queue and saved states for
+// `units` units, and (plan) the unit lists and the cut sequences' state slots.
+struct TcWorkspace {
+  size_t queue_off, saved_off, desc_off, slot_off, total;
+  long units;      // hand-off capacity (units of one launch)
+  int max_desc;    // entries of each unit list
+};
+TcWorkspace tc_workspace_layout(int n_seqs, int H, bool plan);
+// Whether the tensor-core path plans a batch of these sizes (packed: always, up to kSegMaxSeqs
+// sequences; otherwise when the cost model cuts at kSegAssumedSMs SMs) and the workspace bytes
+// it then uses.
+bool tc_plans(bool packed, int B, int T, int H, int n_seqs, int P);
+// The unit planner (one CTA) and the state combination between the two launches.
+int launch_seg_plan(const int32_t *cu, int n_seqs, int T, int H, int P, int force_k, int force_m,
+                    SegHeader *hdr, SegDesc *d1, SegDesc *d3, int *status, cudaStream_t s);
+int launch_seg_combine(const SegHeader *hdr, float *slots, int *queue_count, int H,
+                       cudaStream_t s);
 
 struct DecodeArgs {
   const void *q, *k, *v, *a;
@@ -45,10 +168,6 @@ int launch_chunk_simt(const ChunkArgs &args, cudaStream_t stream);
 
 // Tensor-core chunkwise forward (tcgen05, dk = dv = 128, chunk 64, bf16 io).
 bool chunk_tc_supported(const ChunkArgs &args);
-// Workspace bytes that let the tensor-core kernel hand units whose gates decay past its range to
-// its variant with per-channel references (the header, a queue and one saved state per unit);
-// with less, such chunks run token by token.
-size_t chunk_tc_handoff_bytes(int n_seqs, int H);
 int launch_chunk_tc(const ChunkArgs &args, cudaStream_t stream);
 
 // First chunk slot of sequence n when chunks of C tokens of every sequence are numbered in one

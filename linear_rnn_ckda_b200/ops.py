@@ -45,6 +45,7 @@ SIGNATURES = {
     "ckda_workspace_status": (_i, [_vp, ctypes.POINTER(_i), _vp]),
     "ckda_noalloc_status": (_i, [ctypes.POINTER(_i), _vp]),
     "ckda_debug_wait_injection": (None, [_i, ctypes.c_ulonglong]),
+    "ckda_debug_segment_split": (None, [_i, _i]),
     "ckda_status_string": (ctypes.c_char_p, [_i]),
     "ckda_version": (_i, []),
 }
@@ -200,7 +201,7 @@ def chunk_fwd(q, k, v, a, b, S0=None, cu_seqlens=None, chunk: int = 64, signed_g
     if want_state and S_T is None:
         S_T = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
     if workspace is None:
-        workspace = new_workspace(B, T, H, dk, dv, chunk, N, dev)
+        workspace = new_workspace(B, T, H, dk, dv, chunk, N if cu_seqlens is not None else 0, dev)
     _need(workspace.device == dev, f"workspace is on {workspace.device}, q on {dev}")
     rc = lib.ckda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(S0),
                             _ptr(cu_seqlens), N if cu_seqlens is not None else 0, B, T, H, dk, dv,
@@ -290,6 +291,11 @@ def noalloc_status(device=None) -> int:
 def debug_wait_injection(chunk_index: int, wait_ns: int = 0) -> None:
     """Test hook: see ``ckda_debug_wait_injection`` in ``include/ckda.h`` (-1 switches it off)."""
     load().ckda_debug_wait_injection(int(chunk_index), int(wait_ns))
+
+
+def debug_segment_split(n_split: int, n_segments: int) -> None:
+    """Test hook: see ``ckda_debug_segment_split`` in ``include/ckda.h`` (0, 0 switches it off)."""
+    load().ckda_debug_segment_split(int(n_split), int(n_segments))
 
 
 def workspace_status(workspace: torch.Tensor) -> int:

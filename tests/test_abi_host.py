@@ -69,9 +69,22 @@ def test_workspace_size(lib):
     units = 4 * 16
     assert lib.ckda_chunk_fwd_workspace_size(4, 4096, 16, 128, 128, 64, 0) == \
         256 + 1024 + units * 65536
-    units = 3 * 2   # packed: n_seqs sequences
+    # a packed batch may have its two longest sequences cut into up to 8 segments: the unit
+    # lists hold n_seqs + 2 * 13 entries (32 bytes each, two lists), the hand-off covers that
+    # many units of one launch, and 2 * 13 state slots per head hold the segments' states
+    entries = 3 + 26
+    units = entries * 2
     assert lib.ckda_chunk_fwd_workspace_size(1, 1000, 2, 128, 128, 64, 3) == \
-        256 + 256 + units * 65536
+        256 + 1024 + units * 65536 + 2048 + 26 * 2 * 65536
+    # unpacked: the plan's room only where the cost model (148 SMs) cuts; one sequence of
+    # 65,536 tokens over 16 heads (16 walks of 1,024 chunks) is cut
+    entries = 1 + 26
+    units = entries * 16
+    assert lib.ckda_chunk_fwd_workspace_size(1, 65536, 16, 128, 128, 64, 0) == \
+        256 + 6912 + units * 65536 + 1792 + 26 * 16 * 65536
+    no_plan = lambda B, T, H: 256 + (((B * H * 16) + 255) // 256) * 256 + B * H * 65536
+    for B, T, H in ((4, 4096, 16), (8, 8192, 16), (2, 65536, 64), (1, 2048, 1)):
+        assert lib.ckda_chunk_fwd_workspace_size(B, T, H, 128, 128, 64, 0) == no_plan(B, T, H)
 
 
 # Fake, aligned, never-dereferenced host addresses: every call below has exactly

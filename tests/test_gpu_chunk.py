@@ -200,9 +200,11 @@ def test_chunk_size_invariance(cuda_lib):
         assert_close(f64(S), f64(outs[0][1]), 1e-5, "S_T across chunk sizes")
 
 
-def test_bad_seqlens_sets_status(cuda_lib):
-    """Decreasing offsets: the kernel skips the bad sequences and records the error."""
-    w = synth.CKDA_SPREAD.with_(B=1, H=1, seq_lens=(10, 10), T=20, io_dtype="f32", o_dtype="f32")
+@pytest.mark.parametrize("io", ["f32", "bf16"], ids=["exact", "tensor_core"])
+def test_bad_seqlens_sets_status(cuda_lib, io):
+    """Decreasing offsets: the kernel (the exact one) or the unit planner (tensor-core path)
+    skips the bad sequences and records the error."""
+    w = synth.CKDA_SPREAD.with_(B=1, H=1, seq_lens=(10, 10), T=20, io_dtype=io, o_dtype="f32")
     inp = to_device(synth.make_prefill(w, seed=10))
     cu = torch.tensor([0, 15, 12], dtype=torch.int32, device="cuda")  # ends below start
     ws = cuda_lib.new_workspace(1, 20, 1, 128, 128, 64, 2)
@@ -432,6 +434,94 @@ def test_tc_fast_forgetting_varlen_alias(cuda_lib):
     o, S = run_gpu(cuda_lib, inp, w, S0_alias=True)
     close(o, ro, TOL_BF16, "o")
     close(S, rS, TOL_BF16, "S_T")
+
+
+# ---------------------------------------------------------------- segments of long sequences
+# The longest sequences of a batch may be cut into segments: the first launch runs each segment
+# from a zero state and from the identity with v = 0 (its affine state map), a small kernel
+# chains the maps, and the second launch runs the segments from their true starting states.
+
+
+def _seg_header(ws):
+    """The plan's header in the workspace (byte 128): unit counts of the two launches, the
+    number of cut sequences and each one's segment count."""
+    h = ws[128:176].view(torch.int32).cpu().numpy()
+    return {"n1": int(h[0]), "n3": int(h[1]), "nsplit": int(h[2]),
+            "m": [int(h[4 + 4 * i]) for i in range(2)]}
+
+
+def _run_cut(ops, w, inp, n_split, nseg, S0_alias=True):
+    d = to_device(inp)
+    N = len(w.seq_lens) if w.seq_lens is not None else w.B
+    ws = ops.new_workspace(w.B, w.T, w.H, 128, 128, 64,
+                           N if w.seq_lens is not None else 0, torch.device("cuda"))
+    S = d["S0"].clone() if S0_alias else None
+    ops.debug_segment_split(n_split, nseg)
+    try:
+        o, S = ops.chunk_fwd(d["q"], d["k"], d["v"], d["a"], d["b"], d["S0"], d["cu_seqlens"],
+                             chunk=64, signed_gate=w.signed_gate, o_dtype=torch.float32, S_T=S,
+                             workspace=ws)
+        torch.cuda.synchronize()
+    finally:
+        ops.debug_segment_split(0, 0)
+    assert ops.workspace_status(ws) == 0
+    return o, S, _seg_header(ws)
+
+
+@pytest.mark.parametrize("n_split,nseg", [(1, 3), (2, 4), (2, 8)])
+@pytest.mark.parametrize("sg", [0, 1])
+def test_tc_segments_forced(cuda_lib, n_split, nseg, sg):
+    """A packed batch whose one or two longest sequences are cut (test hook) into 3, 4 or 8
+    segments, the last one ragged, with empty and one-token sequences beside them and S_T
+    written over S0: every row of o and S_T matches the oracle, and the plan's header says
+    how many sequences were cut and into how many segments."""
+    lens = (1500, 0, 2333, 64, 700, 1)
+    base = synth.CKDA_SPREAD if sg else synth.KDA_STD
+    w = base.with_(B=1, H=3, seq_lens=lens, T=sum(lens), o_dtype="f32", s0=True)
+    inp = synth.make_prefill(w, seed=90 + nseg + sg)
+    o, S, hdr = _run_cut(cuda_lib, w, inp, n_split, nseg)
+    assert hdr["nsplit"] == n_split
+    for i, ln in enumerate(sorted(lens, reverse=True)[:n_split]):
+        ch = -(-ln // 64)
+        seg = -(-ch // nseg)
+        assert hdr["m"][i] == -(-ch // seg)
+    ro, rS = oracle_prefill(inp, sg)
+    close(o, ro, TOL_BF16, "o")
+    close(S, rS, TOL_BF16, "S_T")
+
+
+def test_tc_segments_fast_forgetting(cuda_lib):
+    """Cut sequences whose gates forget fast: units of both launches (segments from zero, from
+    the identity, from the chained states) are handed to the kernel with references."""
+    lens = (900, 1300, 50)
+    w = synth.KDA_FAST.with_(B=1, H=2, seq_lens=lens, T=sum(lens), o_dtype="f32", s0=True)
+    inp = synth.make_prefill(w, seed=95)
+    o, S, hdr = _run_cut(cuda_lib, w, inp, 2, 5)
+    assert hdr["nsplit"] == 2
+    ro, rS = oracle_prefill(inp, w.signed_gate)
+    close(o, ro, TOL_BF16, "o")
+    close(S, rS, TOL_BF16, "S_T")
+
+
+def test_tc_segments_chosen_by_cost(cuda_lib):
+    """One long sequence and few heads (B=1, T=16384, H=4: 4 walks of 256 chunks on 148 SMs):
+    the cost model cuts it by itself; without a workspace large enough for the plan the same
+    call runs uncut.  Both match the oracle."""
+    w = synth.KDA_STD.with_(B=1, T=16384, H=4, o_dtype="f32", s0=True)
+    inp = synth.make_prefill(w, seed=96)
+    o, S, hdr = _run_cut(cuda_lib, w, inp, 0, 0, S0_alias=False)
+    assert hdr["nsplit"] == 1 and hdr["m"][0] >= 3
+    ro, rS = oracle_prefill(inp, w.signed_gate)
+    close(o, ro, TOL_BF16, "o")
+    close(S, rS, TOL_BF16, "S_T")
+    d = to_device(inp)
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")   # the header alone: no plan
+    o2, S2 = cuda_lib.chunk_fwd(d["q"], d["k"], d["v"], d["a"], d["b"], d["S0"], None, chunk=64,
+                                signed_gate=w.signed_gate, o_dtype=torch.float32, workspace=ws)
+    torch.cuda.synchronize()
+    assert _seg_header(ws)["nsplit"] == 0 and _seg_header(ws)["n1"] == 0
+    close(o2, ro, TOL_BF16, "o uncut")
+    close(S2, rS, TOL_BF16, "S_T uncut")
 
 
 @pytest.mark.parametrize("signed_gate", [3, 4], ids=["gate_range", "strength_range"])

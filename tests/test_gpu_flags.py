@@ -99,6 +99,19 @@ def test_tensor_core_per_head_fast_decay(cuda_lib, flags):
     _fwd_check(cuda_lib, w, seed=32, flags=flags, tol=TOL_BF16)
 
 
+def test_tensor_core_segments_with_flags(cuda_lib):
+    """Both flags on a packed batch whose longest sequence is cut into four segments (test
+    hook): the segments from the identity (v = 0) normalise q and k and broadcast the gate
+    like every other unit."""
+    lens = (1400, 300, 0, 90)
+    w = synth.CKDA_SPREAD.with_(B=1, H=2, seq_lens=lens, T=sum(lens))
+    cuda_lib.debug_segment_split(1, 4)
+    try:
+        _fwd_check(cuda_lib, w, seed=33, flags=PH | L2, tol=TOL_BF16)
+    finally:
+        cuda_lib.debug_segment_split(0, 0)
+
+
 @pytest.mark.parametrize("flags", [PH, L2, PH | L2], ids=["per_head", "l2norm", "both"])
 @pytest.mark.parametrize("io", ["f32", "bf16"])
 def test_decode(cuda_lib, flags, io):
