@@ -211,8 +211,8 @@ int ckda_decode_step(const void *q, const void *k, const void *v, const void *a,
  * compiled into the library (every GPU that loads the library holds it until
  * the process exits).  The scratch holds the status header only, so chunks
  * whose gates decay past the tensor-core kernel's range run token by token
- * (no hand-off).  Neither this call nor the library calls cudaMalloc or
- * cudaFree.
+ * (no hand-off) and no sequence is cut into segments.  Neither this call nor
+ * the library calls cudaMalloc or cudaFree.
  *   - Every call looks up the scratch array's device address
  *     (cudaGetSymbolAddress) with the caller's device current, so the address
  *     is never stale.  The first call on a device may load the library's
