@@ -503,14 +503,16 @@ def test_tc_segments_fast_forgetting(cuda_lib):
     close(S, rS, TOL_BF16, "S_T")
 
 
-def test_tc_segments_chosen_by_cost(cuda_lib):
-    """One long sequence and few heads (B=1, T=16384, H=4: 4 walks of 256 chunks on 148 SMs):
-    the cost model cuts it by itself; without a workspace large enough for the plan the same
-    call runs uncut.  Both match the oracle."""
-    w = synth.KDA_STD.with_(B=1, T=16384, H=4, o_dtype="f32", s0=True)
-    inp = synth.make_prefill(w, seed=96)
+@pytest.mark.parametrize("B,T,H", [(1, 16384, 4), (2, 8192, 2)])
+def test_tc_segments_chosen_by_cost(cuda_lib, B, T, H):
+    """Few long sequences and few heads (4 walks of 256 chunks, or 4 of 128, on 148 SMs): the
+    cost model cuts every sequence by itself (unpacked rows, so each unit addresses its own
+    batch row); without a workspace large enough for the plan the same call runs uncut.  Both
+    match the oracle."""
+    w = synth.KDA_STD.with_(B=B, T=T, H=H, o_dtype="f32", s0=True)
+    inp = synth.make_prefill(w, seed=96 + B)
     o, S, hdr = _run_cut(cuda_lib, w, inp, 0, 0, S0_alias=False)
-    assert hdr["nsplit"] == 1 and hdr["m"][0] >= 3
+    assert hdr["nsplit"] == B and min(hdr["m"][:B]) >= 3
     ro, rS = oracle_prefill(inp, w.signed_gate)
     close(o, ro, TOL_BF16, "o")
     close(S, rS, TOL_BF16, "S_T")
