@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <math.h>
 #include <stddef.h>
 #include <stdint.h>
 
@@ -80,54 +81,85 @@ struct SegChoice {
   long est, est0;
   int w1, w3;   // waves of the cut sequences' units in the first and second launch
 };
-__host__ __device__ inline long seg_cdiv(long a, long b) { return (a + b - 1) / b; }
-__host__ __device__ inline SegChoice seg_choose(const int *top, int nv, long W, int H, int P,
-                                                int force_k, int force_m) {
+// Divisions by the SM count go through fp32 (an estimate; the same IEEE operations on the host
+// and the device, so both take the same decision) and chunk counts are 32-bit: 64-bit integer
+// division is a long software sequence on the device.
+__host__ __device__ inline long seg_per_sm(long work, int P) {
+  return (long)ceilf((float)work / (float)P);
+}
+// the estimated walk without a cut
+__host__ __device__ inline long seg_est0(const int *top, int nv, long W, int P) {
+  if (nv <= 0) return 0;
+  const long w = seg_per_sm(W, P);
+  return top[0] > w ? (long)top[0] : w;
+}
+// One candidate: the k longest sequences each cut into (up to) nseg segments.  Returns whether
+// it is possible (forced: whatever the length, but every cut sequence needs three segments).
+__host__ __device__ inline bool seg_candidate(const int *top, int nv, long W, int H, int P, int k,
+                                              int nseg, bool forced, long est0, SegChoice &c) {
+  c.k = k;
+  c.est0 = est0;
+  int U1 = 0, U3 = 0;
+  long extra = 0;
+  for (int i = 0; i < k; ++i) {
+    const int ch = top[i];
+    if (!forced && ch < kSegMinChunks) return false;
+    const int L = ch > 0 ? (ch + nseg - 1) / nseg : 1;
+    const int mm = (ch + L - 1) / L;
+    if (mm < 3) return false;
+    c.m[i] = mm;
+    c.seg[i] = L;
+    U1 += H * (2 * mm - 3);
+    U3 += H * (mm - 1);
+    extra += (long)H * L * (2 * mm - 4);
+  }
+  const long L0 = c.seg[0];
+  c.w1 = (U1 + P - 1) / P;
+  c.w3 = (U3 + P - 1) / P;
+  long chain = L0 * (c.w1 + c.w3);
+  if (k < nv) {
+    const long wsmall = c.w1 < c.w3 ? c.w1 : c.w3;
+    const long alt = L0 * wsmall + (long)top[k];
+    if (alt > chain) chain = alt;
+  }
+  const long work = seg_per_sm(W + extra, P);
+  c.est = chain > work ? chain : work;
+  return true;
+}
+constexpr int kSegCandidates = kSegMaxSplit * (kSegMaxSeg - 2);   // (k, nseg) pairs
+__host__ __device__ inline void seg_candidate_of(int idx, int &k, int &nseg) {
+  k = 1 + idx / (kSegMaxSeg - 2);
+  nseg = 3 + idx % (kSegMaxSeg - 2);
+}
+// The choice among evaluated candidates (valid[x]: candidate x is possible), in candidate order
+// (k, then nseg, ascending; the first of equal estimates): a cut costs two more launches and up
+// to twice the work of the cut sequences, so it is taken only for a clear gain (or when forced).
+__host__ __device__ inline SegChoice seg_pick(const SegChoice *cand, const bool *valid, long est0,
+                                              bool forced) {
   SegChoice best;
   best.k = 0;
   best.w1 = best.w3 = 0;
-  best.est0 = nv > 0 ? (top[0] > seg_cdiv(W, P) ? (long)top[0] : seg_cdiv(W, P)) : 0;
-  best.est = best.est0;
-  const int kmax = nv < kSegMaxSplit ? nv : kSegMaxSplit;
-  for (int k = 1; k <= kmax; ++k) {
-    for (int nseg = 3; nseg <= kSegMaxSeg; ++nseg) {
-      if (force_k > 0 && (k != force_k || nseg != force_m)) continue;
-      SegChoice c;
-      c.k = k;
-      long U1 = 0, U3 = 0, extra = 0;
-      bool ok = true;
-      for (int i = 0; i < k; ++i) {
-        const int ch = top[i];
-        if (force_k <= 0 && ch < kSegMinChunks) ok = false;
-        const int L = ch > 0 ? (int)seg_cdiv(ch, nseg) : 1;
-        const int mm = (int)seg_cdiv(ch, L);
-        if (mm < 3) ok = false;
-        c.m[i] = mm;
-        c.seg[i] = L;
-        U1 += (long)H * (2 * mm - 3);
-        U3 += (long)H * (mm - 1);
-        extra += (long)H * L * (2 * mm - 4);
-      }
-      if (!ok) continue;
-      const long L0 = c.seg[0];
-      c.w1 = (int)seg_cdiv(U1, P);
-      c.w3 = (int)seg_cdiv(U3, P);
-      long chain = L0 * (c.w1 + c.w3);
-      if (k < nv) {
-        const long wsmall = c.w1 < c.w3 ? c.w1 : c.w3;
-        const long alt = L0 * wsmall + (long)top[k];
-        if (alt > chain) chain = alt;
-      }
-      const long work = seg_cdiv(W + extra, P);
-      c.est = chain > work ? chain : work;
-      c.est0 = best.est0;
-      if (force_k > 0 || c.est < best.est) best = c;
-    }
-  }
-  // a cut costs two more launches and up to twice the work of the cut sequences: only for a
-  // clear gain
-  if (force_k <= 0 && best.k > 0 && best.est * 10 > best.est0 * 9) best.k = 0;
+  best.est = best.est0 = est0;
+  for (int x = 0; x < kSegCandidates; ++x)
+    if (valid[x] && (forced || cand[x].est < best.est)) best = cand[x];
+  if (!forced && best.k > 0 && best.est * 10 > est0 * 9) best.k = 0;
   return best;
+}
+// The whole cost model, one candidate after the other (the planner kernel evaluates them in
+// parallel).
+__host__ __device__ inline SegChoice seg_choose(const int *top, int nv, long W, int H, int P,
+                                                int force_k, int force_m) {
+  const long est0 = seg_est0(top, nv, W, P);
+  const bool forced = force_k > 0;
+  SegChoice cand[kSegCandidates];
+  bool valid[kSegCandidates];
+  for (int x = 0; x < kSegCandidates; ++x) {
+    int k, nseg;
+    seg_candidate_of(x, k, nseg);
+    valid[x] = k <= nv && (!forced || (k == force_k && nseg == force_m)) &&
+               seg_candidate(top, nv, W, H, P, k, nseg, forced, est0, cand[x]);
+  }
+  return seg_pick(cand, valid, est0, forced);
 }
 
 // Workspace of the tensor-core path: the header, the hand-off queue and saved states for

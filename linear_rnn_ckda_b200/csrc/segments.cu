@@ -35,7 +35,8 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
   __shared__ int s_ch[kSegMaxSeqs];      // chunks, by rank
   __shared__ unsigned long long s_W;
   __shared__ int s_nv, s_n1short;
-  __shared__ SegChoice s_c;
+  __shared__ SegChoice s_c, s_cand[kSegCandidates];
+  __shared__ bool s_valid[kSegCandidates];
   __shared__ long long s_cap1;
   const int tid = threadIdx.x;
   const bool packed = cu != nullptr;
@@ -75,11 +76,28 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
     atomicAdd(&s_W, (unsigned long long)ch * (unsigned long long)H);
   }
   __syncthreads();
+  // the cost model's candidates, one per thread
+  {
+    const int nv = s_nv;
+    int top[kSegMaxSplit + 1];
+    for (int i = 0; i <= kSegMaxSplit; ++i) top[i] = i < nv ? s_ch[i] : 0;
+    if (tid < kSegCandidates) {
+      const long est0 = seg_est0(top, nv, (long)s_W, P);
+      const bool forced = force_k > 0;
+      int k, nseg;
+      seg_candidate_of(tid, k, nseg);
+      SegChoice c;
+      s_valid[tid] = k <= nv && (!forced || (k == force_k && nseg == force_m)) &&
+                     seg_candidate(top, nv, (long)s_W, H, P, k, nseg, forced, est0, c);
+      s_cand[tid] = c;
+    }
+  }
+  __syncthreads();
   if (tid == 0) {
     const int nv = s_nv;
     int top[kSegMaxSplit + 1];
     for (int i = 0; i <= kSegMaxSplit; ++i) top[i] = i < nv ? s_ch[i] : 0;
-    SegChoice c = seg_choose(top, nv, (long)s_W, H, P, force_k, force_m);
+    const SegChoice c = seg_pick(s_cand, s_valid, seg_est0(top, nv, (long)s_W, P), force_k > 0);
     // the first launch's spare capacity (chunk times x SMs) for the uncut sequences: the two
     // launches split the estimated walk in proportion to the cut sequences' waves in each
     long long cap1 = 0x7FFFFFFFFFFFFFFFLL;
@@ -169,63 +187,70 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
   }
 }
 
-// The chain between the launches: CTA (cut sequence i, head h) forms X_s <- Y_s X_{s-1} + X_s for
-// s = 1 .. m-2 in fp32 (states [dk][dv] row-major; Y_s is [dk][dk]).  Thread (ty, tx) owns the
-// 8 x 8 block at rows 8 ty, columns 8 tx.  CTA 0 also clears the hand-off queue's count for the
-// second launch (the first launch's units with references have finished).
+// The chain between the launches: X_s <- Y_s X_{s-1} + X_s for s = 1 .. m-2 in fp32 (states
+// [dk][dv] row-major; Y_s is [dk][dk]).  Column blocks of X are independent through the whole
+// chain, so CTA (cut sequence i, head h, block cb) owns the 32 columns 32 cb .. 32 cb + 31 of
+// every X_s; thread (ty, tx) owns the 4 x 4 block at rows 4 ty, columns 4 tx of it.  CTA 0 also
+// clears the hand-off queue's count for the second launch (the first launch's units with
+// references have finished).
 constexpr int kCombThreads = 256;
-constexpr int kATStride = kD + 4;   // floats per row of A^T in shared memory
-constexpr size_t kCombSmem = (size_t)(kD * kATStride + kD * kD) * sizeof(float);
+constexpr int kCombCols = 32;                 // columns of X per CTA
+constexpr int kCombBlocks = kD / kCombCols;   // CTAs per (cut sequence, head)
+constexpr int kATStride = kD + 4;             // floats per row of A^T in shared memory
+constexpr size_t kCombSmem = (size_t)(kD * kATStride + kD * kCombCols) * sizeof(float);
 
 __global__ void __launch_bounds__(kCombThreads, 1)
     seg_combine_kernel(const SegHeader *hdr, float *slots, int *queue_count, int H) {
   extern __shared__ float4 comb_smem4[];
   float *sAT = reinterpret_cast<float *>(comb_smem4);   // [k][i] = A[i][k]
-  float *sS = sAT + kD * kATStride;                      // [k][j] = S_in[k][j]
+  float *sS = sAT + kD * kATStride;                      // [k][j] = S_in[k][32 cb + j]
   if (blockIdx.x == 0 && threadIdx.x == 0 && queue_count) *queue_count = 0;
-  const int i = blockIdx.x / H, h = blockIdx.x - (blockIdx.x / H) * H;
+  const int cb = blockIdx.x % kCombBlocks, ih = blockIdx.x / kCombBlocks;
+  const int i = ih / H, h = ih - (ih / H) * H;
   if (i >= hdr->nsplit) return;
   const SegSplit sp = hdr->split[i];
-  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  const int tid = threadIdx.x, ty = tid >> 3, tx = tid & 7;
   auto slot = [&](int j) { return slots + ((size_t)(sp.slot_base + j) * H + h) * kD * kD; };
   for (int s = 1; s <= sp.m - 2; ++s) {
     const float *A = slot(sp.m - 1 + s - 1);
-    const float *Sin = slot(s - 1);
-    float *X = slot(s);
+    const float *Sin = slot(s - 1) + kCombCols * cb;
+    float *X = slot(s) + kCombCols * cb;
     for (int e = tid; e < kD * kD; e += kCombThreads) {
       const int r = e >> 7, cc = e & (kD - 1);
       sAT[cc * kATStride + r] = A[e];
-      sS[e] = Sin[e];
+    }
+    for (int e = tid; e < kD * kCombCols; e += kCombThreads) {
+      const int r = e / kCombCols, cc = e % kCombCols;
+      sS[e] = Sin[(size_t)r * kD + cc];
     }
     __syncthreads();
-    float acc[8][8];
+    float acc[4][4];
 #pragma unroll
-    for (int r = 0; r < 8; ++r)
+    for (int r = 0; r < 4; ++r)
 #pragma unroll
-      for (int q = 0; q < 8; ++q) acc[r][q] = 0.f;
-#pragma unroll 2
+      for (int q = 0; q < 4; ++q) acc[r][q] = 0.f;
+#pragma unroll 4
     for (int kk = 0; kk < kD; ++kk) {
-      const float4 a0 = *reinterpret_cast<const float4 *>(sAT + kk * kATStride + 8 * ty);
-      const float4 a1 = *reinterpret_cast<const float4 *>(sAT + kk * kATStride + 8 * ty + 4);
-      const float4 b0 = *reinterpret_cast<const float4 *>(sS + kk * kD + 8 * tx);
-      const float4 b1 = *reinterpret_cast<const float4 *>(sS + kk * kD + 8 * tx + 4);
-      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+      const float4 a = *reinterpret_cast<const float4 *>(sAT + kk * kATStride + 4 * ty);
+      const float4 b = *reinterpret_cast<const float4 *>(sS + kk * kCombCols + 4 * tx);
+      const float av[4] = {a.x, a.y, a.z, a.w};
+      const float bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-      for (int r = 0; r < 8; ++r)
+      for (int r = 0; r < 4; ++r)
 #pragma unroll
-        for (int q = 0; q < 8; ++q) acc[r][q] = fmaf(av[r], bv[q], acc[r][q]);
+        for (int q = 0; q < 4; ++q) acc[r][q] = fmaf(av[r], bv[q], acc[r][q]);
     }
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      float *row = X + (size_t)(8 * ty + r) * kD + 8 * tx;
-      float4 x0 = *reinterpret_cast<float4 *>(row), x1 = *reinterpret_cast<float4 *>(row + 4);
-      x0.x += acc[r][0]; x0.y += acc[r][1]; x0.z += acc[r][2]; x0.w += acc[r][3];
-      x1.x += acc[r][4]; x1.y += acc[r][5]; x1.z += acc[r][6]; x1.w += acc[r][7];
-      *reinterpret_cast<float4 *>(row) = x0;
-      *reinterpret_cast<float4 *>(row + 4) = x1;
+    for (int r = 0; r < 4; ++r) {
+      float4 *row = reinterpret_cast<float4 *>(X + (size_t)(4 * ty + r) * kD + 4 * tx);
+      float4 x = *row;
+      x.x += acc[r][0];
+      x.y += acc[r][1];
+      x.z += acc[r][2];
+      x.w += acc[r][3];
+      *row = x;
     }
-    __syncthreads();   // X_s is the next step's S_in; the tiles are restaged
+    __syncthreads();   // this block of X_s is the next step's S_in block; the tiles are restaged
   }
 }
 
@@ -266,7 +291,8 @@ int launch_seg_combine(const SegHeader *hdr, float *slots, int *queue_count, int
   if (cudaFuncSetAttribute(seg_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)kCombSmem) != cudaSuccess)
     return CKDA_ERR_CUDA;
-  seg_combine_kernel<<<kSegMaxSplit * H, kCombThreads, kCombSmem, s>>>(hdr, slots, queue_count, H);
+  seg_combine_kernel<<<kSegMaxSplit * H * kCombBlocks, kCombThreads, kCombSmem, s>>>(
+      hdr, slots, queue_count, H);
   return cudaGetLastError() == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
 }
 
