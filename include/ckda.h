@@ -275,6 +275,18 @@ void ckda_debug_wait_injection(int chunk_index, unsigned long long wait_ns);
  */
 void ckda_debug_segment_split(int n_split, int n_segments);
 
+/*
+ * TEST HOOK: what the segment cut's cost model decides for a packed batch of
+ * n_seqs sequences of lengths[0 .. n_seqs) tokens with H heads on sm_count
+ * SMs (host arithmetic, no CUDA call; the device planner evaluates the same
+ * model).  *n_cut receives the number of sequences cut (0, 1 or 2: the
+ * longest ones), segments[0..1] how many segments each (0 past *n_cut).
+ * Returns CKDA_OK, CKDA_ERR_NULL or CKDA_ERR_DIM (n_seqs outside
+ * [0, 1024], H or sm_count not positive, a negative length).
+ */
+int ckda_debug_segment_choice(const int32_t *lengths, int n_seqs, int H, int sm_count,
+                              int *n_cut, int *segments);
+
 /* Static, human-readable text for a status code (never NULL). */
 const char *ckda_status_string(int status);
 

@@ -50,6 +50,25 @@ std::atomic<unsigned long long> g_inject_wait_ns{0};
 std::atomic<int> g_force_split{0};
 std::atomic<int> g_force_nseg{0};
 
+// The cost model's choice for a packed batch of these lengths (what the planner decides).
+ckda::SegChoice seg_choice_for_lengths(const int32_t *lengths, int n, int H, int P) {
+  // the planner's view: chunk counts in descending order, their sum over all heads
+  int top[ckda::kSegMaxSplit + 1] = {};
+  long W = 0;
+  for (int x = 0; x < n; ++x) {
+    const int ch = lengths[x] > 0 ? (lengths[x] + 63) / 64 : 0;   // chunks of 64 rows
+    W += (long)ch * H;
+    for (int i = 0; i <= ckda::kSegMaxSplit; ++i)
+      if (ch > top[i]) {
+        for (int j = ckda::kSegMaxSplit; j > i; --j) top[j] = top[j - 1];
+        top[i] = ch;
+        break;
+      }
+  }
+  return ckda::seg_choose(top, n, W, H, P, 0, 0);
+}
+
+
 }  // namespace
 
 namespace ckda {
@@ -82,6 +101,18 @@ extern "C" {
 void ckda_debug_wait_injection(int chunk_index, unsigned long long wait_ns) {
   g_inject_wait_ns.store(wait_ns, std::memory_order_relaxed);
   g_inject_chunk.store(chunk_index < 0 ? -1 : chunk_index, std::memory_order_relaxed);
+}
+
+int ckda_debug_segment_choice(const int32_t *lengths, int n_seqs, int H, int sm_count,
+                              int *n_cut, int *segments) {
+  if (!lengths || !n_cut || !segments) return CKDA_ERR_NULL;
+  if (n_seqs < 0 || n_seqs > ckda::kSegMaxSeqs || H <= 0 || sm_count <= 0) return CKDA_ERR_DIM;
+  for (int x = 0; x < n_seqs; ++x)
+    if (lengths[x] < 0) return CKDA_ERR_DIM;
+  const ckda::SegChoice c = seg_choice_for_lengths(lengths, n_seqs, H, sm_count);
+  *n_cut = c.k;
+  for (int i = 0; i < ckda::kSegMaxSplit; ++i) segments[i] = i < c.k ? c.m[i] : 0;
+  return CKDA_OK;
 }
 
 void ckda_debug_segment_split(int n_split, int n_segments) {

@@ -46,6 +46,8 @@ SIGNATURES = {
     "ckda_noalloc_status": (_i, [ctypes.POINTER(_i), _vp]),
     "ckda_debug_wait_injection": (None, [_i, ctypes.c_ulonglong]),
     "ckda_debug_segment_split": (None, [_i, _i]),
+    "ckda_debug_segment_choice": (_i, [ctypes.POINTER(ctypes.c_int32), _i, _i, _i,
+                                      ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),
     "ckda_status_string": (ctypes.c_char_p, [_i]),
     "ckda_version": (_i, []),
 }
@@ -291,6 +293,19 @@ def noalloc_status(device=None) -> int:
 def debug_wait_injection(chunk_index: int, wait_ns: int = 0) -> None:
     """Test hook: see ``ckda_debug_wait_injection`` in ``include/ckda.h`` (-1 switches it off)."""
     load().ckda_debug_wait_injection(int(chunk_index), int(wait_ns))
+
+
+def debug_segment_choice(lengths, H: int, sm_count: int = 148):
+    """Test hook: see ``ckda_debug_segment_choice`` in ``include/ckda.h``.  Returns
+    (sequences cut, [segments of each])."""
+    n = len(lengths)
+    arr = (ctypes.c_int32 * max(n, 1))(*[int(x) for x in lengths])
+    k = ctypes.c_int(0)
+    m = (ctypes.c_int * 2)()
+    rc = load().ckda_debug_segment_choice(arr, n, int(H), int(sm_count), ctypes.byref(k), m)
+    if rc != 0:
+        raise CkdaError("ckda_debug_segment_choice", rc)
+    return k.value, [m[i] for i in range(k.value)]
 
 
 def debug_segment_split(n_split: int, n_segments: int) -> None:

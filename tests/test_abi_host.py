@@ -272,3 +272,31 @@ def test_bwd_workspace_size(lib):
     assert lib.ckda_chunk_bwd_workspace_size(1, 4096, 16, 128, 128, 3) == 256 + (128 + 4) * per
     rec16 = (3 * 32 * 16 + 3 * 32 * 32 + 32 + 16 + 3) // 4 * 4
     assert lib.ckda_chunk_bwd_workspace_size(1, 32, 1, 16, 48, 0) == 256 + (2 * 16 * 48 + rec16) * 4
+
+
+def test_segment_cost_model(lib):
+    """The segment cut's cost model, which the device planner evaluates for packed batches
+    (ckda_debug_segment_choice runs it on the host).  The long-context varlen batch (16
+    sequences of 512..8192 tokens and one of 65,536, 32 heads) cuts the long one into three
+    segments (32 heads x 3 first-launch units fit one wave of 148 SMs; four segments would not);
+    one 65,536-token sequence over 16 heads is cut into six; two of 8,192 over 2 heads both
+    into eight.  Equal-length batches that already fill the GPU, batches whose total work
+    outweighs their longest walk, and sequences under 48 chunks are not cut."""
+    from linear_rnn_ckda_b200 import synth
+
+    assert ops.debug_segment_choice(synth.varlen_lengths(0), 32) == (1, [3])
+    assert ops.debug_segment_choice([65536], 16) == (1, [6])
+    assert ops.debug_segment_choice([8192, 8192], 2) == (2, [8, 8])
+    assert ops.debug_segment_choice([4096] * 4, 16) == (0, [])
+    assert ops.debug_segment_choice([8192] * 8, 16) == (0, [])
+    assert ops.debug_segment_choice([65536] + [8192] * 200, 32) == (0, [])
+    assert ops.debug_segment_choice([3008, 64, 64], 1) == (0, [])   # 47 chunks
+    assert ops.debug_segment_choice([3009, 64, 64], 1) == (1, [8])   # 48 chunks
+    assert ops.debug_segment_choice([], 4) == (0, [])
+    # half the SMs: six segments would need two waves in both launches (walk 4 x 171 chunks);
+    # five take two waves in the first launch only (3 x 205)
+    assert ops.debug_segment_choice([65536], 16, sm_count=74) == (1, [5])
+    with pytest.raises(ops.CkdaError):
+        ops.debug_segment_choice([100, -1], 4)
+    with pytest.raises(ops.CkdaError):
+        ops.debug_segment_choice([64] * 1025, 4)
