@@ -24,8 +24,8 @@ size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 // One CTA.  Thread x owns sequence x: its offsets are checked (a bad sequence records
 // CKDA_ERR_SEQLENS and gets no unit), it is ranked by length (descending, ties by index), and it
-// writes its own unit list entry; thread 0 runs the cost model and writes the cut sequences'
-// entries and the header.
+// writes its own unit list entry.  The first kSegCandidates threads evaluate one candidate cut
+// each; thread 0 picks one and writes the cut sequences' entries and the header.
 __global__ void __launch_bounds__(kPlanThreads, 1)
     seg_plan_kernel(const int32_t *cu, int n_seqs, int T, int H, int P, int force_k, int force_m,
                     SegHeader *hdr, SegDesc *d1, SegDesc *d3, int *status) {
@@ -86,7 +86,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
       const bool forced = force_k > 0;
       int k, nseg;
       seg_candidate_of(tid, k, nseg);
-      SegChoice c;
+      SegChoice c = {};
       s_valid[tid] = k <= nv && (!forced || (k == force_k && nseg == force_m)) &&
                      seg_candidate(top, nv, (long)s_W, H, P, k, nseg, forced, est0, c);
       s_cand[tid] = c;
