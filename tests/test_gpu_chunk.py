@@ -490,6 +490,27 @@ def test_tc_segments_forced(cuda_lib, n_split, nseg, sg):
     close(S, rS, TOL_BF16, "S_T")
 
 
+def test_tc_segments_without_states(cuda_lib):
+    """A cut packed batch with no S0 (segment 0 starts from zero) and no S_T requested (the
+    last segment writes no end state): o matches the oracle row for row."""
+    lens = (2000, 333, 64)
+    w = synth.KDA_STD.with_(B=1, H=2, seq_lens=lens, T=sum(lens), o_dtype="bf16", s0=False)
+    inp = synth.make_prefill(w, seed=97)
+    d = to_device(inp)
+    ws = cuda_lib.new_workspace(1, w.T, w.H, 128, 128, 64, len(lens), torch.device("cuda"))
+    cuda_lib.debug_segment_split(1, 5)
+    try:
+        o, S = cuda_lib.chunk_fwd(d["q"], d["k"], d["v"], d["a"], d["b"], None, d["cu_seqlens"],
+                                  chunk=64, signed_gate=0, workspace=ws, want_state=False)
+        torch.cuda.synchronize()
+    finally:
+        cuda_lib.debug_segment_split(0, 0)
+    assert S is None and cuda_lib.workspace_status(ws) == 0
+    assert _seg_header(ws)["nsplit"] == 1 and _seg_header(ws)["m"][0] == 5
+    ro, _ = oracle_prefill(inp, 0)
+    close(o, ro, TOL_BF16, "o")
+
+
 def test_tc_segments_fast_forgetting(cuda_lib):
     """Cut sequences whose gates forget fast: units of both launches (segments from zero, from
     the identity, from the chained states) are handed to the kernel with references."""
