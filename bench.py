@@ -337,6 +337,19 @@ class PrefillCase:
         if st != 0:
             raise RuntimeError(f"device status {st} after {what}")
 
+    def plan(self):
+        """What the unit planner decided in the last call (the plan's header at byte 128 of the
+        workspace: units of the two launches per head, sequences cut, segments of each), or
+        None for an unplanned call (unpacked without a cut: the header stays zero)."""
+        if self.ws.numel() < 176:
+            return None
+        h = self.ws[128:176].view(torch.int32).cpu().tolist()
+        n1, n3, nsplit = h[0], h[1], h[2]
+        if n1 == 0 and n3 == 0:
+            return None
+        return {"cut_sequences": nsplit, "segments": [h[4 + 4 * i] for i in range(nsplit)],
+                "first_launch_units": n1 * self.w.H, "second_launch_units": n3 * self.w.H}
+
 
 def prefill_roofline(w, ms_launch, peaks, traffic_key):
     byts = prefill_bytes(w)
@@ -390,7 +403,7 @@ def main():
     run_head = "varlen" in legs
     tokens = w.tokens * world
     ms = ms_step = value = float("nan")
-    roofline = None
+    roofline = head_plan = None
     host = case = None
     clk = ClockSampler(local)
     if run_head:
@@ -400,6 +413,7 @@ def main():
             ms = time_loop(case, args.steps, args.warmup, world, stream)
         ms = max_over_ranks(ms, world)
         case.check("the headline leg")
+        head_plan = case.plan()
         ms_step = ms / args.steps
         value = tokens * args.steps / (ms / 1000.0)
         # dominant kernel: the chunk kernel.  A packed step is six launches (the 256-byte status
@@ -585,7 +599,7 @@ def main():
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded; same shapes and distributions as the pages' workloads)",
             "config": headline_config(w),
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "plan": head_plan,
             "workloads": workloads, "fwd_bwd": fwd_bwd, "decode": decode_obj,
             "gpu_launches": (6 if w.seq_lens is not None else 2) * args.steps, "clocks": clocks, "peaks_source": peaks["source"],
         }
